@@ -1,0 +1,197 @@
+/*
+ * cider.h -- C ABI of the B200 (sm_100a) W8A8 / W4A8 activation-quantized linear.
+ *
+ * The operation (sources: juejin post "在Mac上跑大模型，MLX 不是终点", sections
+ * "W8A8 对称量化：Cider 的选择", "INT8 TensorOps 内核设计", "三种量化粒度的实现";
+ * Cider README (WeHub translation), tables "模式" and "量化", sections
+ * "Metal Kernel 流水线" and "底层 API"):
+ *
+ *   per token m:   scale_x[m] = max_k |x[m,k]| / 127                 (fp32)
+ *                  q[m,k]     = clamp(round(x[m,k] / scale_x[m]), -128, 127)
+ *   per-channel:   y[m,n] = (sum_k q[m,k] * w[n,k]) * scale_x[m] * scale_w[n]
+ *   per-group:     y[m,n] = scale_x[m] * sum_g (sum_{k in g} q[m,k] * w[n,k]) * scale_w[g][n]
+ *   W4A8:          w[n,k] = nibble(n,k) - 8, nibbles packed two per byte
+ *
+ * round() is round-half-away-from-zero; x / scale_x is one correctly rounded
+ * fp32 division; an all-zero token has scale 0 and q = 0.  Products are
+ * summed exactly in INT32.  The output is fp16 or bf16, round to nearest even.
+ *
+ * Conventions shared by every entry point below:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or synchronises on these calls.  Each call is
+ *    enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream)
+ *    and returns as soon as its kernels are launched.
+ *  - Layouts are dense row-major: x [M][K], w [N][K] (nn.Linear convention:
+ *    output channel n, input channel k), y [M][N], q [M][K].  Per-group weight
+ *    scales are GROUP-MAJOR, scale_w[K/gs][N], so that one group's scales for
+ *    consecutive output channels are contiguous.  Packed INT4 weights are
+ *    [N][K/2] bytes; byte j of row n holds k = 2j in its low nibble and
+ *    k = 2j+1 in its high nibble, each as the offset-binary value q + 8.
+ *  - Argument checks happen before any launch.  A call that fails them
+ *    returns CIDER_ERR_INVALID_ARG and launches nothing; cider_last_error()
+ *    then names the failed check.  Requirements: M >= 0 (M == 0 is a no-op),
+ *    N, K >= 1; K % 16 == 0; N % 8 == 0; K <= 131072; tensor pointers and
+ *    scale_w 16-byte aligned and non-NULL (scale_x 4-byte aligned); per-group
+ *    gs is 64 or 128 and divides K; W4A8 also needs K % 32 == 0; y must not
+ *    overlap any input or the workspace (checked by address range).
+ *  - On a device that is not compute capability 10.x the calls return
+ *    CIDER_ERR_UNSUPPORTED; there is no CPU fallback.
+ *  - Launch failures return CIDER_ERR_CUDA.  Faults that happen later on the
+ *    device surface at the caller's next synchronisation, as usual in CUDA.
+ *  - Every wait inside the kernels is bounded in time.  A wait that runs out
+ *    records CIDER_ERR_TIMEOUT in a device status word, which
+ *    cider_device_status() reads back.
+ */
+#ifndef CIDER_H
+#define CIDER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CIDER_API __attribute__((visibility("default")))
+#else
+#define CIDER_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CIDER_OK = 0,
+    CIDER_ERR_INVALID_ARG = 1, /* an argument check failed; nothing was launched */
+    CIDER_ERR_UNSUPPORTED = 2, /* the current device is not sm_100-family */
+    CIDER_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
+    CIDER_ERR_TIMEOUT = 4      /* a bounded device-side wait ran out */
+} cider_status_t;
+
+typedef enum {
+    CIDER_F16 = 0,  /* IEEE binary16 */
+    CIDER_BF16 = 1  /* bfloat16 */
+} cider_dtype_t;
+
+/* ---- availability and diagnostics ------------------------------------- */
+
+/* 1 iff the calling thread's current CUDA device is compute capability 10.x
+ * (the hardware this library is built for), else 0.  Mirrors the pages'
+ * is_available() (Cider README, section "条件编译（M4 / M5）"). */
+CIDER_API int cider_is_available(void);
+
+/* Static, NUL-terminated description of a status code. */
+CIDER_API const char* cider_status_string(cider_status_t status);
+
+/* Message of the last failing call on this host thread ("" if none).  The
+ * string stays valid until the next call on the same thread. */
+CIDER_API const char* cider_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device: CIDER_OK, or CIDER_ERR_TIMEOUT if a bounded wait in some
+ * kernel ran out since the last read.  Not for the hot path. */
+CIDER_API cider_status_t cider_device_status(void* stream);
+
+/* Bytes of workspace the linear entry points need for M tokens of K inputs:
+ * the quantized activations q [M][K] int8 and scale_x [M] fp32, each start
+ * 256-byte aligned.  0 when M is small enough for the fused small-M kernel
+ * (M <= cider_get_small_m_threshold()), which keeps q in shared memory. */
+CIDER_API size_t cider_workspace_bytes(int64_t M, int64_t K);
+
+/* Calls with 1 <= M <= threshold use the fused small-M (decode-shaped) kernel;
+ * larger M use quantize + the tcgen05 GEMM.  The threshold is process-wide;
+ * 0 sends every call to the GEMM path.  Values above 16 are rejected.  The
+ * pages pick a dedicated matrix-vector kernel for single-token decode (juejin
+ * post, section "INT8 TensorOps 内核设计", "双路径自动切换"). */
+CIDER_API cider_status_t cider_set_small_m_threshold(int64_t threshold);
+CIDER_API int64_t cider_get_small_m_threshold(void);
+
+/* ---- the four operations of the pages' interface ----------------------- */
+
+/* Online per-token activation quantization (Cider README, section
+ * "Metal Kernel 流水线", step quantize_per_token; juejin post, section
+ * "W8A8 对称量化：Cider 的选择").
+ * x: [M][K] fp16/bf16 (xdt); q: [M][K] int8 out; scale_x: [M] fp32 out. */
+CIDER_API cider_status_t cider_quantize_act(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
+                                  int8_t* q, float* scale_x, void* stream);
+
+/* W8A8 linear, per-output-channel weight scales (Cider README, section
+ * "底层 API" perchannel_linear; table "W8A8 量化粒度", Per-channel).
+ * w: [N][K] int8; scale_w: [N] fp32; y: [M][N] (ydt).
+ * workspace: device buffer of at least cider_workspace_bytes(M, K) bytes
+ * (NULL allowed when that is 0); its contents on return are unspecified. */
+CIDER_API cider_status_t cider_w8a8_linear_pc(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
+                                    const int8_t* w, const float* scale_w, int64_t N,
+                                    void* y, cider_dtype_t ydt,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* W8A8 linear, per-group weight scales along K (gs = 64 or 128; Cider README,
+ * table "W8A8 量化粒度"; juejin post, section "三种量化粒度的实现").
+ * scale_w: [K/gs][N] fp32 (group-major).  The INT32 partial sum of each group
+ * is rescaled by its scale in fp32 and the rescaled partials are summed. */
+CIDER_API cider_status_t cider_w8a8_linear_pg(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
+                                    const int8_t* w, const float* scale_w, int64_t N, int64_t gs,
+                                    void* y, cider_dtype_t ydt,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* W4A8 linear, per-group scales (Cider README, table "模式" W4A8, section
+ * "Metal Kernel 流水线" (INT4 -> INT8 unpack in the load path), section
+ * "底层 API" w4a8_linear).  w_packed: [N][K/2] bytes as described above;
+ * scale_w: [K/gs][N] fp32. */
+CIDER_API cider_status_t cider_w4a8_linear_pg(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
+                                    const uint8_t* w_packed, const float* scale_w, int64_t N,
+                                    int64_t gs, void* y, cider_dtype_t ydt,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- the GEMM stage on pre-quantized activations ------------------------ */
+/* The same products and epilogues as the linears above, fed q [M][K] int8 and
+ * scale_x [M] fp32 from cider_quantize_act or a fused producer.  Always the
+ * tcgen05 tensor-core path. */
+CIDER_API cider_status_t cider_w8a8_gemm_pc_q(const int8_t* q, const float* scale_x, int64_t M, int64_t K,
+                                    const int8_t* w, const float* scale_w, int64_t N,
+                                    void* y, cider_dtype_t ydt, void* stream);
+CIDER_API cider_status_t cider_w8a8_gemm_pg_q(const int8_t* q, const float* scale_x, int64_t M, int64_t K,
+                                    const int8_t* w, const float* scale_w, int64_t N, int64_t gs,
+                                    void* y, cider_dtype_t ydt, void* stream);
+CIDER_API cider_status_t cider_w4a8_gemm_pg_q(const int8_t* q, const float* scale_x, int64_t M, int64_t K,
+                                    const uint8_t* w_packed, const float* scale_w, int64_t N,
+                                    int64_t gs, void* y, cider_dtype_t ydt, void* stream);
+
+/* ---- decoder-MLP producer ------------------------------------------------ */
+/* a = round_dt(silu(gate) * up) evaluated in fp32, then per-token quantized as
+ * cider_quantize_act does, in one pass: the input of a down projection that
+ * follows SiLU(gate) * up.  gate, up: [M][F] (dt); q: [M][F] int8 out;
+ * scale_x: [M] fp32 out; a_out: optional [M][F] (dt) copy of a (NULL = skip).
+ * Requires F % 16 == 0. */
+CIDER_API cider_status_t cider_silu_mul_quantize(const void* gate, const void* up, cider_dtype_t dt,
+                                       int64_t M, int64_t F, int8_t* q, float* scale_x,
+                                       void* a_out, void* stream);
+
+/* ---- offline weight quantization (Cider README, section "底层 API":
+ * quantize_weight_int8, pack_weight_int4) -------------------------------- */
+/* W: [N][K] fp32.  Per channel: scale_w[n] = max_k |W[n,k]| / 127,
+ * w = clamp(round(W / scale_w), -128, 127). */
+CIDER_API cider_status_t cider_quantize_weight_pc(const float* W, int64_t N, int64_t K,
+                                        int8_t* w, float* scale_w, void* stream);
+/* Per group of gs along K: scale_w[g][n] = max |W[n, g*gs:(g+1)*gs]| / 127 (group-major). */
+CIDER_API cider_status_t cider_quantize_weight_pg(const float* W, int64_t N, int64_t K, int64_t gs,
+                                        int8_t* w, float* scale_w, void* stream);
+/* INT4 per group: scale_w[g][n] = max|W_group| / 7, q = clamp(round(W/scale), -8, 7),
+ * packed as described above. */
+CIDER_API cider_status_t cider_pack_weight_int4_pg(const float* W, int64_t N, int64_t K, int64_t gs,
+                                         uint8_t* w_packed, float* scale_w, void* stream);
+
+/* ---- test exports (stable, but not part of the operation's interface) ---- */
+/* The tcgen05 GEMM with an INT32 store epilogue: acc[m][n] = sum_k q[m,k]*w[n,k]. */
+CIDER_API cider_status_t cider_test_gemm_i32(const int8_t* q, const int8_t* w, int64_t M, int64_t N,
+                                   int64_t K, int32_t* acc, void* stream);
+/* Per-group INT32 partials acc_g[g][m][n] = sum_{k in group g} q[m,k]*w[n,k]. */
+CIDER_API cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8_t* w, int64_t M, int64_t N,
+                                           int64_t K, int64_t gs, int32_t* acc_g, void* stream);
+/* The W4A8 load path's unpack: w[n][k] = nibble(n, k) - 8. */
+CIDER_API cider_status_t cider_test_unpack_int4(const uint8_t* w_packed, int64_t N, int64_t K, int8_t* w,
+                                      void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CIDER_H */

@@ -1,0 +1,106 @@
+"""CPU-side checks of the C-ABI boundary: the library builds and loads, exports
+every entry point that include/cider.h declares, and rejects bad arguments on
+the host before touching a device (so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w8a8_activation_quantized_b200 as cider
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "cider.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"CIDER_API[^;]*?\b(cider_\w+)\s*\(", text, flags=re.S)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w8a8_activation_quantized_b200._build import build_library
+    build_library()
+    return cider.lib()
+
+
+def test_header_declares_the_four_operations():
+    names = _declared()
+    for op in ("cider_quantize_act", "cider_w8a8_linear_pc", "cider_w8a8_linear_pg", "cider_w4a8_linear_pg"):
+        assert op in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in cider.h but not exported"
+    assert sorted(cider.EXPORTS) == names  # the binding covers exactly the header
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.cider_status_string(s)
+
+
+P = ctypes.c_void_p(256)  # a 16-byte aligned, never dereferenced address
+
+
+def _lin_pc(lib, **kw):
+    a = dict(x=P, xdt=0, M=4, K=64, w=ctypes.c_void_p(4096), sw=ctypes.c_void_p(8192), N=16,
+             y=ctypes.c_void_p(1 << 20), ydt=0, ws=None, wsb=0, st=None)
+    a.update(kw)
+    return lib.cider_w8a8_linear_pc(a["x"], a["xdt"], a["M"], a["K"], a["w"], a["sw"], a["N"], a["y"],
+                                    a["ydt"], a["ws"], a["wsb"], a["st"])
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(K=40), "K % 16"),
+    (dict(N=12), "N % 8"),
+    (dict(M=-1), "M < 0"),
+    (dict(K=0), "K < 1"),
+    (dict(K=131072 + 16), "K too large"),
+    (dict(xdt=7), "dtype"),
+    (dict(x=None), "NULL"),
+    (dict(x=ctypes.c_void_p(258)), "misaligned"),
+    (dict(y=ctypes.c_void_p(256 + 64)), "y overlaps x"),
+])
+def test_invalid_arguments_rejected_on_host(lib, kw, why):
+    assert _lin_pc(lib, **kw) == 1, why
+    assert lib.cider_last_error()
+
+
+def test_empty_input_is_a_noop(lib):
+    assert _lin_pc(lib, M=0) == 0
+
+
+def test_group_size_checks(lib):
+    f = lib.cider_w8a8_linear_pg
+    base = (P, 0, 4, 256, ctypes.c_void_p(4096), ctypes.c_void_p(8192), 16)
+    assert f(*base, 32, ctypes.c_void_p(1 << 20), 0, None, 0, None) == 1       # gs not 64/128
+    assert f(P, 0, 4, 192, ctypes.c_void_p(4096), ctypes.c_void_p(8192), 16, 128,
+             ctypes.c_void_p(1 << 20), 0, None, 0, None) == 1                   # gs does not divide K
+    g = lib.cider_w4a8_linear_pg
+    assert g(P, 0, 4, 192, ctypes.c_void_p(4096), ctypes.c_void_p(8192), 16, 128,
+             ctypes.c_void_p(1 << 20), 0, None, 0, None) == 1                   # gs does not divide K
+    assert lib.cider_set_small_m_threshold(17) == 1
+    assert lib.cider_set_small_m_threshold(-1) == 1
+
+
+def test_workspace_size(lib):
+    thr = lib.cider_get_small_m_threshold()
+    assert lib.cider_workspace_bytes(1, 2560) == 0 if thr >= 1 else True
+    M, K = 4096, 2560
+    assert lib.cider_workspace_bytes(M, K) == M * K + ((M * 4 + 255) // 256) * 256
+    assert lib.cider_workspace_bytes(0, 64) == 0
+
+
+def test_no_device_means_unsupported_or_cuda_error(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert lib.cider_is_available() == 0
+    # valid arguments, no device: the call must fail loudly, never compute on the CPU
+    st = _lin_pc(lib)
+    assert st in (2, 3)

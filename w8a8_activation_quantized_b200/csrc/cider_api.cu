@@ -1,0 +1,444 @@
+// cider_api.cu -- the extern "C" entry points declared in include/cider.h:
+// argument checks, device checks, path selection and launches.  No entry
+// point allocates, frees or synchronises (cider_device_status excepted).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/cider.h"
+#include "cider_kernels.h"
+
+namespace cider {
+
+// Device status word: bit 0 = a bounded wait ran out (kStatusTimeout).
+__device__ unsigned g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxK = 131072;            // 127 * 128 * K < 2^31 keeps INT32 exact
+constexpr int64_t kMaxSmallM = 16;
+constexpr int64_t kSmallSmemLimit = 160 * 1024;  // q rows of the small-M kernel in shared memory
+
+struct DeviceInfo {
+    int ready = 0;     // 1 = filled in
+    int cc_major = 0;
+    int num_sms = 0;
+    unsigned* status = nullptr;  // device address of g_status_word on this device
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+std::atomic<int64_t> g_small_m_threshold{4};
+thread_local char t_last_error[512] = "";
+
+cider_status_t fail(cider_status_t s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_last_error, sizeof t_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+cider_status_t cuda_fail(cudaError_t e, const char* what) {
+    return fail(CIDER_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Fills in (once per device, with that device current) the compute
+// capability, SM count and the device address of the status word.
+cider_status_t device_info(DeviceInfo** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(CIDER_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    DeviceInfo& d = g_dev[dev];
+    if (!__atomic_load_n(&d.ready, __ATOMIC_ACQUIRE)) {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        if (!d.ready) {
+            int major = 0, sms = 0;
+            if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+                return cuda_fail(e, "cudaDeviceGetAttribute");
+            if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+                return cuda_fail(e, "cudaDeviceGetAttribute");
+            void* addr = nullptr;
+            if (major == 10) {
+                if ((e = cudaGetSymbolAddress(&addr, g_status_word)) != cudaSuccess)
+                    return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+            }
+            d.cc_major = major;
+            d.num_sms = sms;
+            d.status = static_cast<unsigned*>(addr);
+            __atomic_store_n(&d.ready, 1, __ATOMIC_RELEASE);
+        }
+    }
+    if (d.cc_major != 10)
+        return fail(CIDER_ERR_UNSUPPORTED, "device %d is compute capability %d.x; this library needs 10.x (sm_100a)",
+                    dev, d.cc_major);
+    *out = &d;
+    return CIDER_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+    uintptr_t lo, hi;
+};
+Range rng(const void* p, size_t bytes) {
+    uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return {a, a + bytes};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+bool small_m_path(int64_t M, int64_t K) {
+    return M >= 1 && M <= g_small_m_threshold.load() && M * K <= kSmallSmemLimit;
+}
+
+// Common checks of the linear / GEMM entry points.
+cider_status_t check_common(const void* x, int64_t M, int64_t K, const void* w, const float* sw,
+                            int64_t N, const void* y, int dt_in, int dt_out) {
+    if (M < 0) return fail(CIDER_ERR_INVALID_ARG, "M = %lld must be >= 0", (long long)M);
+    if (N < 1 || K < 1) return fail(CIDER_ERR_INVALID_ARG, "N = %lld and K = %lld must be >= 1", (long long)N, (long long)K);
+    if (K % 16) return fail(CIDER_ERR_INVALID_ARG, "K = %lld must be a multiple of 16", (long long)K);
+    if (N % 8) return fail(CIDER_ERR_INVALID_ARG, "N = %lld must be a multiple of 8", (long long)N);
+    if (K > kMaxK) return fail(CIDER_ERR_INVALID_ARG, "K = %lld exceeds %lld", (long long)K, (long long)kMaxK);
+    if (M > INT32_MAX || N > INT32_MAX) return fail(CIDER_ERR_INVALID_ARG, "M and N must be < 2^31");
+    if (dt_in != CIDER_F16 && dt_in != CIDER_BF16) return fail(CIDER_ERR_INVALID_ARG, "input dtype %d unknown", dt_in);
+    if (dt_out != CIDER_F16 && dt_out != CIDER_BF16) return fail(CIDER_ERR_INVALID_ARG, "output dtype %d unknown", dt_out);
+    if (M == 0) return CIDER_OK;
+    if (!x || !w || !sw || !y) return fail(CIDER_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(x) || !aligned16(w) || !aligned16(sw) || !aligned16(y))
+        return fail(CIDER_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    return CIDER_OK;
+}
+
+cider_status_t check_gs(int64_t K, int64_t gs, bool w4) {
+    if (gs != 64 && gs != 128) return fail(CIDER_ERR_INVALID_ARG, "gs = %lld must be 64 or 128", (long long)gs);
+    if (K % gs) return fail(CIDER_ERR_INVALID_ARG, "gs = %lld must divide K = %lld", (long long)gs, (long long)K);
+    if (w4 && K % 32) return fail(CIDER_ERR_INVALID_ARG, "W4A8 needs K %% 32 == 0 (K = %lld)", (long long)K);
+    return CIDER_OK;
+}
+
+int pick_bn(int64_t M, int64_t N, int num_sms) {
+    const int64_t tiles256 = ((M + 127) / 128) * ((N + 255) / 256);
+    return tiles256 < num_sms ? 128 : 256;
+}
+
+cider_status_t run_gemm(int mode, const int8_t* q, const float* sx, int64_t M, int64_t K,
+                        const void* w, const float* sw, int64_t N, int64_t gs, void* y, int ydt,
+                        const DeviceInfo* d, cudaStream_t st) {
+    GemmLaunch L;
+    L.mode = mode;
+    L.q = q;
+    L.w = w;
+    L.sx = sx;
+    L.sw = sw;
+    L.y = y;
+    L.M = static_cast<int>(M);
+    L.N = static_cast<int>(N);
+    L.K = static_cast<int>(K);
+    L.gs = static_cast<int>(gs);
+    L.ydt = ydt;
+    L.bn = (mode == kModePC || mode == kModeI32) ? pick_bn(M, N, d->num_sms) : 128;
+    L.num_sms = d->num_sms;
+    L.status = d->status;
+    cudaError_t e = launch_gemm(L, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tcgen05 GEMM launch");
+    return CIDER_OK;
+}
+
+// The three linears share this body: quantize + tensor-core GEMM, or the
+// fused small-M kernel.
+cider_status_t linear(int mode, const void* x, int xdt, int64_t M, int64_t K, const void* w,
+                      const float* sw, int64_t N, int64_t gs, void* y, int ydt, void* ws,
+                      size_t ws_bytes, void* stream) {
+    t_last_error[0] = '\0';
+    cider_status_t s = check_common(x, M, K, w, sw, N, y, xdt, ydt);
+    if (s != CIDER_OK) return s;
+    if (mode != kModePC && (s = check_gs(K, gs, mode == kModeW4)) != CIDER_OK) return s;
+    if (M == 0) return CIDER_OK;
+    const size_t ysz = static_cast<size_t>(M) * N * 2;
+    const size_t wbytes = mode == kModeW4 ? static_cast<size_t>(N) * K / 2 : static_cast<size_t>(N) * K;
+    const size_t swbytes = mode == kModePC ? N * 4 : static_cast<size_t>(K / gs) * N * 4;
+    const Range ry = rng(y, ysz);
+    if (overlap(ry, rng(x, static_cast<size_t>(M) * K * 2)) || overlap(ry, rng(w, wbytes)) ||
+        overlap(ry, rng(sw, swbytes)))
+        return fail(CIDER_ERR_INVALID_ARG, "y overlaps an input");
+    DeviceInfo* d = nullptr;
+    if ((s = device_info(&d)) != CIDER_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (small_m_path(M, K)) {
+        cudaError_t e = launch_small_m(mode, x, xdt, static_cast<int>(M), static_cast<int>(K), w, sw,
+                                       static_cast<int>(N), static_cast<int>(gs), y, ydt, d->num_sms, st);
+        if (e != cudaSuccess) return cuda_fail(e, "small-M kernel launch");
+        return CIDER_OK;
+    }
+    const size_t need = cider_workspace_bytes(M, K);
+    if (!ws || ws_bytes < need)
+        return fail(CIDER_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, ws ? ws_bytes : 0);
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(CIDER_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (overlap(ry, rng(ws, need))) return fail(CIDER_ERR_INVALID_ARG, "y overlaps the workspace");
+    int8_t* q = static_cast<int8_t*>(ws);
+    float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(static_cast<size_t>(M) * K));
+    cudaError_t e = launch_quantize_act(x, xdt, M, static_cast<int>(K), q, sx, st);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+    return run_gemm(mode, q, sx, M, K, w, sw, N, gs, y, ydt, d, st);
+}
+
+cider_status_t gemm_q(int mode, const int8_t* q, const float* sx, int64_t M, int64_t K, const void* w,
+                      const float* sw, int64_t N, int64_t gs, void* y, int ydt, void* stream) {
+    t_last_error[0] = '\0';
+    cider_status_t s = check_common(q, M, K, w, sw, N, y, CIDER_F16, ydt);
+    if (s != CIDER_OK) return s;
+    if (mode != kModePC && (s = check_gs(K, gs, mode == kModeW4)) != CIDER_OK) return s;
+    if (M == 0) return CIDER_OK;
+    if (!sx || (reinterpret_cast<uintptr_t>(sx) & 3u)) return fail(CIDER_ERR_INVALID_ARG, "scale_x must be non-NULL and 4-byte aligned");
+    const Range ry = rng(y, static_cast<size_t>(M) * N * 2);
+    if (overlap(ry, rng(q, static_cast<size_t>(M) * K)) || overlap(ry, rng(sx, M * 4)))
+        return fail(CIDER_ERR_INVALID_ARG, "y overlaps an input");
+    DeviceInfo* d = nullptr;
+    if ((s = device_info(&d)) != CIDER_OK) return s;
+    return run_gemm(mode, q, sx, M, K, w, sw, N, gs, y, ydt, d, static_cast<cudaStream_t>(stream));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+}  // namespace
+
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t rank, void* base,
+                       const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                       const cuuint32_t* elem_strides, CUtensorMapSwizzle swizzle) {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode) return false;
+    return g_encode(map, dtype, rank, base, dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace cider
+
+using namespace cider;
+
+extern "C" {
+
+int cider_is_available(void) {
+    int dev = -1, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return major == 10 ? 1 : 0;
+}
+
+const char* cider_status_string(cider_status_t s) {
+    switch (s) {
+        case CIDER_OK: return "ok";
+        case CIDER_ERR_INVALID_ARG: return "invalid argument";
+        case CIDER_ERR_UNSUPPORTED: return "unsupported device (needs compute capability 10.x)";
+        case CIDER_ERR_CUDA: return "CUDA error";
+        case CIDER_ERR_TIMEOUT: return "a bounded device wait ran out";
+    }
+    return "unknown status";
+}
+
+const char* cider_last_error(void) { return t_last_error; }
+
+cider_status_t cider_device_status(void* stream) {
+    t_last_error[0] = '\0';
+    DeviceInfo* d = nullptr;
+    cider_status_t s = device_info(&d);
+    if (s != CIDER_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned v = 0;
+    if ((e = cudaMemcpy(&v, d->status, sizeof v, cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "reading the status word");
+    if (v != 0) {
+        unsigned zero = 0;
+        if ((e = cudaMemcpy(d->status, &zero, sizeof zero, cudaMemcpyHostToDevice)) != cudaSuccess)
+            return cuda_fail(e, "clearing the status word");
+        if (v & kStatusTimeout) return fail(CIDER_ERR_TIMEOUT, "a bounded device-side wait ran out");
+    }
+    return CIDER_OK;
+}
+
+size_t cider_workspace_bytes(int64_t M, int64_t K) {
+    if (M <= 0 || K <= 0 || small_m_path(M, K)) return 0;
+    return align256(static_cast<size_t>(M) * K) + align256(static_cast<size_t>(M) * 4);
+}
+
+cider_status_t cider_set_small_m_threshold(int64_t threshold) {
+    if (threshold < 0 || threshold > kMaxSmallM)
+        return fail(CIDER_ERR_INVALID_ARG, "threshold %lld outside [0, %lld]", (long long)threshold, (long long)kMaxSmallM);
+    g_small_m_threshold.store(threshold);
+    return CIDER_OK;
+}
+
+int64_t cider_get_small_m_threshold(void) { return g_small_m_threshold.load(); }
+
+cider_status_t cider_quantize_act(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, int8_t* q,
+                                  float* scale_x, void* stream) {
+    t_last_error[0] = '\0';
+    if (M < 0 || K < 1) return fail(CIDER_ERR_INVALID_ARG, "M >= 0 and K >= 1 required");
+    if (K % 16) return fail(CIDER_ERR_INVALID_ARG, "K = %lld must be a multiple of 16", (long long)K);
+    if (K > kMaxK) return fail(CIDER_ERR_INVALID_ARG, "K exceeds %lld", (long long)kMaxK);
+    if (xdt != CIDER_F16 && xdt != CIDER_BF16) return fail(CIDER_ERR_INVALID_ARG, "dtype %d unknown", (int)xdt);
+    if (M == 0) return CIDER_OK;
+    if (M > INT32_MAX) return fail(CIDER_ERR_INVALID_ARG, "M must be < 2^31");
+    if (!x || !q || !scale_x) return fail(CIDER_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scale_x) & 3u))
+        return fail(CIDER_ERR_INVALID_ARG, "x and q must be 16-byte aligned, scale_x 4-byte aligned");
+    const Range rx = rng(x, static_cast<size_t>(M) * K * 2);
+    if (overlap(rx, rng(q, static_cast<size_t>(M) * K)) || overlap(rx, rng(scale_x, M * 4)) ||
+        overlap(rng(q, static_cast<size_t>(M) * K), rng(scale_x, M * 4)))
+        return fail(CIDER_ERR_INVALID_ARG, "x, q and scale_x must not overlap");
+    DeviceInfo* d = nullptr;
+    cider_status_t s = device_info(&d);
+    if (s != CIDER_OK) return s;
+    cudaError_t e = launch_quantize_act(x, xdt, M, static_cast<int>(K), q, scale_x, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "quantize launch");
+}
+
+cider_status_t cider_w8a8_linear_pc(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, const int8_t* w,
+                                    const float* scale_w, int64_t N, void* y, cider_dtype_t ydt,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+    return linear(kModePC, x, xdt, M, K, w, scale_w, N, 0, y, ydt, workspace, workspace_bytes, stream);
+}
+
+cider_status_t cider_w8a8_linear_pg(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, const int8_t* w,
+                                    const float* scale_w, int64_t N, int64_t gs, void* y, cider_dtype_t ydt,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+    return linear(kModePG, x, xdt, M, K, w, scale_w, N, gs, y, ydt, workspace, workspace_bytes, stream);
+}
+
+cider_status_t cider_w4a8_linear_pg(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
+                                    const uint8_t* w_packed, const float* scale_w, int64_t N, int64_t gs,
+                                    void* y, cider_dtype_t ydt, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+    return linear(kModeW4, x, xdt, M, K, w_packed, scale_w, N, gs, y, ydt, workspace, workspace_bytes, stream);
+}
+
+cider_status_t cider_w8a8_gemm_pc_q(const int8_t* q, const float* scale_x, int64_t M, int64_t K, const int8_t* w,
+                                    const float* scale_w, int64_t N, void* y, cider_dtype_t ydt, void* stream) {
+    return gemm_q(kModePC, q, scale_x, M, K, w, scale_w, N, 0, y, ydt, stream);
+}
+
+cider_status_t cider_w8a8_gemm_pg_q(const int8_t* q, const float* scale_x, int64_t M, int64_t K, const int8_t* w,
+                                    const float* scale_w, int64_t N, int64_t gs, void* y, cider_dtype_t ydt,
+                                    void* stream) {
+    return gemm_q(kModePG, q, scale_x, M, K, w, scale_w, N, gs, y, ydt, stream);
+}
+
+cider_status_t cider_w4a8_gemm_pg_q(const int8_t* q, const float* scale_x, int64_t M, int64_t K,
+                                    const uint8_t* w_packed, const float* scale_w, int64_t N, int64_t gs,
+                                    void* y, cider_dtype_t ydt, void* stream) {
+    return gemm_q(kModeW4, q, scale_x, M, K, w_packed, scale_w, N, gs, y, ydt, stream);
+}
+
+cider_status_t cider_silu_mul_quantize(const void* gate, const void* up, cider_dtype_t dt, int64_t M, int64_t F,
+                                       int8_t* q, float* scale_x, void* a_out, void* stream) {
+    t_last_error[0] = '\0';
+    if (M < 0 || F < 1) return fail(CIDER_ERR_INVALID_ARG, "M >= 0 and F >= 1 required");
+    if (F % 16 || F > 32768) return fail(CIDER_ERR_INVALID_ARG, "F = %lld must be a multiple of 16 and <= 32768", (long long)F);
+    if (dt != CIDER_F16 && dt != CIDER_BF16) return fail(CIDER_ERR_INVALID_ARG, "dtype %d unknown", (int)dt);
+    if (M == 0) return CIDER_OK;
+    if (M > INT32_MAX) return fail(CIDER_ERR_INVALID_ARG, "M must be < 2^31");
+    if (!gate || !up || !q || !scale_x) return fail(CIDER_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(gate) || !aligned16(up) || !aligned16(q) || (a_out && !aligned16(a_out)) ||
+        (reinterpret_cast<uintptr_t>(scale_x) & 3u))
+        return fail(CIDER_ERR_INVALID_ARG, "misaligned pointer");
+    DeviceInfo* d = nullptr;
+    cider_status_t s = device_info(&d);
+    if (s != CIDER_OK) return s;
+    cudaError_t e = launch_silu_mul_quantize(gate, up, dt, M, static_cast<int>(F), q, scale_x, a_out,
+                                             static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "silu-mul-quantize launch");
+}
+
+static cider_status_t quantize_weight(int mode, const float* W, int64_t N, int64_t K, int64_t gs, void* out,
+                                      float* sw, void* stream) {
+    t_last_error[0] = '\0';
+    if (N < 1 || K < 1) return fail(CIDER_ERR_INVALID_ARG, "N, K >= 1 required");
+    if (N > INT32_MAX || K > kMaxK) return fail(CIDER_ERR_INVALID_ARG, "size out of range");
+    if (mode != 0) {
+        cider_status_t s = check_gs(K, gs, mode == 2);
+        if (s != CIDER_OK) return s;
+    }
+    if (!W || !out || !sw) return fail(CIDER_ERR_INVALID_ARG, "NULL pointer");
+    DeviceInfo* d = nullptr;
+    cider_status_t s = device_info(&d);
+    if (s != CIDER_OK) return s;
+    cudaError_t e = launch_quantize_weight(mode, W, N, static_cast<int>(K), static_cast<int>(gs), out, sw,
+                                           static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "weight quantize launch");
+}
+
+cider_status_t cider_quantize_weight_pc(const float* W, int64_t N, int64_t K, int8_t* w, float* scale_w,
+                                        void* stream) {
+    return quantize_weight(0, W, N, K, 0, w, scale_w, stream);
+}
+
+cider_status_t cider_quantize_weight_pg(const float* W, int64_t N, int64_t K, int64_t gs, int8_t* w,
+                                        float* scale_w, void* stream) {
+    return quantize_weight(1, W, N, K, gs, w, scale_w, stream);
+}
+
+cider_status_t cider_pack_weight_int4_pg(const float* W, int64_t N, int64_t K, int64_t gs, uint8_t* w_packed,
+                                         float* scale_w, void* stream) {
+    return quantize_weight(2, W, N, K, gs, w_packed, scale_w, stream);
+}
+
+cider_status_t cider_test_gemm_i32(const int8_t* q, const int8_t* w, int64_t M, int64_t N, int64_t K,
+                                   int32_t* acc, void* stream) {
+    t_last_error[0] = '\0';
+    alignas(16) static const float dummy[4] = {1, 1, 1, 1};  // scales are never read by the INT32 epilogue
+    cider_status_t s = check_common(q, M, K, w, dummy, N, acc, CIDER_F16, CIDER_F16);
+    if (s != CIDER_OK) return s;
+    if (M == 0) return CIDER_OK;
+    DeviceInfo* d = nullptr;
+    if ((s = device_info(&d)) != CIDER_OK) return s;
+    return run_gemm(kModeI32, q, nullptr, M, K, w, nullptr, N, 0, acc, 0, d, static_cast<cudaStream_t>(stream));
+}
+
+cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8_t* w, int64_t M, int64_t N, int64_t K,
+                                           int64_t gs, int32_t* acc_g, void* stream) {
+    t_last_error[0] = '\0';
+    alignas(16) static const float dummy[4] = {1, 1, 1, 1};
+    cider_status_t s = check_common(q, M, K, w, dummy, N, acc_g, CIDER_F16, CIDER_F16);
+    if (s != CIDER_OK) return s;
+    if ((s = check_gs(K, gs, false)) != CIDER_OK) return s;
+    if (M == 0) return CIDER_OK;
+    DeviceInfo* d = nullptr;
+    if ((s = device_info(&d)) != CIDER_OK) return s;
+    return run_gemm(kModeI32G, q, nullptr, M, K, w, nullptr, N, gs, acc_g, 0, d, static_cast<cudaStream_t>(stream));
+}
+
+cider_status_t cider_test_unpack_int4(const uint8_t* w_packed, int64_t N, int64_t K, int8_t* w, void* stream) {
+    t_last_error[0] = '\0';
+    if (N < 1 || K < 1 || K % 32) return fail(CIDER_ERR_INVALID_ARG, "N >= 1, K >= 1, K %% 32 == 0 required");
+    if (!w_packed || !w || !aligned16(w_packed) || !aligned16(w)) return fail(CIDER_ERR_INVALID_ARG, "bad pointer");
+    DeviceInfo* d = nullptr;
+    cider_status_t s = device_info(&d);
+    if (s != CIDER_OK) return s;
+    cudaError_t e = launch_unpack_int4(w_packed, N, static_cast<int>(K), w, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "unpack launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// cider_kernels.h -- host-side launchers shared between the library's
+// translation units (not part of the public C ABI; see include/cider.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace cider {
+
+// Device status word bits (read back by cider_device_status()).
+constexpr unsigned kStatusTimeout = 1u;
+
+enum : int {
+    kModePC = 0,    // per-channel dequant epilogue
+    kModePG = 1,    // per-group dequant epilogue
+    kModeW4 = 2,    // per-group epilogue, INT4 packed weights unpacked on chip
+    kModeI32 = 3,   // test: store the INT32 accumulator
+    kModeI32G = 4,  // test: store every per-group INT32 partial
+};
+
+struct GemmLaunch {
+    int mode;
+    const int8_t* q;   // [M][K]
+    const void* w;     // [N][K] int8, or [N][K/2] packed int4
+    const float* sx;   // [M]
+    const float* sw;   // [N] or [K/gs][N]
+    void* y;           // output
+    int M, N, K, gs;
+    int ydt;           // 0 fp16, 1 bf16
+    int bn;            // N tile for per-channel modes: 256 or 128
+    int num_sms;
+    unsigned* status;  // device status word
+};
+
+// Encodes a TMA descriptor through the driver entry point (no libcuda link).
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t rank, void* base,
+                       const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                       const cuuint32_t* elem_strides, CUtensorMapSwizzle swizzle);
+
+cudaError_t launch_quantize_act(const void* x, int xdt, int64_t M, int K, int8_t* q, float* sx,
+                                cudaStream_t st);
+cudaError_t launch_silu_mul_quantize(const void* g, const void* u, int dt, int64_t M, int F,
+                                     int8_t* q, float* sx, void* a_out, cudaStream_t st);
+// mode 0: per channel (out = int8 [N][K]); 1: per group int8; 2: per group int4 packed
+cudaError_t launch_quantize_weight(int mode, const float* W, int64_t N, int K, int gs, void* out,
+                                   float* sw, cudaStream_t st);
+cudaError_t launch_unpack_int4(const uint8_t* packed, int64_t N, int K, int8_t* w, cudaStream_t st);
+cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const void* w,
+                           const float* sw, int N, int gs, void* y, int ydt, int num_sms,
+                           cudaStream_t st);
+cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t st);
+
+}  // namespace cider

@@ -1,0 +1,325 @@
+// quantize.cu -- memory-bound kernels around the GEMM:
+//  * per-token activation quantization (one pass over x: absmax, scale, codes);
+//  * the fused SiLU(gate) * up -> quantize producer of a decoder MLP;
+//  * offline weight quantization (per channel, per group, INT4 packed);
+//  * the INT4 unpack of the W4A8 load path, as a standalone test kernel.
+//
+// Activation quantization follows the juejin post "在Mac上跑大模型，MLX 不是终点",
+// section "W8A8 对称量化：Cider 的选择" (scale = max|x|/127, codes
+// round(x/scale) clamped to [-128,127]); weight quantization the Cider README,
+// section "底层 API" (quantize_weight_int8, pack_weight_int4) and table "量化".
+//
+// Layout: a token row is read with 16-byte vector loads (8 fp16/bf16 values),
+// lane-strided so that each warp load covers 512 contiguous bytes; codes are
+// written as 8-byte vectors.  Rows up to 4096 wide are handled by one warp
+// (the row stays in registers between the max and the quantize pass); wider
+// rows by one 256-thread CTA, which keeps up to 16384 values in registers
+// and re-reads beyond that.
+#include "cider_device.cuh"
+#include "cider_kernels.h"
+
+namespace cider {
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Quantize eight values with `scale` and store them as 8 bytes.
+__device__ __forceinline__ void quant_store8(const float (&f)[8], float scale, int8_t* dst) {
+    int c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = quant_code(f[i], scale);
+    *reinterpret_cast<uint2*>(dst) = pack8_i8(c);
+}
+
+// ---- one warp per token row, row kept in registers (K <= 256 * NV) -------
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) k_quantize_warp(const T* __restrict__ x, int64_t M, int K,
+                                                       int8_t* __restrict__ q,
+                                                       float* __restrict__ sx) {
+    const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (row >= M) return;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
+    const int nch = K >> 3;
+    uint4 v[NV];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = lane + 32 * i;
+        if (c < nch) {
+            v[i] = __ldcs(xr + c);
+            float f[8];
+            unpack8_f32<T>(v[i], f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+        }
+    }
+    amax = warp_max(amax);
+    const float s = act_scale(amax);
+    if (lane == 0) sx[row] = s;
+    int8_t* qr = q + row * K;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = lane + 32 * i;
+        if (c < nch) {
+            float f[8];
+            unpack8_f32<T>(v[i], f);
+            quant_store8(f, s, qr + 8 * c);
+        }
+    }
+}
+
+// ---- one CTA (256 threads) per token row ---------------------------------
+// NV > 0: up to NV 16-byte chunks per thread stay in registers; NV == 0:
+// any width, the quantize pass re-reads the row (L1/L2 hits).
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) k_quantize_cta(const T* __restrict__ x, int K,
+                                                      int8_t* __restrict__ q,
+                                                      float* __restrict__ sx) {
+    __shared__ float red[8];
+    const int64_t row = blockIdx.x;
+    const int tid = threadIdx.x;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
+    const int nch = K >> 3;
+    constexpr int R = NV > 0 ? NV : 1;
+    uint4 v[R];
+    float amax = 0.0f;
+    if (NV > 0) {
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int c = tid + 256 * i;
+            if (c < nch) {
+                v[i] = __ldcs(xr + c);
+                float f[8];
+                unpack8_f32<T>(v[i], f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+            }
+        }
+    } else {
+        for (int c = tid; c < nch; c += 256) {
+            float f[8];
+            unpack8_f32<T>(__ldg(xr + c), f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+        }
+    }
+    amax = warp_max(amax);
+    if ((tid & 31) == 0) red[tid >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+    const float s = act_scale(amax);
+    if (tid == 0) sx[row] = s;
+    int8_t* qr = q + row * K;
+    if (NV > 0) {
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int c = tid + 256 * i;
+            if (c < nch) {
+                float f[8];
+                unpack8_f32<T>(v[i], f);
+                quant_store8(f, s, qr + 8 * c);
+            }
+        }
+    } else {
+        for (int c = tid; c < nch; c += 256) {
+            float f[8];
+            unpack8_f32<T>(__ldg(xr + c), f);
+            quant_store8(f, s, qr + 8 * c);
+        }
+    }
+}
+
+template <typename T>
+static cudaError_t launch_quantize_t(const void* x, int64_t M, int K, int8_t* q, float* sx,
+                                     cudaStream_t st) {
+    const T* xt = static_cast<const T*>(x);
+    if (M == 0) return cudaSuccess;
+    if (K <= 4096) {
+        const unsigned grid = static_cast<unsigned>((M + 7) / 8);
+        const int nv = (K + 255) / 256;
+        if (nv <= 1) k_quantize_warp<T, 1><<<grid, 256, 0, st>>>(xt, M, K, q, sx);
+        else if (nv <= 2) k_quantize_warp<T, 2><<<grid, 256, 0, st>>>(xt, M, K, q, sx);
+        else if (nv <= 4) k_quantize_warp<T, 4><<<grid, 256, 0, st>>>(xt, M, K, q, sx);
+        else if (nv <= 8) k_quantize_warp<T, 8><<<grid, 256, 0, st>>>(xt, M, K, q, sx);
+        else k_quantize_warp<T, 16><<<grid, 256, 0, st>>>(xt, M, K, q, sx);
+    } else {
+        const unsigned grid = static_cast<unsigned>(M);
+        const int nv = (K / 8 + 255) / 256;
+        if (nv <= 4) k_quantize_cta<T, 4><<<grid, 256, 0, st>>>(xt, K, q, sx);
+        else if (nv <= 8) k_quantize_cta<T, 8><<<grid, 256, 0, st>>>(xt, K, q, sx);
+        else k_quantize_cta<T, 0><<<grid, 256, 0, st>>>(xt, K, q, sx);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_act(const void* x, int xdt, int64_t M, int K, int8_t* q, float* sx,
+                                cudaStream_t st) {
+    return xdt == 1 ? launch_quantize_t<__nv_bfloat16>(x, M, K, q, sx, st)
+                    : launch_quantize_t<__half>(x, M, K, q, sx, st);
+}
+
+// ---- SiLU(gate) * up -> quantize, one CTA per token row ---------------------
+// a = round_T(silu(g) * u) in fp32 with silu(g) = g / (1 + e^-g); the codes
+// are taken from the rounded a, exactly as quantizing a stored `a` would.
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) k_silu_mul_quantize(const T* __restrict__ gate,
+                                                           const T* __restrict__ up, int F,
+                                                           int8_t* __restrict__ q,
+                                                           float* __restrict__ sx,
+                                                           T* __restrict__ a_out) {
+    __shared__ float red[8];
+    const int64_t row = blockIdx.x;
+    const int tid = threadIdx.x;
+    const uint4* gr = reinterpret_cast<const uint4*>(gate + row * F);
+    const uint4* ur = reinterpret_cast<const uint4*>(up + row * F);
+    const int nch = F >> 3;
+    uint4 av[NV];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = tid + 256 * i;
+        if (c < nch) {
+            float g[8], u[8];
+            unpack8_f32<T>(__ldcs(gr + c), g);
+            unpack8_f32<T>(__ldcs(ur + c), u);
+            T* ah = reinterpret_cast<T*>(&av[i]);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float sg = __fdiv_rn(g[j], 1.0f + expf(-g[j]));
+                ah[j] = from_f32<T>(sg * u[j]);
+                amax = fmaxf(amax, fabsf(to_f32<T>(ah[j])));
+            }
+            if (a_out) reinterpret_cast<uint4*>(a_out + row * F)[c] = av[i];
+        }
+    }
+    amax = warp_max(amax);
+    if ((tid & 31) == 0) red[tid >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+    const float s = act_scale(amax);
+    if (tid == 0) sx[row] = s;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = tid + 256 * i;
+        if (c < nch) {
+            float f[8];
+            unpack8_f32<T>(av[i], f);
+            quant_store8(f, s, q + row * F + 8 * c);
+        }
+    }
+}
+
+template <typename T>
+static cudaError_t launch_silu_t(const void* g, const void* u, int64_t M, int F, int8_t* q,
+                                 float* sx, void* a_out, cudaStream_t st) {
+    if (M == 0) return cudaSuccess;
+    const int nv = (F / 8 + 255) / 256;
+    const T* gt = static_cast<const T*>(g);
+    const T* ut = static_cast<const T*>(u);
+    T* at = static_cast<T*>(a_out);
+    const unsigned grid = static_cast<unsigned>(M);
+    if (nv <= 2) k_silu_mul_quantize<T, 2><<<grid, 256, 0, st>>>(gt, ut, F, q, sx, at);
+    else if (nv <= 8) k_silu_mul_quantize<T, 8><<<grid, 256, 0, st>>>(gt, ut, F, q, sx, at);
+    else if (nv <= 16) k_silu_mul_quantize<T, 16><<<grid, 256, 0, st>>>(gt, ut, F, q, sx, at);
+    else return cudaErrorInvalidValue;  // F > 32768: rejected by the host checks first
+    return cudaGetLastError();
+}
+
+cudaError_t launch_silu_mul_quantize(const void* g, const void* u, int dt, int64_t M, int F,
+                                     int8_t* q, float* sx, void* a_out, cudaStream_t st) {
+    return dt == 1 ? launch_silu_t<__nv_bfloat16>(g, u, M, F, q, sx, a_out, st)
+                   : launch_silu_t<__half>(g, u, M, F, q, sx, a_out, st);
+}
+
+// ---- offline weight quantization --------------------------------------------
+// Per channel: one CTA per output row, two passes (max, then codes).
+__global__ void __launch_bounds__(256) k_quantize_weight_pc(const float* __restrict__ W, int K,
+                                                            int8_t* __restrict__ w,
+                                                            float* __restrict__ sw) {
+    __shared__ float red[8];
+    const int64_t n = blockIdx.x;
+    const float* wr = W + n * K;
+    float amax = 0.0f;
+    for (int k = threadIdx.x; k < K; k += 256) amax = fmaxf(amax, fabsf(wr[k]));
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+    const float s = act_scale(amax);
+    if (threadIdx.x == 0) sw[n] = s;
+    for (int k = threadIdx.x; k < K; k += 256) w[n * K + k] = static_cast<int8_t>(quant_code(wr[k], s));
+}
+
+// Per group (INT8 or INT4): one warp per (row n, group g); scales group-major [G][N].
+template <bool INT4>
+__global__ void __launch_bounds__(256) k_quantize_weight_group(const float* __restrict__ W,
+                                                               int64_t N, int K, int gs,
+                                                               void* __restrict__ out,
+                                                               float* __restrict__ sw) {
+    const int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = K / gs;
+    if (item >= N * G) return;
+    const int64_t n = item / G;
+    const int g = static_cast<int>(item % G);
+    const float* wg = W + n * K + static_cast<int64_t>(g) * gs;
+    float amax = 0.0f;
+    for (int k = lane; k < gs; k += 32) amax = fmaxf(amax, fabsf(wg[k]));
+    amax = warp_max(amax);
+    const float s = INT4 ? __fdiv_rn(amax, 7.0f) : act_scale(amax);
+    if (lane == 0) sw[static_cast<int64_t>(g) * N + n] = s;
+    if (!INT4) {
+        int8_t* w = static_cast<int8_t*>(out) + n * K + static_cast<int64_t>(g) * gs;
+        for (int k = lane; k < gs; k += 32) w[k] = static_cast<int8_t>(quant_code(wg[k], s));
+    } else {
+        uint8_t* p = static_cast<uint8_t*>(out) + n * (K / 2) + static_cast<int64_t>(g) * (gs / 2);
+        for (int j = lane; j < gs / 2; j += 32) {
+            int c0 = 0, c1 = 0;
+            if (s != 0.0f) {
+                c0 = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(wg[2 * j], s)), -8.0f), 7.0f));
+                c1 = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(wg[2 * j + 1], s)), -8.0f), 7.0f));
+            }
+            p[j] = static_cast<uint8_t>((c0 + 8) | ((c1 + 8) << 4));
+        }
+    }
+}
+
+cudaError_t launch_quantize_weight(int mode, const float* W, int64_t N, int K, int gs, void* out,
+                                   float* sw, cudaStream_t st) {
+    if (mode == 0) {
+        k_quantize_weight_pc<<<static_cast<unsigned>(N), 256, 0, st>>>(W, K, static_cast<int8_t*>(out), sw);
+    } else {
+        const int64_t items = N * (K / gs);
+        const unsigned grid = static_cast<unsigned>((items + 7) / 8);
+        if (mode == 1)
+            k_quantize_weight_group<false><<<grid, 256, 0, st>>>(W, N, K, gs, out, sw);
+        else
+            k_quantize_weight_group<true><<<grid, 256, 0, st>>>(W, N, K, gs, out, sw);
+    }
+    return cudaGetLastError();
+}
+
+// ---- INT4 unpack (the W4A8 load path's conversion), standalone ---------------
+__global__ void k_unpack_int4(const uint32_t* __restrict__ packed, int64_t words, uint2* __restrict__ w) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i < words) w[i] = unpack_int4x8(packed[i]);
+}
+
+cudaError_t launch_unpack_int4(const uint8_t* packed, int64_t N, int K, int8_t* w, cudaStream_t st) {
+    const int64_t words = N * (K / 8);  // K % 32 == 0 keeps rows whole words
+    if (words == 0) return cudaSuccess;
+    k_unpack_int4<<<static_cast<unsigned>((words + 255) / 256), 256, 0, st>>>(
+        reinterpret_cast<const uint32_t*>(packed), words, reinterpret_cast<uint2*>(w));
+    return cudaGetLastError();
+}
+
+}  // namespace cider
