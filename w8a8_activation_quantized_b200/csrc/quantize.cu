@@ -165,7 +165,7 @@ cudaError_t launch_quantize_act(const void* x, int xdt, int64_t M, int K, int8_t
 }
 
 // ---- SiLU(gate) * up -> quantize, one CTA per token row ---------------------
-// a = round_T(silu(g) * u) in fp32 with silu(g) = g / (1 + e^-g); the codes
+// a = round_T(silu(g) * u) in fp32 with silu(g) = g * sigmoid(g); the codes
 // are taken from the rounded a, exactly as quantizing a stored `a` would.
 template <typename T, int NV>
 __global__ void __launch_bounds__(256) k_silu_mul_quantize(const T* __restrict__ gate,
@@ -191,8 +191,11 @@ __global__ void __launch_bounds__(256) k_silu_mul_quantize(const T* __restrict__
             T* ah = reinterpret_cast<T*>(&av[i]);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float sg = __fdiv_rn(g[j], 1.0f + expf(-g[j]));
-                ah[j] = from_f32<T>(sg * u[j]);
+                // sigmoid(g) = 1/(1+e^-g) for g >= 0 and e^g/(1+e^g) for g < 0:
+                // e^-|g| never overflows, so large negative g keep their tiny value.
+                const float e = expf(-fabsf(g[j]));
+                const float sig = __fdiv_rn(g[j] >= 0.0f ? 1.0f : e, 1.0f + e);
+                ah[j] = from_f32<T>((g[j] * sig) * u[j]);
                 amax = fmaxf(amax, fabsf(to_f32<T>(ah[j])));
             }
             if (a_out) reinterpret_cast<uint4*>(a_out + row * F)[c] = av[i];
