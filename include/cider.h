@@ -141,6 +141,32 @@ CIDER_API cider_status_t cider_w4a8_linear_pg(const void* x, cider_dtype_t xdt, 
                                     int64_t gs, void* y, cider_dtype_t ydt,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* W8A8 per-channel linear for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is an addition of this library.
+ *
+ * Some callers cannot call cudaMalloc and so cannot pass a workspace: a host
+ * application or framework that owns all of the GPU's memory through its own
+ * pool and forbids outside allocations, or code that must stay inside a
+ * memory budget fixed at start-up.  This entry point computes exactly what
+ * cider_w8a8_linear_pc computes, but keeps the quantized activations and
+ * their scales in a scratch array built into the library: 32 MiB of device
+ * memory, which every GPU that loads the library holds until the process
+ * exits.  It allocates nothing and calls no allocating routine.
+ *  - Limit: cider_workspace_bytes(M, K) must not exceed 32 MiB (roughly
+ *    M * K + 4 * M <= 32 MiB); larger calls return CIDER_ERR_INVALID_ARG with
+ *    a message and launch nothing.  Calls that take the fused small-M kernel
+ *    do not touch the scratch.
+ *  - The first call on each device looks up the scratch's device address,
+ *    with that device current; make that first call before any stream capture.
+ *  - All calls on a device share the one scratch array and it keeps the last
+ *    call's contents.  Calls whose kernels overlap on the GPU (on different
+ *    streams, or from different host threads) race on it and give wrong
+ *    results; serialise them, e.g. on one stream.
+ * Arguments, layouts and errors are as for cider_w8a8_linear_pc. */
+CIDER_API cider_status_t cider_w8a8_linear_pc_noalloc(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
+                                                      const int8_t* w, const float* scale_w, int64_t N,
+                                                      void* y, cider_dtype_t ydt, void* stream);
+
 /* ---- the GEMM stage on pre-quantized activations ------------------------ */
 /* The same products and epilogues as the linears above, fed q [M][K] int8 and
  * scale_x [M] fp32 from cider_quantize_act or a fused producer.  Always the

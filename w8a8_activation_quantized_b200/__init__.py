@@ -45,6 +45,7 @@ _SIGNATURES = {
     "cider_w8a8_linear_pc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P, _SZ, _P]),
     "cider_w8a8_linear_pg": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P, _SZ, _P]),
     "cider_w4a8_linear_pg": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P, _SZ, _P]),
+    "cider_w8a8_linear_pc_noalloc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_w8a8_gemm_pc_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_w8a8_gemm_pg_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P]),
     "cider_w4a8_gemm_pg_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P]),
@@ -181,6 +182,21 @@ def cider_w4a8_linear_pg(x, w_packed, scale_w, gs, y=None, out_dtype=None, works
     _check("cider_w4a8_linear_pg", lib().cider_w4a8_linear_pg(
         _ptr(x), _DT[x.dtype], M, K, _ptr(w_packed), _ptr(scale_w), N, gs, _ptr(y), _DT[y.dtype],
         _ptr(ws), ws_bytes, _stream(stream, x.device)))
+    return y
+
+
+def cider_w8a8_linear_pc_noalloc(x, w, scale_w, y=None, out_dtype=None, stream=None):
+    """The per-channel linear without a workspace, for callers that cannot
+    allocate device memory: its scratch is a fixed 32 MiB array inside the
+    library, shared by every call on the device (calls that overlap on the GPU
+    race on it).  Raises CiderError when M*K is too large for that scratch."""
+    _contig(x, "x"), _contig(w, "w")
+    M, K = x.shape
+    N = w.shape[0]
+    y = _out(y, M, N, out_dtype or x.dtype, x.device)
+    _check("cider_w8a8_linear_pc_noalloc", lib().cider_w8a8_linear_pc_noalloc(
+        _ptr(x), _DT[x.dtype], M, K, _ptr(w), _ptr(scale_w), N, _ptr(y), _DT[y.dtype],
+        _stream(stream, x.device)))
     return y
 
 

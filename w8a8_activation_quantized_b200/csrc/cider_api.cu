@@ -212,6 +212,14 @@ std::once_flag g_encode_once;
 
 }  // namespace
 
+cider_status_t set_error(cider_status_t s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_last_error, sizeof t_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
 bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t rank, void* base,
                        const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
                        const cuuint32_t* elem_strides, CUtensorMapSwizzle swizzle) {

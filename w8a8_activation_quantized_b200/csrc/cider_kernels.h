@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/cider.h"
+
 namespace cider {
 
 // Device status word bits (read back by cider_device_status()).
@@ -32,6 +34,9 @@ struct GemmLaunch {
     int num_sms;
     unsigned* status;  // device status word
 };
+
+// Records a message for cider_last_error() on this thread and returns `s`.
+cider_status_t set_error(cider_status_t s, const char* fmt, ...);
 
 // Encodes a TMA descriptor through the driver entry point (no libcuda link).
 bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t rank, void* base,
