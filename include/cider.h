@@ -212,6 +212,11 @@ CIDER_API cider_status_t cider_test_gemm_i32(const int8_t* q, const int8_t* w, i
 /* Per-group INT32 partials acc_g[g][m][n] = sum_{k in group g} q[m,k]*w[n,k]. */
 CIDER_API cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8_t* w, int64_t M, int64_t N,
                                            int64_t K, int64_t gs, int32_t* acc_g, void* stream);
+/* Forces the kernel variant of the per-channel and INT32 GEMM for later calls
+ * (process-wide): 0 = automatic (default), 1 = single-CTA 128x128 tiles,
+ * 2 = single-CTA 128x256 tiles, 3 = CTA-pair 256x256 tiles.  Lets tests cover
+ * every variant on small shapes. */
+CIDER_API cider_status_t cider_test_set_gemm_variant(int variant);
 /* The W4A8 load path's unpack: w[n][k] = nibble(n, k) - 8. */
 CIDER_API cider_status_t cider_test_unpack_int4(const uint8_t* w_packed, int64_t N, int64_t K, int8_t* w,
                                       void* stream);

@@ -1,0 +1,75 @@
+"""Every kernel variant of the per-channel GEMM against the oracle on small and
+ragged shapes: single-CTA 128x128 and 128x256 tiles, and the CTA-pair
+256x256 tile (tcgen05.mma.cta_group::2).  Bit-exact INT32 accumulators, and
+the fused dequant within the row-relative tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import w8a8_activation_quantized_b200 as cider
+from w8a8_activation_quantized_b200 import synth
+from tests.parity import act, check_y, dev, dev_bits
+
+pytestmark = pytest.mark.gpu
+
+VARIANTS = {"single128": 1, "single256": 2, "pair256": 3}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    yield
+    cider.cider_test_set_gemm_variant(0)
+    cider.cider_device_status()
+
+
+@pytest.fixture(params=sorted(VARIANTS))
+def variant(request):
+    cider.cider_test_set_gemm_variant(VARIANTS[request.param])
+    yield request.param
+    cider.cider_test_set_gemm_variant(0)
+
+
+def _codes(M, N, K, seed):
+    rng = np.random.default_rng(seed)
+    q = rng.integers(-127, 128, size=(M, K), dtype=np.int64).astype(np.int8)
+    w = rng.integers(-128, 128, size=(N, K), dtype=np.int64).astype(np.int8)
+    return q, w
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 128), (1, 8, 16), (257, 264, 272), (300, 520, 1040),
+                                   (512, 1024, 2560), (130, 3080, 96), (1283, 4104, 272)])
+def test_gemm_i32_variant(variant, M, N, K):
+    q, w = _codes(M, N, K, seed=M * 3 + N + K)
+    acc = cider.cider_test_gemm_i32(dev(q), dev(w))
+    np.testing.assert_array_equal(acc.cpu().numpy(), oracle.gemm_i32(q, w))
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 256), (300, 1032, 2560), (129, 264, 4096), (520, 2056, 1040)])
+def test_linear_pc_variant(variant, M, N, K):
+    cider.cider_set_small_m_threshold(4)
+    x = act(M, K, seed=M + N + K)
+    qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed=M + K))
+    y = cider.cider_w8a8_linear_pc(dev_bits(x, oracle.F16), dev(qw), dev(sw))
+    check_y(y, oracle.linear_pc(x, qw, sw), oracle.F16)
+
+
+def test_pair_is_chosen_for_large_m():
+    """The automatic choice sends the headline shape to the CTA-pair kernel; the
+    result must equal the forced single-CTA result bit for bit (same arithmetic)."""
+    M, N, K = 2048, 4096, 1024
+    x = act(M, K, seed=5)
+    qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed=5))
+    xd, wd, sd = dev_bits(x, oracle.F16), dev(qw), dev(sw)
+    cider.cider_test_set_gemm_variant(3)
+    y_pair = cider.cider_w8a8_linear_pc(xd, wd, sd)
+    cider.cider_test_set_gemm_variant(2)
+    y_single = cider.cider_w8a8_linear_pc(xd, wd, sd)
+    cider.cider_test_set_gemm_variant(0)
+    y_auto = cider.cider_w8a8_linear_pc(xd, wd, sd)
+    torch.cuda.synchronize()
+    assert torch.equal(y_pair, y_single) and torch.equal(y_auto, y_pair)
+    rows = np.arange(0, M, 97)
+    check_y(y_auto, oracle.linear_pc(x[rows], qw, sw), oracle.F16, rows=rows)

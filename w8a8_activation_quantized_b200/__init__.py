@@ -56,6 +56,7 @@ _SIGNATURES = {
     "cider_test_gemm_i32": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P]),
     "cider_test_gemm_i32_grouped": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _P, _P]),
     "cider_test_unpack_int4": (_INT, [_P, _I64, _I64, _P, _P]),
+    "cider_test_set_gemm_variant": (_INT, [_INT]),
 }
 EXPORTS = tuple(_SIGNATURES)
 
@@ -291,6 +292,11 @@ def cider_test_gemm_i32_grouped(q, w, gs, acc_g=None, stream=None):
     _check("cider_test_gemm_i32_grouped", lib().cider_test_gemm_i32_grouped(
         _ptr(q), _ptr(w), M, N, K, gs, _ptr(acc_g), _stream(stream, q.device)))
     return acc_g
+
+
+def cider_test_set_gemm_variant(variant: int):
+    """0 automatic, 1 single-CTA 128x128, 2 single-CTA 128x256, 3 CTA-pair 256x256."""
+    _check("cider_test_set_gemm_variant", lib().cider_test_set_gemm_variant(variant))
 
 
 def cider_test_unpack_int4(w_packed, K, w=None, stream=None):

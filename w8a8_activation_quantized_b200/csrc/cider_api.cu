@@ -24,6 +24,7 @@ constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxK = 131072;            // 127 * 128 * K < 2^31 keeps INT32 exact
 constexpr int64_t kMaxSmallM = 16;
 constexpr int64_t kSmallSmemLimit = 160 * 1024;  // q rows of the small-M kernel in shared memory
+constexpr int64_t kSmallMaxK = 32768;
 
 struct DeviceInfo {
     int ready = 0;     // 1 = filled in
@@ -96,8 +97,10 @@ bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// The fused small-M kernel keeps the M code rows in shared memory and at most
+// 8 passes of 512 weights per warp in registers (K <= 32768).
 bool small_m_path(int64_t M, int64_t K) {
-    return M >= 1 && M <= g_small_m_threshold.load() && M * K <= kSmallSmemLimit;
+    return M >= 1 && M <= g_small_m_threshold.load() && M * K <= kSmallSmemLimit && K <= kSmallMaxK;
 }
 
 // Common checks of the linear / GEMM entry points.
@@ -125,9 +128,17 @@ cider_status_t check_gs(int64_t K, int64_t gs, bool w4) {
     return CIDER_OK;
 }
 
-int pick_bn(int64_t M, int64_t N, int num_sms) {
+std::atomic<int> g_gemm_variant{kGemmAuto};  // test override
+
+// Per-channel GEMM variant: the CTA-pair 256x256 tile when it still gives
+// every pair of SMs a tile, else single-CTA tiles of 128x256 or 128x128.
+int pick_variant(int64_t M, int64_t N, int num_sms) {
+    const int forced = g_gemm_variant.load();
+    if (forced != kGemmAuto) return forced;
+    const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    if (M > 128 && pair_tiles >= num_sms / 2) return kGemmPair;
     const int64_t tiles256 = ((M + 127) / 128) * ((N + 255) / 256);
-    return tiles256 < num_sms ? 128 : 256;
+    return tiles256 < num_sms ? kGemmSingle128 : kGemmSingle256;
 }
 
 cider_status_t run_gemm(int mode, const int8_t* q, const float* sx, int64_t M, int64_t K,
@@ -145,7 +156,7 @@ cider_status_t run_gemm(int mode, const int8_t* q, const float* sx, int64_t M, i
     L.K = static_cast<int>(K);
     L.gs = static_cast<int>(gs);
     L.ydt = ydt;
-    L.bn = (mode == kModePC || mode == kModeI32) ? pick_bn(M, N, d->num_sms) : 128;
+    L.variant = (mode == kModePC || mode == kModeI32) ? pick_variant(M, N, d->num_sms) : kGemmSingle128;
     L.num_sms = d->num_sms;
     L.status = d->status;
     cudaError_t e = launch_gemm(L, st);
@@ -436,6 +447,13 @@ cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8_t* w, int
     DeviceInfo* d = nullptr;
     if ((s = device_info(&d)) != CIDER_OK) return s;
     return run_gemm(kModeI32G, q, nullptr, M, K, w, nullptr, N, gs, acc_g, 0, d, static_cast<cudaStream_t>(stream));
+}
+
+cider_status_t cider_test_set_gemm_variant(int variant) {
+    if (variant < kGemmAuto || variant > kGemmPair)
+        return fail(CIDER_ERR_INVALID_ARG, "variant %d outside [0, 3]", variant);
+    g_gemm_variant.store(variant);
+    return CIDER_OK;
 }
 
 cider_status_t cider_test_unpack_int4(const uint8_t* w_packed, int64_t N, int64_t K, int8_t* w, void* stream) {

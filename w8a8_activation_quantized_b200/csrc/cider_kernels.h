@@ -21,6 +21,10 @@ enum : int {
     kModeI32G = 4,  // test: store every per-group INT32 partial
 };
 
+// Kernel variants of the per-channel GEMM (the grouped modes always use the
+// single-CTA kernel with 128-wide N tiles).
+enum : int { kGemmAuto = 0, kGemmSingle128 = 1, kGemmSingle256 = 2, kGemmPair = 3 };
+
 struct GemmLaunch {
     int mode;
     const int8_t* q;   // [M][K]
@@ -30,7 +34,7 @@ struct GemmLaunch {
     void* y;           // output
     int M, N, K, gs;
     int ydt;           // 0 fp16, 1 bf16
-    int bn;            // N tile for per-channel modes: 256 or 128
+    int variant;       // per-channel modes: kGemmSingle128, kGemmSingle256 or kGemmPair
     int num_sms;
     unsigned* status;  // device status word
 };

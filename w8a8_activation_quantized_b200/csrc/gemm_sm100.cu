@@ -98,6 +98,34 @@ __device__ __forceinline__ void store_row8(TY* dst, const float (&v)[8]) {
     *reinterpret_cast<uint4*>(dst) = o;
 }
 
+// Per-channel (or INT32) epilogue for 32 accumulator columns of one row m:
+// y[m, n0..n0+31] = acc * scale_x[m] * scale_w[n], or the raw INT32 values.
+template <int MODE, typename TY>
+__device__ __forceinline__ void store_chunk_pc(const GemmArgs& p, const uint32_t (&r)[32], int m, int n0, float sxm) {
+    if (MODE == kModeI32) {
+        int32_t* out = static_cast<int32_t*>(p.y) + static_cast<int64_t>(m) * p.N;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (n0 + 4 * j < p.N)
+                *reinterpret_cast<uint4*>(out + n0 + 4 * j) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+    } else {
+        TY* out = static_cast<TY*>(p.y) + static_cast<int64_t>(m) * p.N;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (n0 + 8 * j < p.N) {
+                const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.sw + n0 + 8 * j));
+                const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.sw + n0 + 8 * j + 4));
+                const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    v[e] = (static_cast<float>(static_cast<int32_t>(r[8 * j + e])) * sxm) * ws[e];
+                store_row8<TY>(out + n0 + 8 * j, v);
+            }
+        }
+    }
+}
+
 template <typename Cfg, typename TY>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     k_gemm_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -252,30 +280,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                         tc_fence_before();
                         mbar_arrive(&acce[b]);
                     }
-                    const int n0 = n_base + c * 32;
-                    if (!mvalid) continue;
-                    if (Cfg::MODE == kModeI32) {
-                        int32_t* out = static_cast<int32_t*>(p.y) + static_cast<int64_t>(m) * p.N;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            if (n0 + 4 * j < p.N)
-                                *reinterpret_cast<uint4*>(out + n0 + 4 * j) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-                    } else {
-                        TY* out = static_cast<TY*>(p.y) + static_cast<int64_t>(m) * p.N;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            if (n0 + 8 * j < p.N) {
-                                const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.sw + n0 + 8 * j));
-                                const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.sw + n0 + 8 * j + 4));
-                                const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                                float v[8];
-#pragma unroll
-                                for (int e = 0; e < 8; ++e)
-                                    v[e] = (static_cast<float>(static_cast<int32_t>(r[8 * j + e])) * sxm) * ws[e];
-                                store_row8<TY>(out + n0 + 8 * j, v);
-                            }
-                        }
-                    }
+                    if (mvalid) store_chunk_pc<Cfg::MODE, TY>(p, r, m, n_base + c * 32, sxm);
                 }
                 ++acc_i;
             } else {
@@ -377,6 +382,170 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
+// CTA-pair kernel (per-channel and INT32 modes): one 256 x 256 output tile per
+// cluster of two CTAs with tcgen05.mma.cta_group::2.  Each CTA stages its own
+// 128 rows of A and its half (128 rows) of B, so per multiply-add a CTA moves
+// two thirds of the bytes of the single-CTA 128 x 256 tile.  The even CTA
+// (the pair's leader) issues the MMAs; its full barrier counts the TMA bytes of
+// both CTAs, the MMA commits arrive on both CTAs' barriers, and the epilogue
+// warps of both CTAs report to the leader's accumulator-empty barriers.
+// Each CTA's TMEM holds the accumulator rows of its own 128 rows of A.
+// ---------------------------------------------------------------------------
+struct PairCfg {
+    static constexpr int BM = 256;                   // rows of the pair tile
+    static constexpr int BN = 256;                   // columns of the pair tile
+    static constexpr int A_BYTES = 128 * kBK;        // this CTA's rows of A
+    static constexpr int B_BYTES = (BN / 2) * kBK;   // this CTA's half of B
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = kSmemBudget / STAGE_BYTES;  // 6
+    static constexpr int ACC_BUFS = 2;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int EPI_WARPS = 4;
+    static constexpr int THREADS = 32 * (2 + EPI_WARPS);
+    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * ACC_BUFS) + 16;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+};
+
+template <int MODE, typename TY>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs p) {
+    using C = PairCfg;
+    constexpr int S = C::STAGES;
+    constexpr int NB = C::ACC_BUFS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + S * C::A_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::B_BYTES);
+    uint64_t* empty = full + S;
+    uint64_t* accf = empty + S;
+    uint64_t* acce = accf + NB;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + NB);
+    __shared__ int s_abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = (rank == 0);
+    const int cid = static_cast<int>(cluster_id_x());
+    const int ncl = static_cast<int>(cluster_count_x());
+    const int num_tiles = p.num_m_blocks * p.num_n_blocks;
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], 2 * C::EPI_WARPS);  // one arrival per epilogue warp of either CTA
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    volatile int* abort_flag = &s_abort;
+
+    if (warp == 0) {
+        // ---------------- TMA producer (both CTAs): own A rows, own half of B ----------------
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = cid; t < num_tiles && ok; t += ncl) {
+                int mb, nb;
+                tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
+                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                    if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, p.status, abort_flag)) { ok = false; break; }
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+                    const uint32_t bar = map_to_rank(&full[stage], 0);
+                    tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, bar, kb * kBK, mb * C::BM + static_cast<int>(rank) * 128);
+                    tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, bar, kb * kBK, nb * C::BN + static_cast<int>(rank) * (C::BN / 2));
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (leader CTA only) ----------------
+        if (leader && lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_i8(C::BM, C::BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t acc_i = 0;
+            bool ok = true;
+            for (int t = cid; t < num_tiles && ok; t += ncl) {
+                const uint32_t b = acc_i % NB;
+                if (!mbar_wait_cluster(&acce[b], ((acc_i / NB) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem_base + b * C::BN;
+                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                    if (!mbar_wait_cluster(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
+                    const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+                        umma_i8_pair(d, adesc + (kk * kUmmaK >> 4), bdesc + (kk * kUmmaK >> 4), idesc,
+                                     (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit_pair(&empty[stage]);
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                umma_commit_pair(&accf[b]);
+                ++acc_i;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- epilogue (both CTAs): this CTA's 128 rows x 256 columns ----------------
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        uint32_t acc_i = 0;
+        bool ok = true;
+        for (int t = cid; t < num_tiles && ok; t += ncl) {
+            int mb, nb;
+            tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
+            const int m = mb * C::BM + static_cast<int>(rank) * 128 + row;
+            const bool mvalid = m < p.M;
+            const uint32_t b = acc_i % NB;
+            if (!mbar_wait_cluster(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const float sxm = (MODE == kModePC && mvalid) ? __ldg(p.sx + m) : 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < C::BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + b * C::BN + c * 32, r);
+                tmem_ld_wait();
+                if (c == C::BN / 32 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(map_to_rank(&acce[b], 0));
+                }
+                if (mvalid) store_chunk_pc<MODE, TY>(p, r, m, nb * C::BN + c * 32, sxm);
+            }
+            ++acc_i;
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();  // all MMAs of the pair consumed, no peer arrivals in flight
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Host side: tensor maps and launch.
 // ---------------------------------------------------------------------------
 static bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
@@ -421,9 +590,36 @@ static cudaError_t launch_gemm_cfg(const GemmLaunch& L, cudaStream_t st) {
 }
 
 template <int MODE, typename TY>
+static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
+    CUtensorMap tmA, tmB;
+    if (!make_map_2d(&tmA, L.q, L.K, L.M, kBK, 128, true)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&tmB, L.w, L.K, L.N, kBK, PairCfg::BN / 2, true)) return cudaErrorInvalidValue;
+    GemmArgs a;
+    a.M = L.M;
+    a.N = L.N;
+    a.K = L.K;
+    a.gs = 0;
+    a.num_m_blocks = (L.M + PairCfg::BM - 1) / PairCfg::BM;
+    a.num_n_blocks = (L.N + PairCfg::BN - 1) / PairCfg::BN;
+    a.num_k_blocks = (L.K + kBK - 1) / kBK;
+    a.sx = L.sx;
+    a.sw = L.sw;
+    a.y = L.y;
+    a.status = L.status;
+    const int tiles = a.num_m_blocks * a.num_n_blocks;
+    const int clusters = tiles < L.num_sms / 2 ? tiles : L.num_sms / 2;
+    auto kern = k_gemm_pair<MODE, TY>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<2 * clusters, PairCfg::THREADS, PairCfg::SMEM_BYTES, st>>>(tmA, tmB, a);
+    return cudaGetLastError();
+}
+
+template <int MODE, typename TY>
 static cudaError_t launch_gemm_mode(const GemmLaunch& L, cudaStream_t st) {
     if constexpr (MODE == kModePC || MODE == kModeI32) {
-        if (L.bn == 128) return launch_gemm_cfg<GemmCfg<128, MODE>, TY>(L, st);
+        if (L.variant == kGemmPair) return launch_gemm_pair<MODE, TY>(L, st);
+        if (L.variant == kGemmSingle128) return launch_gemm_cfg<GemmCfg<128, MODE>, TY>(L, st);
         return launch_gemm_cfg<GemmCfg<256, MODE>, TY>(L, st);
     } else {
         return launch_gemm_cfg<GemmCfg<128, MODE>, TY>(L, st);

@@ -26,17 +26,16 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-// Quantize eight values with `scale` and store them as 8 bytes.
-__device__ __forceinline__ void quant_store8(const float (&f)[8], float scale, int8_t* dst) {
-    int c[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) c[i] = quant_code(f[i], scale);
-    *reinterpret_cast<uint2*>(dst) = pack8_i8(c);
+// Quantize eight values with `scale` (reciprocal `rcp`) and store them as 8 bytes.
+__device__ __forceinline__ void quant_store8(const float (&f)[8], float scale, float rcp, int8_t* dst) {
+    *reinterpret_cast<uint2*>(dst) = quant8_codes(f, scale, rcp);
 }
 
 // ---- one warp per token row, row kept in registers (K <= 256 * NV) -------
+// 128-thread CTAs (4 rows each) and NV sized to K keep registers low, so many
+// warps per SM have loads in flight while others quantize.
 template <typename T, int NV>
-__global__ void __launch_bounds__(256) k_quantize_warp(const T* __restrict__ x, int64_t M, int K,
+__global__ void __launch_bounds__(128, (NV <= 10 ? 8 : 5)) k_quantize_warp(const T* __restrict__ x, int64_t M, int K,
                                                        int8_t* __restrict__ q,
                                                        float* __restrict__ sx) {
     const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -59,6 +58,7 @@ __global__ void __launch_bounds__(256) k_quantize_warp(const T* __restrict__ x, 
     }
     amax = warp_max(amax);
     const float s = act_scale(amax);
+    const float rs = act_rcp(s);
     if (lane == 0) sx[row] = s;
     int8_t* qr = q + row * K;
 #pragma unroll
@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(256) k_quantize_warp(const T* __restrict__ x, 
         if (c < nch) {
             float f[8];
             unpack8_f32<T>(v[i], f);
-            quant_store8(f, s, qr + 8 * c);
+            quant_store8(f, s, rs, qr + 8 * c);
         }
     }
 }
@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(256) k_quantize_cta(const T* __restrict__ x, i
 #pragma unroll
     for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
     const float s = act_scale(amax);
+    const float rs = act_rcp(s);
     if (tid == 0) sx[row] = s;
     int8_t* qr = q + row * K;
     if (NV > 0) {
@@ -123,14 +124,14 @@ __global__ void __launch_bounds__(256) k_quantize_cta(const T* __restrict__ x, i
             if (c < nch) {
                 float f[8];
                 unpack8_f32<T>(v[i], f);
-                quant_store8(f, s, qr + 8 * c);
+                quant_store8(f, s, rs, qr + 8 * c);
             }
         }
     } else {
         for (int c = tid; c < nch; c += 256) {
             float f[8];
             unpack8_f32<T>(__ldg(xr + c), f);
-            quant_store8(f, s, qr + 8 * c);
+            quant_store8(f, s, rs, qr + 8 * c);
         }
     }
 }
@@ -141,13 +142,16 @@ static cudaError_t launch_quantize_t(const void* x, int64_t M, int K, int8_t* q,
     const T* xt = static_cast<const T*>(x);
     if (M == 0) return cudaSuccess;
     if (K <= 4096) {
-        const unsigned grid = static_cast<unsigned>((M + 7) / 8);
+        const unsigned grid = static_cast<unsigned>((M + 3) / 4);
         const int nv = (K + 255) / 256;
-        if (nv <= 1) k_quantize_warp<T, 1><<<grid, 256, 0, st>>>(xt, M, K, q, sx);
-        else if (nv <= 2) k_quantize_warp<T, 2><<<grid, 256, 0, st>>>(xt, M, K, q, sx);
-        else if (nv <= 4) k_quantize_warp<T, 4><<<grid, 256, 0, st>>>(xt, M, K, q, sx);
-        else if (nv <= 8) k_quantize_warp<T, 8><<<grid, 256, 0, st>>>(xt, M, K, q, sx);
-        else k_quantize_warp<T, 16><<<grid, 256, 0, st>>>(xt, M, K, q, sx);
+        if (nv <= 1) k_quantize_warp<T, 1><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
+        else if (nv <= 2) k_quantize_warp<T, 2><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
+        else if (nv <= 4) k_quantize_warp<T, 4><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
+        else if (nv <= 6) k_quantize_warp<T, 6><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
+        else if (nv <= 8) k_quantize_warp<T, 8><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
+        else if (nv <= 10) k_quantize_warp<T, 10><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
+        else if (nv <= 12) k_quantize_warp<T, 12><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
+        else k_quantize_warp<T, 16><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
     } else {
         const unsigned grid = static_cast<unsigned>(M);
         const int nv = (K / 8 + 255) / 256;
@@ -208,6 +212,7 @@ __global__ void __launch_bounds__(256) k_silu_mul_quantize(const T* __restrict__
 #pragma unroll
     for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
     const float s = act_scale(amax);
+    const float rs = act_rcp(s);
     if (tid == 0) sx[row] = s;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(256) k_silu_mul_quantize(const T* __restrict__
         if (c < nch) {
             float f[8];
             unpack8_f32<T>(av[i], f);
-            quant_store8(f, s, q + row * F + 8 * c);
+            quant_store8(f, s, rs, q + row * F + 8 * c);
         }
     }
 }
