@@ -400,15 +400,55 @@ struct PairCfg {
     static constexpr int STAGES = kSmemBudget / STAGE_BYTES;  // 6
     static constexpr int ACC_BUFS = 2;
     static constexpr int TMEM_COLS = 512;
-    static constexpr int EPI_WARPS = 4;
+    static constexpr int EPI_WARPS = 8;                 // two per TMEM lane quarter
+    static constexpr int EPI_COLS = BN / 2;             // columns per epilogue warp
     static constexpr int THREADS = 32 * (2 + EPI_WARPS);
+    static constexpr int STG_BYTES = 32 * 32 * 2;       // one 32 x 32 fp16 output box
+    static constexpr int STG_PER_WARP = 2;              // double-buffered
     static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * ACC_BUFS) + 16;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_WARPS * STG_PER_WARP * STG_BYTES + BAR_BYTES;
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
+
+// 32 accumulators of one row -> 32 outputs, written as 4 swizzled 16-byte
+// chunks into row `r` of a 32 x 32 staging box laid out for the TMA 64-byte
+// swizzle (16-byte chunk j of row r lands at chunk j ^ ((r >> 1) & 3)).
+template <typename TY>
+__device__ __forceinline__ void stage_row32(uint8_t* box, int r, const uint32_t (&acc)[32], const float (&ws)[32],
+                                            float sxm) {
+    uint8_t* row = box + r * 64;
+    const int sw = (r >> 1) & 3;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            v[e] = (static_cast<float>(static_cast<int32_t>(acc[8 * j + e])) * sxm) * ws[8 * j + e];
+        uint4 o;
+        o.x = pack2_out<TY>(v[0], v[1]);
+        o.y = pack2_out<TY>(v[2], v[3]);
+        o.z = pack2_out<TY>(v[4], v[5]);
+        o.w = pack2_out<TY>(v[6], v[7]);
+        *reinterpret_cast<uint4*>(row + ((j ^ sw) << 4)) = o;
+    }
+}
+
+__device__ __forceinline__ void load_scales32(const float* sw, int n0, int N, float (&ws)[32]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (n0 + 4 * j < N) v = __ldg(reinterpret_cast<const float4*>(sw + n0 + 4 * j));
+        ws[4 * j] = v.x;
+        ws[4 * j + 1] = v.y;
+        ws[4 * j + 2] = v.z;
+        ws[4 * j + 3] = v.w;
+    }
+}
 
 template <int MODE, typename TY>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
-    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs p) {
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
     using C = PairCfg;
     constexpr int S = C::STAGES;
     constexpr int NB = C::ACC_BUFS;
@@ -416,7 +456,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + S * C::A_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::B_BYTES);
+    uint8_t* sStg = sB + S * C::B_BYTES;  // [EPI_WARPS][2][32 x 32 outputs]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sStg + C::EPI_WARPS * C::STG_PER_WARP * C::STG_BYTES);
     uint64_t* empty = full + S;
     uint64_t* accf = empty + S;
     uint64_t* acce = accf + NB;
@@ -447,6 +488,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (MODE == kModePC) tma_prefetch_desc(&tmY);
     }
     if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
     tc_fence_before();
@@ -507,34 +549,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         __syncwarp();
     } else {
         // ---------------- epilogue (both CTAs): this CTA's 128 rows x 256 columns ----------------
+        // Warp w reads TMEM lanes 32*(w%4).. and columns [half*128, half*128+128) in
+        // chunks of 32, loading chunk c+1 (and its scales) before converting chunk c.
+        // Per-channel outputs go through a swizzled shared-memory box and a TMA store.
+        const int ew = warp - 2;
         const int quarter = warp & 3;
-        const int row = quarter * 32 + lane;
+        const int half = ew / 4;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        uint32_t acc_i = 0;
+        uint8_t* stg = sStg + ew * C::STG_PER_WARP * C::STG_BYTES;
+        constexpr int NCH = C::EPI_COLS / 32;
+        uint32_t acc_i = 0, nstore = 0;
         bool ok = true;
         for (int t = cid; t < num_tiles && ok; t += ncl) {
             int mb, nb;
             tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
-            const int m = mb * C::BM + static_cast<int>(rank) * 128 + row;
+            const int m0 = mb * C::BM + static_cast<int>(rank) * 128 + quarter * 32;  // first row of this warp
+            const int m = m0 + lane;
             const bool mvalid = m < p.M;
+            const int nw = nb * C::BN + half * C::EPI_COLS;  // first column of this warp
             const uint32_t b = acc_i % NB;
+            const float sxm = (MODE == kModePC && mvalid) ? __ldg(p.sx + m) : 0.0f;
+            float ws[2][32];
+            if (MODE == kModePC) load_scales32(p.sw, nw, p.N, ws[0]);
             if (!mbar_wait_cluster(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const float sxm = (MODE == kModePC && mvalid) ? __ldg(p.sx + m) : 0.0f;
-#pragma unroll 1
-            for (int c = 0; c < C::BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_base + lane_addr + b * C::BN + c * 32, r);
+            uint32_t r[2][32];
+            const uint32_t tbase = tmem_base + lane_addr + b * C::BN + half * C::EPI_COLS;
+            tmem_ld_32x32b_x32(tbase, r[0]);
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
                 tmem_ld_wait();
-                if (c == C::BN / 32 - 1) {
+                if (c + 1 < NCH) {
+                    tmem_ld_32x32b_x32(tbase + (c + 1) * 32, r[(c + 1) & 1]);
+                    if (MODE == kModePC) load_scales32(p.sw, nw + (c + 1) * 32, p.N, ws[(c + 1) & 1]);
+                } else {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(map_to_rank(&acce[b], 0));
                 }
-                if (mvalid) store_chunk_pc<MODE, TY>(p, r, m, nb * C::BN + c * 32, sxm);
+                const int n0 = nw + c * 32;
+                if (MODE == kModeI32) {
+                    if (mvalid) store_chunk_pc<MODE, TY>(p, r[c & 1], m, n0, sxm);
+                } else {
+                    uint8_t* box = stg + (nstore & 1) * C::STG_BYTES;
+                    if (lane == 0) bulk_wait_read<1>();  // the store issued two boxes ago has read `box`
+                    __syncwarp();
+                    stage_row32<TY>(box, lane, r[c & 1], ws[c & 1], sxm);
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && n0 < p.N && m0 < p.M) {
+                        tma_store_2d(&tmY, box, n0, m0);
+                        bulk_commit();
+                    }
+                    ++nstore;
+                }
             }
             ++acc_i;
         }
+        if (MODE == kModePC && lane == 0) bulk_wait<0>();
     }
 
     tc_fence_before();
@@ -589,11 +661,27 @@ static cudaError_t launch_gemm_cfg(const GemmLaunch& L, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// Output map for the TMA stores of the epilogue: [M][N] 16-bit values, 32 x 32
+// boxes, 64-byte swizzle.
+static bool make_map_out(CUtensorMap* map, void* y, int M, int N, int ydt) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return encode_tensor_map(map, ydt == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, y,
+                             dims, strides, box, estr, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 template <int MODE, typename TY>
 static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
-    CUtensorMap tmA, tmB;
+    CUtensorMap tmA, tmB, tmY;
     if (!make_map_2d(&tmA, L.q, L.K, L.M, kBK, 128, true)) return cudaErrorInvalidValue;
     if (!make_map_2d(&tmB, L.w, L.K, L.N, kBK, PairCfg::BN / 2, true)) return cudaErrorInvalidValue;
+    if (MODE == kModePC) {
+        if (!make_map_out(&tmY, L.y, L.M, L.N, L.ydt)) return cudaErrorInvalidValue;
+    } else {
+        tmY = tmA;  // unused by the INT32 epilogue
+    }
     GemmArgs a;
     a.M = L.M;
     a.N = L.N;
@@ -611,7 +699,7 @@ static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
     auto kern = k_gemm_pair<MODE, TY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<2 * clusters, PairCfg::THREADS, PairCfg::SMEM_BYTES, st>>>(tmA, tmB, a);
+    kern<<<2 * clusters, PairCfg::THREADS, PairCfg::SMEM_BYTES, st>>>(tmA, tmB, tmY, a);
     return cudaGetLastError();
 }
 
