@@ -46,6 +46,22 @@ L2_BYTES = 126 * 1024 * 1024
 INT8_PER_BF16 = 2.0
 
 
+def gemm_traffic():
+    """DRAM bytes per launch of the headline GEMM from the committed ncu capture,
+    or None when the kernel's sources changed since that capture."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "roofline_traffic.json")) as f:
+            rec = json.load(f)
+        m = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                m.update(f.read())
+        return rec["traffic_bytes_per_launch"] if m.hexdigest() == rec["source_sha256"] else None
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -344,7 +360,8 @@ def run_cider(args):
         "breakdown_ms": {"quantize_act": ms_quant, "gemm_pc": ms_gemm},
         "roofline": {"bound": "tensor", "kernel": "k_gemm_sm100 per-channel (tcgen05.mma kind::i8)",
                      "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
-                     "traffic": None,
+                     "traffic": gemm_traffic(), "traffic_unit": "bytes per launch (ncu dram read+write)",
+                     "algorithmic_bytes": M * K + N * K + M * N * 2 + 4 * (M + N),
                      "peak_note": f"dense INT8 = {INT8_PER_BF16:g} x {pk['src']} bf16 cuBLAS burst {pk['bf16']:.1f} TFLOP/s"},
         "e2e": {"value": e2e_tops, "unit": UNIT, "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": x0.numel() * 2, "d2h_bytes_per_step": M * N * 2},
@@ -444,6 +461,45 @@ def bench_rows(device, pk, steps, warmup):
     return out
 
 
+ROW_CASES = {
+    # name: (kind, M, N, K, gs)
+    "pc_m1": ("pc", 1, 10240, 2560, 0), "pc_m128": ("pc", 128, 10240, 2560, 0),
+    "pc_m1024": ("pc", 1024, 10240, 2560, 0), "pc_m4096": ("pc", 4096, 10240, 2560, 0),
+    "pc_m8192": ("pc", 8192, 10240, 2560, 0),
+    "pg128_m1": ("pg", 1, 2560, 10240, 128), "pg128_m4096": ("pg", 4096, 2560, 10240, 128),
+    "pg64_m1": ("pg", 1, 2560, 10240, 64), "pg64_m4096": ("pg", 4096, 2560, 10240, 64),
+    "w4a8_m2048": ("w4", 2048, 12288, 4096, 64),
+}
+
+
+def run_row(args):
+    """One hot-path row alone (for profiling): device time per call, one JSON line."""
+    import w8a8_activation_quantized_b200 as cider
+    from w8a8_activation_quantized_b200 import synth
+    kind, M, N, K, gs = ROW_CASES[args.row]
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    x = torch.from_numpy(synth.activations(M, K, 1000 + M)).to(device)
+    W = torch.from_numpy(synth.weights(N, K, 1001)).to(device)
+    if kind == "pc":
+        w, s = cider.cider_quantize_weight_pc(W)
+        call = lambda y, ws_: cider.cider_w8a8_linear_pc(x, w, s, y=y, workspace=ws_)
+    elif kind == "pg":
+        w, s = cider.cider_quantize_weight_pg(W, gs)
+        call = lambda y, ws_: cider.cider_w8a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)
+    else:
+        w, s = cider.cider_pack_weight_int4_pg(W, gs)
+        call = lambda y, ws_: cider.cider_w4a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)
+    del W
+    y = torch.empty((M, N), dtype=torch.float16, device=device)
+    wsp = torch.empty((max(1, cider.cider_workspace_bytes(M, K)),), dtype=torch.uint8, device=device)
+    ms = graph_time(lambda i: call(y, wsp), args.steps, args.warmup)
+    cider.cider_device_status()
+    print(json.dumps({"row": args.row, "kind": kind, "M": M, "N": N, "K": K, "gs": gs, "ms": ms,
+                      "TOPS": 2.0 * M * N * K / (ms * 1e-3) / 1e12}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -452,11 +508,14 @@ def main():
     ap.add_argument("--impl", choices=["cider", "reference"], default="cider")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--row", choices=sorted(ROW_CASES), help="time one hot-path row alone (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.row:
+        return run_row(args)
     return run_cider(args)
 
 

@@ -361,6 +361,34 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
     return __bfloat162float(v);
 }
 
+// Running max of |v| over 16-bit values, two at a time (exact: max and abs
+// do not round).
+template <typename T>
+struct Pack2;
+template <>
+struct Pack2<__half> {
+    using type = __half2;
+};
+template <>
+struct Pack2<__nv_bfloat16> {
+    using type = __nv_bfloat162;
+};
+
+template <typename T>
+__device__ __forceinline__ typename Pack2<T>::type absmax8(const uint4& v, typename Pack2<T>::type m) {
+    using P = typename Pack2<T>::type;
+    const P* h = reinterpret_cast<const P*>(&v);
+    m = __hmax2(m, __habs2(h[0]));
+    m = __hmax2(m, __habs2(h[1]));
+    m = __hmax2(m, __habs2(h[2]));
+    return __hmax2(m, __habs2(h[3]));
+}
+
+template <typename T>
+__device__ __forceinline__ float absmax_to_f32(typename Pack2<T>::type m) {
+    return fmaxf(to_f32<T>(m.x), to_f32<T>(m.y));
+}
+
 // Eight 16-bit values packed in a uint4 -> eight floats (exact widening).
 template <typename T>
 __device__ __forceinline__ void unpack8_f32(const uint4& v, float (&f)[8]) {

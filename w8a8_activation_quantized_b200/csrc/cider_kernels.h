@@ -59,5 +59,6 @@ cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const
                            const float* sw, int N, int gs, void* y, int ydt, int num_sms,
                            cudaStream_t st);
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t st);
+cudaError_t launch_gemm_grouped(const GemmLaunch& L, cudaStream_t st);
 
 }  // namespace cider

@@ -1,0 +1,90 @@
+// gemm_common.cuh -- pieces shared by the tcgen05 GEMM kernels: tile sizes,
+// kernel arguments, the tile raster, tensor maps and the output staging.
+#pragma once
+
+#include "cider_device.cuh"
+#include "cider_kernels.h"
+
+namespace cider {
+
+constexpr int kBM = 128;          // rows of A per CTA tile
+constexpr int kBK = 128;          // int8 K values per stage = one 128-byte swizzle row
+constexpr int kUmmaK = 32;        // K per kind::i8 MMA
+constexpr int kGroupM = 8;        // tile raster: 8 M-blocks share each N-block in turn
+constexpr int kSmemBudget = 196608;
+constexpr int kSmemMax = 232448;  // dynamic shared memory per CTA on sm_100
+
+struct GemmArgs {
+    int M, N, K;
+    int gs;             // group size (grouped modes)
+    int num_m_blocks, num_n_blocks, num_k_blocks;
+    const float* sx;    // [M]
+    const float* sw;    // [N] or [G][N]
+    void* y;            // [M][N] output (fp16/bf16), or int32 acc / acc_g in test modes
+    unsigned* status;   // device status word
+};
+
+// Raster: kGroupM consecutive M-blocks walk the N-blocks together, so the
+// CTAs running at the same time share B tiles in L2.
+__device__ __forceinline__ void tile_coords(int t, int nm, int nn, int& mb, int& nb) {
+    const int per_group = kGroupM * nn;
+    const int grp = t / per_group;
+    const int first_m = grp * kGroupM;
+    const int gm = min(nm - first_m, kGroupM);
+    const int r = t % per_group;
+    mb = first_m + r % gm;
+    nb = r / gm;
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Eight outputs of one row packed into a 16-byte vector.
+template <typename TY>
+__device__ __forceinline__ uint4 pack8_out(const float* v) {
+    uint4 o;
+    o.x = pack2_out<TY>(v[0], v[1]);
+    o.y = pack2_out<TY>(v[2], v[3]);
+    o.z = pack2_out<TY>(v[4], v[5]);
+    o.w = pack2_out<TY>(v[6], v[7]);
+    return o;
+}
+
+// Row `r` of a 32 x 32 staging box of 16-bit outputs, laid out for the TMA
+// 64-byte swizzle: 16-byte chunk j of row r lands at chunk j ^ ((r >> 1) & 3),
+// so the 32 lanes writing 32 rows hit distinct banks.
+template <typename TY>
+__device__ __forceinline__ void stage_row32_f(uint8_t* box, int r, const float (&v)[32]) {
+    uint8_t* row = box + r * 64;
+    const int sw = (r >> 1) & 3;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(row + ((j ^ sw) << 4)) = pack8_out<TY>(v + 8 * j);
+}
+
+// ---------------------------------------------------------------------------
+// Host-side tensor maps
+// ---------------------------------------------------------------------------
+// 2-D uint8 map over a row-major [rows][inner] byte matrix.
+inline bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                        uint32_t box_rows, bool swizzle128) {
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return encode_tensor_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Output map for the epilogues' TMA stores: [M][N] 16-bit values, 32 x 32
+// boxes, 64-byte swizzle.
+inline bool make_map_out(CUtensorMap* map, void* y, int M, int N, int ydt) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return encode_tensor_map(map, ydt == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, y,
+                             dims, strides, box, estr, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+}  // namespace cider

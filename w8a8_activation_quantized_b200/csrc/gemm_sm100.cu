@@ -2,91 +2,49 @@
 // cores (tcgen05.mma kind::i8), fused with the dequant epilogue.
 //
 // What it computes (juejin post "在Mac上跑大模型，MLX 不是终点", sections
-// "INT8 TensorOps 内核设计" and "三种量化粒度的实现"; Cider README, table "量化"):
-//   per-channel  y[m,n] = acc[m,n] * scale_x[m] * scale_w[n]
-//   per-group    y[m,n] = scale_x[m] * sum_g acc_g[m,n] * scale_w[g][n]
-//   W4A8         the per-group form with INT4 weights unpacked to INT8 on chip
-// acc = sum_k q[m,k] * w[n,k] in INT32, exact.
+// "INT8 TensorOps 内核设计" and "W8A8 对称量化"; Cider README, table "量化"):
+//   per-channel  y[m,n] = acc[m,n] * scale_x[m] * scale_w[n],
+//   acc = sum_k q[m,k] * w[n,k] in INT32, exact.
+// (The per-group and W4A8 forms are in gemm_grouped.cu.)
 //
-// Design (sm_100a, one CTA per SM, persistent over output tiles):
-//  * tile BM=128 x BN (256 per-channel, 128 per-group) x BK=128 int8 per stage;
-//    A = q [M][K] and B = w [N][K] are both K-major and land in shared
-//    memory through TMA with the 128-byte swizzle the UMMA descriptors expect;
-//  * warp 0 (one lane) issues the TMA loads into a ring of mbarrier-guarded
-//    stages; warp 1 (one lane) issues tcgen05.mma into tensor-memory (TMEM)
-//    INT32 accumulators and releases stages with tcgen05.commit;
-//  * per-channel: two TMEM accumulators of BN columns, so the epilogue of
-//    tile i overlaps the main loop of tile i+1;
-//  * per-group: every group of gs (64 or 128) K values gets its own INT32
-//    partial in a ring of TMEM buffers; the epilogue warps read each partial
-//    (tcgen05.ld), rescale it by its group's weight scale in fp32 and keep the
-//    running sums in registers -- the "piecewise multiply" of the pages;
-//  * W4A8: packed [N][K/2] tiles arrive by TMA unswizzled; four converter warps
-//    expand each nibble to int8 (nibble - 8) into the swizzled B stage, fence
-//    the writes to the async proxy, and hand the stage to the MMA warp;
-//  * every mbarrier wait is bounded (see mbar_wait).
+// Two kernels, one CTA (or CTA pair) per SM, persistent over output tiles:
+//  * k_gemm_pair -- the large-M kernel: a 256 x 256 tile per cluster of two
+//    CTAs with tcgen05.mma.cta_group::2 (see its comment);
+//  * k_gemm_sm100 -- single-CTA 128 x BN tiles (BN 256 or 128) for shapes with
+//    too few 256 x 256 tiles to fill the GPU.
+// Common to both: A = q [M][K] and B = w [N][K] are K-major and land in shared
+// memory through TMA with the 128-byte swizzle the UMMA descriptors expect;
+// warp 0 (one lane) issues the TMA loads into a ring of mbarrier-guarded
+// stages of 128 K values; warp 1 (one lane) issues the MMAs into INT32 TMEM
+// accumulators and releases stages with tcgen05.commit; two accumulators let
+// the epilogue of one tile overlap the main loop of the next.  Every mbarrier
+// wait is bounded (mbar_wait).
 //
 // The pages' own tiles (BM128 BN128 BK512 on Apple TensorOps) are prior art;
 // the sizes here follow from TMEM (512 columns x 128 lanes x 32 bit per SM),
-// the 128x256x32 kind::i8 MMA shape and 227 KB of shared memory.
-#include "cider_device.cuh"
-#include "cider_kernels.h"
+// the 256x256x32 kind::i8 pair MMA shape and 227 KB of shared memory.
+#include "gemm_common.cuh"
 
 namespace cider {
 
-constexpr int kBM = 128;
-constexpr int kBK = 128;      // int8 K values per stage = one 128-byte swizzle row
-constexpr int kUmmaK = 32;    // K per kind::i8 MMA
-constexpr int kGroupM = 8;    // tile raster: 8 M-blocks share each N-block in turn
-constexpr int kSmemBudget = 196608;
-
+// Single-CTA per-channel (and INT32 test) kernel: 128 x BN tiles.
 template <int BN_, int MODE_>
 struct GemmCfg {
     static constexpr int BN = BN_;
     static constexpr int MODE = MODE_;
-    static constexpr bool GROUPED = (MODE == kModePG || MODE == kModeW4 || MODE == kModeI32G);
-    static constexpr bool W4 = (MODE == kModeW4);
-    static constexpr int EPI_WARPS = GROUPED ? 8 : 4;
-    static constexpr int CONV_WARPS = W4 ? 4 : 0;
-    static constexpr int THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
+    static constexpr int EPI_WARPS = 4;
+    static constexpr int THREADS = 32 * (2 + EPI_WARPS);
     static constexpr int A_BYTES = kBM * kBK;
     static constexpr int B_BYTES = BN * kBK;
-    static constexpr int BP_BYTES = W4 ? BN * kBK / 2 : 0;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + BP_BYTES;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = (kSmemBudget / STAGE_BYTES) > 8 ? 8 : (kSmemBudget / STAGE_BYTES);
-    static constexpr int ACC_BUFS = GROUPED ? 512 / BN : 2;
+    static constexpr int ACC_BUFS = 2;
     static constexpr int TMEM_COLS = ACC_BUFS * BN;  // 256 or 512
-    static constexpr int EPI_COLS = GROUPED ? BN / 2 : BN;  // columns per epilogue thread
-    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 2 * ACC_BUFS) + 16;
+    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * ACC_BUFS) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
     static_assert(BN % 32 == 0 && BN <= 256, "BN");
     static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
-    static_assert(STAGES >= 2, "stages");
 };
-
-struct GemmArgs {
-    int M, N, K;
-    int gs;             // group size (grouped modes)
-    int num_m_blocks, num_n_blocks, num_k_blocks;
-    const float* sx;    // [M]
-    const float* sw;    // [N] or [G][N]
-    void* y;            // [M][N] output (fp16/bf16), or int32 acc / acc_g in test modes
-    unsigned* status;   // device status word
-};
-
-__device__ __forceinline__ void tile_coords(int t, int nm, int nn, int& mb, int& nb) {
-    const int per_group = kGroupM * nn;
-    const int grp = t / per_group;
-    const int first_m = grp * kGroupM;
-    const int gm = min(nm - first_m, kGroupM);
-    const int r = t % per_group;
-    mb = first_m + r % gm;
-    nb = r / gm;
-}
-
-__device__ __forceinline__ void fence_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 template <typename TY>
 __device__ __forceinline__ void store_row8(TY* dst, const float (&v)[8]) {
@@ -137,11 +95,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + S * Cfg::A_BYTES;
-    uint8_t* sBP = sB + S * Cfg::B_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sBP + S * Cfg::BP_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * Cfg::B_BYTES);
     uint64_t* empty = full + S;
-    uint64_t* conv = empty + S;
-    uint64_t* accf = conv + S;
+    uint64_t* accf = empty + S;
     uint64_t* acce = accf + NB;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + NB);
     __shared__ int s_abort;
@@ -155,7 +111,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&conv[s], Cfg::CONV_WARPS * 32);
         }
         for (int b = 0; b < NB; ++b) {
             mbar_init(&accf[b], 1);
@@ -180,19 +135,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            const uint32_t tx = Cfg::A_BYTES + (Cfg::W4 ? Cfg::BP_BYTES : Cfg::B_BYTES);
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 int mb, nb;
                 tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
                 for (int kb = 0; kb < p.num_k_blocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full[stage], tx);
+                    mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
                     tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, &full[stage], kb * kBK, mb * kBM);
-                    if (Cfg::W4)
-                        tma_load_2d(sBP + stage * Cfg::BP_BYTES, &tmB, &full[stage], kb * (kBK / 2), nb * BN);
-                    else
-                        tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, &full[stage], kb * kBK, nb * BN);
+                    tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, &full[stage], kb * kBK, nb * BN);
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -205,171 +156,57 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             uint32_t phase = 0;
             uint32_t acc_i = 0;  // accumulator-buffer uses so far
             bool ok = true;
-            const int G = Cfg::GROUPED ? p.K / p.gs : 0;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                int g = 0;  // next group of this tile (grouped modes)
-                if (!Cfg::GROUPED) {
-                    const uint32_t b = acc_i % NB;
-                    if (!mbar_wait(&acce[b], ((acc_i / NB) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                }
-                for (int kb = 0; kb < p.num_k_blocks && ok; ++kb) {
+                const uint32_t b = acc_i % NB;
+                if (!mbar_wait(&acce[b], ((acc_i / NB) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem_base + b * BN;
+                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
                     if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
-                    if (Cfg::W4 && !mbar_wait(&conv[stage], phase, p.status, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * Cfg::A_BYTES));
                     const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * Cfg::B_BYTES));
-                    if (!Cfg::GROUPED) {
-                        const uint32_t d = tmem_base + (acc_i % NB) * BN;
 #pragma unroll
-                        for (int kk = 0; kk < kBK / kUmmaK; ++kk)
-                            umma_i8(d, adesc + (kk * kUmmaK >> 4), bdesc + (kk * kUmmaK >> 4), idesc,
-                                    (kb > 0 || kk > 0) ? 1u : 0u);
-                    } else {
-                        const int gpk = kBK / p.gs;  // groups per stage: 1 or 2
-                        const int steps = p.gs / kUmmaK;
-                        for (int j = 0; j < gpk && g < G; ++j, ++g) {
-                            const uint32_t b = acc_i % NB;
-                            if (!mbar_wait(&acce[b], ((acc_i / NB) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
-                            tc_fence_after();
-                            const uint32_t d = tmem_base + b * BN;
-                            for (int kk = 0; kk < steps; ++kk) {
-                                const int off = (j * steps + kk) * kUmmaK;
-                                umma_i8(d, adesc + (off >> 4), bdesc + (off >> 4), idesc, kk > 0 ? 1u : 0u);
-                            }
-                            umma_commit(&accf[b]);
-                            ++acc_i;
-                        }
-                    }
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+                        umma_i8(d, adesc + (kk * kUmmaK >> 4), bdesc + (kk * kUmmaK >> 4), idesc,
+                                (kb > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty[stage]);
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
-                if (!Cfg::GROUPED && ok) {
-                    umma_commit(&accf[acc_i % NB]);
-                    ++acc_i;
-                }
+                if (!ok) break;
+                umma_commit(&accf[b]);
+                ++acc_i;
             }
         }
         __syncwarp();
-    } else if (warp < 2 + Cfg::EPI_WARPS) {
+    } else {
         // ------------------------------ epilogue ----------------------------------
         const int quarter = warp & 3;  // TMEM lanes this warp may access
-        const int colhalf = Cfg::GROUPED ? (warp - 2) / 4 : 0;
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         uint32_t acc_i = 0;
         bool ok = true;
-        const int G = Cfg::GROUPED ? p.K / p.gs : 0;
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
             int mb, nb;
             tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
             const int m = mb * kBM + row;
             const bool mvalid = m < p.M;
-            const int n_base = nb * BN + colhalf * Cfg::EPI_COLS;
-            if (!Cfg::GROUPED) {
-                const uint32_t b = acc_i % NB;
-                if (!mbar_wait(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const float sxm = (Cfg::MODE == kModePC && mvalid) ? __ldg(p.sx + m) : 0.0f;
+            const uint32_t b = acc_i % NB;
+            if (!mbar_wait(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const float sxm = (Cfg::MODE == kModePC && mvalid) ? __ldg(p.sx + m) : 0.0f;
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tmem_base + lane_addr + b * BN + c * 32, r);
-                    tmem_ld_wait();
-                    if (c == BN / 32 - 1) {
-                        tc_fence_before();
-                        mbar_arrive(&acce[b]);
-                    }
-                    if (mvalid) store_chunk_pc<Cfg::MODE, TY>(p, r, m, n_base + c * 32, sxm);
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + b * BN + c * 32, r);
+                tmem_ld_wait();
+                if (c == BN / 32 - 1) {
+                    tc_fence_before();
+                    mbar_arrive(&acce[b]);
                 }
-                ++acc_i;
-            } else {
-                float sum[Cfg::EPI_COLS];
-#pragma unroll
-                for (int j = 0; j < Cfg::EPI_COLS; ++j) sum[j] = 0.0f;
-                for (int g = 0; g < G; ++g) {
-                    const uint32_t b = acc_i % NB;
-                    if (!mbar_wait(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    const float* swg = p.sw + static_cast<int64_t>(g) * p.N;
-#pragma unroll
-                    for (int c = 0; c < Cfg::EPI_COLS / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(tmem_base + lane_addr + b * BN + colhalf * Cfg::EPI_COLS + c * 32, r);
-                        tmem_ld_wait();
-                        if (c == Cfg::EPI_COLS / 32 - 1) {
-                            tc_fence_before();
-                            mbar_arrive(&acce[b]);
-                        }
-                        const int n0 = n_base + c * 32;
-                        if (Cfg::MODE == kModeI32G) {
-                            if (mvalid) {
-                                int32_t* out = static_cast<int32_t*>(p.y) +
-                                               (static_cast<int64_t>(g) * p.M + m) * p.N;
-#pragma unroll
-                                for (int j = 0; j < 8; ++j)
-                                    if (n0 + 4 * j < p.N)
-                                        *reinterpret_cast<uint4*>(out + n0 + 4 * j) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                                if (n0 + 4 * j < p.N) w4 = __ldg(reinterpret_cast<const float4*>(swg + n0 + 4 * j));
-                                sum[c * 32 + 4 * j + 0] = fmaf(static_cast<float>(static_cast<int32_t>(r[4 * j + 0])), w4.x, sum[c * 32 + 4 * j + 0]);
-                                sum[c * 32 + 4 * j + 1] = fmaf(static_cast<float>(static_cast<int32_t>(r[4 * j + 1])), w4.y, sum[c * 32 + 4 * j + 1]);
-                                sum[c * 32 + 4 * j + 2] = fmaf(static_cast<float>(static_cast<int32_t>(r[4 * j + 2])), w4.z, sum[c * 32 + 4 * j + 2]);
-                                sum[c * 32 + 4 * j + 3] = fmaf(static_cast<float>(static_cast<int32_t>(r[4 * j + 3])), w4.w, sum[c * 32 + 4 * j + 3]);
-                            }
-                        }
-                    }
-                    ++acc_i;
-                }
-                if (!ok) break;
-                if (Cfg::MODE != kModeI32G && mvalid) {
-                    const float sxm = __ldg(p.sx + m);
-                    TY* out = static_cast<TY*>(p.y) + static_cast<int64_t>(m) * p.N;
-#pragma unroll
-                    for (int j = 0; j < Cfg::EPI_COLS / 8; ++j) {
-                        if (n_base + 8 * j < p.N) {
-                            float v[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) v[e] = sum[8 * j + e] * sxm;
-                            store_row8<TY>(out + n_base + 8 * j, v);
-                        }
-                    }
-                }
+                if (mvalid) store_chunk_pc<Cfg::MODE, TY>(p, r, m, nb * BN + c * 32, sxm);
             }
-        }
-    } else {
-        // --------------------- W4A8 converter warps: INT4 -> INT8 ------------------
-        if (Cfg::W4) {
-            const int ct = threadIdx.x - 32 * (2 + Cfg::EPI_WARPS);  // 0..127
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
-                    const uint8_t* src = sBP + stage * Cfg::BP_BYTES;  // [BN][64] packed, row-major
-                    uint8_t* dst = sB + stage * Cfg::B_BYTES;          // [BN][128] int8, 128B swizzle
-#pragma unroll
-                    for (int it = 0; it < BN * 4 / 128; ++it) {
-                        const int item = ct + 128 * it;
-                        const int r = item >> 2, j = item & 3;  // row, 16-byte packed chunk
-                        const uint4 pk = *reinterpret_cast<const uint4*>(src + r * 64 + j * 16);
-                        const uint2 u0 = unpack_int4x8(pk.x), u1 = unpack_int4x8(pk.y);
-                        const uint2 u2 = unpack_int4x8(pk.z), u3 = unpack_int4x8(pk.w);
-                        uint8_t* row = dst + r * 128;
-                        const int sw = r & 7;
-                        *reinterpret_cast<uint4*>(row + (((2 * j) ^ sw) << 4)) = make_uint4(u0.x, u0.y, u1.x, u1.y);
-                        *reinterpret_cast<uint4*>(row + (((2 * j + 1) ^ sw) << 4)) = make_uint4(u2.x, u2.y, u3.x, u3.y);
-                    }
-                    fence_async_smem();
-                    mbar_arrive(&conv[stage]);
-                    if (++stage == S) { stage = 0; phase ^= 1u; }
-                }
-            }
+            ++acc_i;
         }
     }
 
@@ -618,28 +455,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Host side: tensor maps and launch.
+// Host side: launch.
 // ---------------------------------------------------------------------------
-static bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
-                        uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
-    cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {inner};  // bytes (uint8 elements)
-    cuuint32_t box[2] = {box_inner, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return encode_tensor_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
-                             strides, box, estr,
-                             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
-}
-
 template <typename Cfg, typename TY>
 static cudaError_t launch_gemm_cfg(const GemmLaunch& L, cudaStream_t st) {
     CUtensorMap tmA, tmB;
     if (!make_map_2d(&tmA, L.q, L.K, L.M, kBK, kBM, true)) return cudaErrorInvalidValue;
-    if (Cfg::W4) {
-        if (!make_map_2d(&tmB, L.w, L.K / 2, L.N, kBK / 2, Cfg::BN, false)) return cudaErrorInvalidValue;
-    } else {
-        if (!make_map_2d(&tmB, L.w, L.K, L.N, kBK, Cfg::BN, true)) return cudaErrorInvalidValue;
-    }
+    if (!make_map_2d(&tmB, L.w, L.K, L.N, kBK, Cfg::BN, true)) return cudaErrorInvalidValue;
     GemmArgs a;
     a.M = L.M;
     a.N = L.N;
@@ -659,17 +481,6 @@ static cudaError_t launch_gemm_cfg(const GemmLaunch& L, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(tmA, tmB, a);
     return cudaGetLastError();
-}
-
-// Output map for the TMA stores of the epilogue: [M][N] 16-bit values, 32 x 32
-// boxes, 64-byte swizzle.
-static bool make_map_out(CUtensorMap* map, void* y, int M, int N, int ydt) {
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
-    cuuint32_t box[2] = {32, 32};
-    cuuint32_t estr[2] = {1, 1};
-    return encode_tensor_map(map, ydt == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, y,
-                             dims, strides, box, estr, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 template <int MODE, typename TY>
@@ -705,23 +516,19 @@ static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
 
 template <int MODE, typename TY>
 static cudaError_t launch_gemm_mode(const GemmLaunch& L, cudaStream_t st) {
-    if constexpr (MODE == kModePC || MODE == kModeI32) {
-        if (L.variant == kGemmPair) return launch_gemm_pair<MODE, TY>(L, st);
-        if (L.variant == kGemmSingle128) return launch_gemm_cfg<GemmCfg<128, MODE>, TY>(L, st);
-        return launch_gemm_cfg<GemmCfg<256, MODE>, TY>(L, st);
-    } else {
-        return launch_gemm_cfg<GemmCfg<128, MODE>, TY>(L, st);
-    }
+    if (L.variant == kGemmPair) return launch_gemm_pair<MODE, TY>(L, st);
+    if (L.variant == kGemmSingle128) return launch_gemm_cfg<GemmCfg<128, MODE>, TY>(L, st);
+    return launch_gemm_cfg<GemmCfg<256, MODE>, TY>(L, st);
 }
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t st) {
     const bool bf = (L.ydt == 1);
     switch (L.mode) {
         case kModePC: return bf ? launch_gemm_mode<kModePC, __nv_bfloat16>(L, st) : launch_gemm_mode<kModePC, __half>(L, st);
-        case kModePG: return bf ? launch_gemm_mode<kModePG, __nv_bfloat16>(L, st) : launch_gemm_mode<kModePG, __half>(L, st);
-        case kModeW4: return bf ? launch_gemm_mode<kModeW4, __nv_bfloat16>(L, st) : launch_gemm_mode<kModeW4, __half>(L, st);
         case kModeI32: return launch_gemm_mode<kModeI32, __half>(L, st);
-        case kModeI32G: return launch_gemm_mode<kModeI32G, __half>(L, st);
+        case kModePG:
+        case kModeW4:
+        case kModeI32G: return launch_gemm_grouped(L, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -35,7 +35,7 @@ __device__ __forceinline__ void quant_store8(const float (&f)[8], float scale, f
 // 128-thread CTAs (4 rows each) and NV sized to K keep registers low, so many
 // warps per SM have loads in flight while others quantize.
 template <typename T, int NV>
-__global__ void __launch_bounds__(128, (NV <= 10 ? 8 : 5)) k_quantize_warp(const T* __restrict__ x, int64_t M, int K,
+__global__ void __launch_bounds__(128, (NV <= 10 ? 6 : 4)) k_quantize_warp(const T* __restrict__ x, int64_t M, int K,
                                                        int8_t* __restrict__ q,
                                                        float* __restrict__ sx) {
     const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -44,19 +44,16 @@ __global__ void __launch_bounds__(128, (NV <= 10 ? 8 : 5)) k_quantize_warp(const
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
     const int nch = K >> 3;
     uint4 v[NV];
-    float amax = 0.0f;
+    // all loads of the row in flight before any of them is used
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
         const int c = lane + 32 * i;
-        if (c < nch) {
-            v[i] = __ldcs(xr + c);
-            float f[8];
-            unpack8_f32<T>(v[i], f);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
-        }
+        v[i] = c < nch ? __ldcs(xr + c) : make_uint4(0, 0, 0, 0);
     }
-    amax = warp_max(amax);
+    typename Pack2<T>::type m2 = {};
+#pragma unroll
+    for (int i = 0; i < NV; ++i) m2 = absmax8<T>(v[i], m2);
+    const float amax = warp_max(absmax_to_f32<T>(m2));
     const float s = act_scale(amax);
     const float rs = act_rcp(s);
     if (lane == 0) sx[row] = s;
@@ -91,14 +88,12 @@ __global__ void __launch_bounds__(256) k_quantize_cta(const T* __restrict__ x, i
 #pragma unroll
         for (int i = 0; i < R; ++i) {
             const int c = tid + 256 * i;
-            if (c < nch) {
-                v[i] = __ldcs(xr + c);
-                float f[8];
-                unpack8_f32<T>(v[i], f);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
-            }
+            v[i] = c < nch ? __ldcs(xr + c) : make_uint4(0, 0, 0, 0);
         }
+        typename Pack2<T>::type m2 = {};
+#pragma unroll
+        for (int i = 0; i < R; ++i) m2 = absmax8<T>(v[i], m2);
+        amax = absmax_to_f32<T>(m2);
     } else {
         for (int c = tid; c < nch; c += 256) {
             float f[8];
@@ -185,13 +180,20 @@ __global__ void __launch_bounds__(256) k_silu_mul_quantize(const T* __restrict__
     const int nch = F >> 3;
     uint4 av[NV];
     float amax = 0.0f;
+    uint4 gv[NV], uv[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = tid + 256 * i;
+        gv[i] = c < nch ? __ldcs(gr + c) : make_uint4(0, 0, 0, 0);
+        uv[i] = c < nch ? __ldcs(ur + c) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
         const int c = tid + 256 * i;
         if (c < nch) {
             float g[8], u[8];
-            unpack8_f32<T>(__ldcs(gr + c), g);
-            unpack8_f32<T>(__ldcs(ur + c), u);
+            unpack8_f32<T>(gv[i], g);
+            unpack8_f32<T>(uv[i], u);
             T* ah = reinterpret_cast<T*>(&av[i]);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
