@@ -96,6 +96,19 @@ __device__ __forceinline__ void cp_async_wait() {
 
 // 10 or 12 warps: three of them share a 16K-register SM sub-partition, so
 // the launch bound caps registers at 168 per thread.
+// Test mode: 32 per-group INT32 partials of one row (preset removed).
+__device__ __forceinline__ void store_partial32(const GemmArgs& p, const uint32_t (&r)[32], int g, int m, bool mvalid,
+                                                int n0) {
+    if (!mvalid) return;
+    int32_t* out = static_cast<int32_t*>(p.y) + (static_cast<int64_t>(g) * p.M + m) * p.N;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (n0 + 4 * j < p.N)
+            *reinterpret_cast<int4*>(out + n0 + 4 * j) =
+                make_int4(static_cast<int>(r[4 * j] - kPartialBias), static_cast<int>(r[4 * j + 1] - kPartialBias),
+                          static_cast<int>(r[4 * j + 2] - kPartialBias), static_cast<int>(r[4 * j + 3] - kPartialBias));
+}
+
 template <int MODE, typename TY>
 __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
     k_gemm_grouped(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -228,24 +241,32 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
         if (lane == 0)
             for (int b = 0; b < NB; ++b) mbar_arrive(&acce[b]);
 
-        // scale prefetch: group index gi -> (tile, group) of this CTA's sequence
-        const int tiles_mine = num_tiles > static_cast<int>(blockIdx.x)
-                                   ? (num_tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
-                                   : 0;
-        const int total_groups = tiles_mine * G;
-        auto prefetch = [&](int gi) {
-            if (MODE != kModeI32G && gi < total_groups && lane < C::EPI_COLS / 4) {
-                const int t = static_cast<int>(blockIdx.x) + (gi / G) * static_cast<int>(gridDim.x);
-                const int g = gi % G;
+        // Scale prefetch runs kScaleSlots-1 groups ahead of the rescale along this
+        // CTA's (tile, group) sequence; a running pointer avoids divisions.
+        int pf_t = blockIdx.x, pf_g = 0, pf_slot = 0, pf_col = 0;
+        auto pf_tile = [&]() {
+            if (pf_t < num_tiles) {
                 int mb, nb;
-                tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
-                const int n = nb * BN + half * C::EPI_COLS + 4 * lane;
-                const float* src = p.sw + static_cast<int64_t>(g) * p.N + (n < p.N ? n : 0);
-                cp_async16(scl + (gi % kScaleSlots) * C::SCL_BYTES + 16 * lane, src, n < p.N ? 16u : 0u);
+                tile_coords(pf_t, p.num_m_blocks, p.num_n_blocks, mb, nb);
+                pf_col = nb * BN + half * C::EPI_COLS + 4 * lane;
+            }
+        };
+        pf_tile();
+        auto prefetch = [&]() {
+            if (MODE != kModeI32G && pf_t < num_tiles && lane < C::EPI_COLS / 4) {
+                const bool in = pf_col < p.N;
+                const float* src = p.sw + static_cast<int64_t>(pf_g) * p.N + (in ? pf_col : 0);
+                cp_async16(scl + pf_slot * C::SCL_BYTES + 16 * lane, src, in ? 16u : 0u);
             }
             cp_async_commit();
+            pf_slot = (pf_slot + 1) % kScaleSlots;
+            if (++pf_g == G) {
+                pf_g = 0;
+                pf_t += gridDim.x;
+                pf_tile();
+            }
         };
-        for (int gi = 0; gi < kScaleSlots - 1; ++gi) prefetch(gi);
+        for (int i = 0; i < kScaleSlots - 1; ++i) prefetch();
 
         const uint64_t neg_bias2 = pack_u32x2(__float_as_uint(-12582912.0f), __float_as_uint(-12582912.0f));
         uint32_t acc_i = 0, nstore = 0;
@@ -261,7 +282,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < C::EPI_COLS / 2; ++j) sum2[j] = 0;
             for (int g = 0; g < G; ++g) {
-                prefetch(static_cast<int>(acc_i) + kScaleSlots - 1);
+                prefetch();
                 const uint32_t b = acc_i % NB;
                 if (!mbar_wait(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
                 tc_fence_after();
@@ -273,37 +294,31 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
                     cp_async_wait<kScaleSlots - 1>();  // this group's scales have landed
                     __syncwarp();
                 }
+                uint32_t r[2][32];
+                tmem_ld_32x32b_x32(taddr, r[0]);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(taddr + 32 * h, r);
                     tmem_ld_wait();
                     tmem_st_32x32b_x32(taddr + 32 * h, kPartialBias);
-                    if (h == 1) {
+                    if (h == 0) {
+                        tmem_ld_32x32b_x32(taddr + 32, r[1]);  // in flight while half 0 is rescaled
+                    } else {
                         tmem_st_wait();
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&acce[b]);
                     }
                     if (MODE == kModeI32G) {
-                        if (mvalid) {
-                            int32_t* out = static_cast<int32_t*>(p.y) + (static_cast<int64_t>(g) * p.M + m) * p.N;
-#pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                if (nw + 32 * h + 4 * j < p.N)
-                                    *reinterpret_cast<int4*>(out + nw + 32 * h + 4 * j) = make_int4(
-                                        static_cast<int>(r[4 * j] - kPartialBias), static_cast<int>(r[4 * j + 1] - kPartialBias),
-                                        static_cast<int>(r[4 * j + 2] - kPartialBias), static_cast<int>(r[4 * j + 3] - kPartialBias));
-                        }
+                        store_partial32(p, r[h], g, m, mvalid, nw + 32 * h);
                     } else {
                         // each 16-byte scale load feeds two packed FMAs
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const ulonglong2 sc = s2[8 * h + j];
-                            sum2[16 * h + 2 * j] =
-                                f32x2_fma(f32x2_add(pack_u32x2(r[4 * j], r[4 * j + 1]), neg_bias2), sc.x, sum2[16 * h + 2 * j]);
-                            sum2[16 * h + 2 * j + 1] = f32x2_fma(f32x2_add(pack_u32x2(r[4 * j + 2], r[4 * j + 3]), neg_bias2),
-                                                                 sc.y, sum2[16 * h + 2 * j + 1]);
+                            sum2[16 * h + 2 * j] = f32x2_fma(f32x2_add(pack_u32x2(r[h][4 * j], r[h][4 * j + 1]), neg_bias2),
+                                                             sc.x, sum2[16 * h + 2 * j]);
+                            sum2[16 * h + 2 * j + 1] = f32x2_fma(
+                                f32x2_add(pack_u32x2(r[h][4 * j + 2], r[h][4 * j + 3]), neg_bias2), sc.y, sum2[16 * h + 2 * j + 1]);
                         }
                     }
                 }
