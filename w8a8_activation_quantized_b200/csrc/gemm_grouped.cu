@@ -81,6 +81,22 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, uint32_t v) {
         "r"(v)
         : "memory");
 }
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+        "r"(v)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 16 bytes global -> shared, zero-filled when `bytes` is 0.
@@ -96,13 +112,35 @@ __device__ __forceinline__ void cp_async_wait() {
 
 // 10 or 12 warps: three of them share a 16K-register SM sub-partition, so
 // the launch bound caps registers at 168 per thread.
-// Test mode: 32 per-group INT32 partials of one row (preset removed).
-__device__ __forceinline__ void store_partial32(const GemmArgs& p, const uint32_t (&r)[32], int g, int m, bool mvalid,
+// Scales of 4 consecutive columns as two packed pairs; the load is ordered
+// (volatile) so the compiler keeps scale registers short-lived.
+__device__ __forceinline__ void lds_scale4(const uint8_t* p, uint64_t& a, uint64_t& b) {
+    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(smem_u32(p)) : "memory");
+}
+
+// sum += (partial - preset) * scale for 16 columns, two per instruction; the
+// next 16 bytes of scales are loaded while the current ones are used.
+__device__ __forceinline__ void rescale16(uint64_t* sum2, const uint32_t (&r)[16], const uint8_t* scales,
+                                          uint64_t neg_bias2) {
+    uint64_t a0, a1, b0, b1;
+    lds_scale4(scales, a0, a1);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (j + 1 < 4) lds_scale4(scales + 16 * (j + 1), b0, b1);
+        sum2[2 * j] = f32x2_fma(f32x2_add(pack_u32x2(r[4 * j], r[4 * j + 1]), neg_bias2), a0, sum2[2 * j]);
+        sum2[2 * j + 1] = f32x2_fma(f32x2_add(pack_u32x2(r[4 * j + 2], r[4 * j + 3]), neg_bias2), a1, sum2[2 * j + 1]);
+        a0 = b0;
+        a1 = b1;
+    }
+}
+
+// Test mode: 16 per-group INT32 partials of one row (preset removed).
+__device__ __forceinline__ void store_partial16(const GemmArgs& p, const uint32_t (&r)[16], int g, int m, bool mvalid,
                                                 int n0) {
     if (!mvalid) return;
     int32_t* out = static_cast<int32_t*>(p.y) + (static_cast<int64_t>(g) * p.M + m) * p.N;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
         if (n0 + 4 * j < p.N)
             *reinterpret_cast<int4*>(out + n0 + 4 * j) =
                 make_int4(static_cast<int>(r[4 * j] - kPartialBias), static_cast<int>(r[4 * j + 1] - kPartialBias),
@@ -281,48 +319,48 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
             uint64_t sum2[C::EPI_COLS / 2];
 #pragma unroll
             for (int j = 0; j < C::EPI_COLS / 2; ++j) sum2[j] = 0;
-            for (int g = 0; g < G; ++g) {
+            // Each group's 64 columns go in four 16-column steps; the TMEM load of
+            // the next step (crossing into the next group) is in flight while the
+            // current step is rescaled, and the preset restore completes behind the
+            // last step.
+            uint32_t rr[2][16];
+            {
+                const uint32_t b0 = acc_i % NB;
+                if (!mbar_wait(&accf[b0], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                tmem_ld_32x32b_x16(tmem_base + lane_addr + b0 * BN + half * C::EPI_COLS, rr[0]);
+            }
+            for (int g = 0; g < G && ok; ++g) {
                 prefetch();
                 const uint32_t b = acc_i % NB;
-                if (!mbar_wait(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                // the two 32-column halves one after the other: load, restore the
-                // preset, rescale (32 partials live at a time)
                 const uint32_t taddr = tmem_base + lane_addr + b * BN + half * C::EPI_COLS;
-                const ulonglong2* s2 = reinterpret_cast<const ulonglong2*>(scl + (acc_i % kScaleSlots) * C::SCL_BYTES);
+                const uint8_t* slot = scl + (acc_i % kScaleSlots) * C::SCL_BYTES;
                 if (MODE != kModeI32G) {
                     cp_async_wait<kScaleSlots - 1>();  // this group's scales have landed
                     __syncwarp();
                 }
-                uint32_t r[2][32];
-                tmem_ld_32x32b_x32(taddr, r[0]);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    tmem_ld_wait();
-                    tmem_st_32x32b_x32(taddr + 32 * h, kPartialBias);
-                    if (h == 0) {
-                        tmem_ld_32x32b_x32(taddr + 32, r[1]);  // in flight while half 0 is rescaled
-                    } else {
-                        tmem_st_wait();
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&acce[b]);
+                for (int c = 0; c < 4; ++c) {
+                    tmem_ld_wait();  // rr[c & 1] = columns 16c .. 16c+15 of group g
+                    tmem_st_32x32b_x16(taddr + 16 * c, kPartialBias);
+                    if (c < 3) {
+                        tmem_ld_32x32b_x16(taddr + 16 * (c + 1), rr[(c + 1) & 1]);
+                    } else if (g + 1 < G) {  // first step of the next group
+                        const uint32_t bn = (acc_i + 1) % NB;
+                        if (!mbar_wait(&accf[bn], ((acc_i + 1) / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        tmem_ld_32x32b_x16(tmem_base + lane_addr + bn * BN + half * C::EPI_COLS, rr[0]);
                     }
-                    if (MODE == kModeI32G) {
-                        store_partial32(p, r[h], g, m, mvalid, nw + 32 * h);
-                    } else {
-                        // each 16-byte scale load feeds two packed FMAs
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const ulonglong2 sc = s2[8 * h + j];
-                            sum2[16 * h + 2 * j] = f32x2_fma(f32x2_add(pack_u32x2(r[h][4 * j], r[h][4 * j + 1]), neg_bias2),
-                                                             sc.x, sum2[16 * h + 2 * j]);
-                            sum2[16 * h + 2 * j + 1] = f32x2_fma(
-                                f32x2_add(pack_u32x2(r[h][4 * j + 2], r[h][4 * j + 3]), neg_bias2), sc.y, sum2[16 * h + 2 * j + 1]);
-                        }
-                    }
+                    if (MODE == kModeI32G)
+                        store_partial16(p, rr[c & 1], g, m, mvalid, nw + 16 * c);
+                    else
+                        rescale16(sum2 + 8 * c, rr[c & 1], slot + 64 * c, neg_bias2);
                 }
-                if (MODE != kModeI32G) __syncwarp();  // every lane has read the slot before it is refilled
+                if (!ok) break;
+                tmem_st_wait();  // buffer b holds the preset again
+                tc_fence_before();
+                __syncwarp();  // also: every lane has read the scale slot before it is refilled
+                if (lane == 0) mbar_arrive(&acce[b]);
                 ++acc_i;
             }
             if (!ok) break;
