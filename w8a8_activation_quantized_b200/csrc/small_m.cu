@@ -10,17 +10,19 @@
 // GEMM path (activations quantized per token, integer products), so one
 // oracle covers every M.
 //
-// Work split.  The grid is persistent (two CTAs per SM): each CTA quantizes
-// the M activation rows once into shared memory, then walks blocks of R
-// output channels.  Its 8 warps form R rows x S K-slices (R*S = 8).  A weight
-// row is read as 16-byte chunks (16 int8 weights, or 32 packed int4 weights);
-// 32 lanes read 32 consecutive chunks per "pass" (512 or 1024 k values), and
-// a warp's slice is a whole number of passes, so a weight group (64 or 128
-// values) never straddles warps.  Each warp issues all loads of its slice
-// before using any (up to kMaxPass passes), and loads the next block's slice
-// while it computes the current one.  Per-group: the lanes of one group reduce
-// its INT32 partial with shuffles and one lane rescales it by scale_w[g][n]
-// in fp32.  Slices combine through shared memory.
+// Work split.  The grid is persistent (two CTAs per SM): all warps of a CTA
+// quantize the M activation rows into shared memory, then the CTA walks
+// blocks of R output channels.  Its 8 warps form R rows x S K-slices
+// (R*S = 8).  A weight row is read as 16-byte chunks (16 int8 weights, or 32
+// packed int4 weights); 32 lanes read 32 consecutive chunks per "pass" (512 or
+// 1024 k values), and a warp's slice is a whole number of passes, so a weight
+// group (64 or 128 values) never straddles warps.  Each warp keeps a ring of
+// three row blocks in registers -- all loads of a slice issued at once, two
+// blocks ahead of the one being used -- and its first two blocks start
+// loading before the activations are quantized.  Per-group: the lanes of one
+// group reduce its INT32 partial with shuffles and one lane rescales it by
+// scale_w[g][n] in fp32.  With one warp per row (S = 1) a warp writes its
+// outputs directly; otherwise the slices combine through shared memory.
 #include "cider_device.cuh"
 #include "cider_kernels.h"
 
@@ -28,7 +30,7 @@ namespace cider {
 
 constexpr int kSmallThreads = 256;
 constexpr int kSmallWarps = kSmallThreads / 32;
-constexpr int kMaxPass = 8;  // passes of 32 chunks a warp keeps in flight
+constexpr int kRing = 3;  // row blocks per warp: one being used, two loading
 
 __device__ __forceinline__ int dp4a(uint32_t a, uint32_t b, int c) {
     return __dp4a(static_cast<int>(a), static_cast<int>(b), c);
@@ -60,55 +62,62 @@ __device__ __forceinline__ int chunk_dot(const uint4& wv, const int8_t* qrow, in
 }
 
 struct SmallGeom {
-    int S, R;          // K-slices per row, rows per block (R * S = 8)
-    int ppw;           // passes per warp slice
-    int nblocks;       // row blocks
+    int S, R;     // K-slices per row, rows per block (R * S = 8)
+    int ppw;      // passes (32 chunks) per warp slice
+    int nblocks;  // row blocks
 };
 
-template <typename TX, typename TY, bool PG, bool W4, int MAXM>
-__global__ void __launch_bounds__(kSmallThreads) k_small_m(const TX* __restrict__ x, int M, int K,
-                                                           const uint8_t* __restrict__ w,
-                                                           const float* __restrict__ sw, int N,
-                                                           int gs, TY* __restrict__ y, SmallGeom geo) {
+template <typename TX, bool PG, bool W4, int MAXM, int PPW>
+__global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restrict__ x, int M, int K,
+                                                              const uint8_t* __restrict__ w,
+                                                              const float* __restrict__ sw, int N, int gs,
+                                                              void* __restrict__ y, int ydt, SmallGeom geo) {
     extern __shared__ __align__(16) int8_t s_q[];  // [M][K] codes
     __shared__ float s_sx[MAXM];
-    __shared__ float s_part[kSmallWarps][MAXM];  // per-warp partials (int32 bits for per-channel)
-    constexpr int KC = W4 ? 32 : 16;            // weights per 16-byte chunk
+    __shared__ float s_red[MAXM][kSmallWarps];
+    __shared__ float s_part[kSmallWarps][MAXM];
+    constexpr int KC = W4 ? 32 : 16;  // weights per 16-byte chunk
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row_bytes = W4 ? K / 2 : K;
     const int nch = K / KC;
     const int r_in_blk = warp / geo.S, slice = warp % geo.S;
     const int pass0 = slice * geo.ppw;
 
-    uint4 cur[kMaxPass], nxt[kMaxPass];
-    auto load = [&](uint4 (&dst)[kMaxPass], int blk) {
+    uint4 ring[kRing][PPW];
+    auto load = [&](uint4 (&dst)[PPW], int blk) {
         const int n = blk * geo.R + r_in_blk;
         const uint4* wr = reinterpret_cast<const uint4*>(w + static_cast<int64_t>(n) * row_bytes);
 #pragma unroll
-        for (int p = 0; p < kMaxPass; ++p) {
+        for (int p = 0; p < PPW; ++p) {
             const int c = (pass0 + p) * 32 + lane;
             dst[p] = (p < geo.ppw && blk < geo.nblocks && n < N && c < nch) ? __ldcs(wr + c) : make_uint4(0, 0, 0, 0);
         }
     };
-    int blk = blockIdx.x;
-    load(cur, blk);
-
-    // Quantize the M activation rows into shared memory (one warp per row).
-    for (int m = warp; m < M; m += kSmallWarps) {
-        const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K);
-        float amax = 0.0f;
-        for (int c = lane; c < K / 8; c += 32) {
-            float f[8];
-            unpack8_f32<TX>(__ldg(xr + c), f);
+    // weight traffic starts before the activations are quantized
 #pragma unroll
-            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
-        }
+    for (int i = 0; i < kRing - 1; ++i) load(ring[i], blockIdx.x + i * gridDim.x);
+
+    // Quantize the M activation rows into shared memory, all warps on every row.
+    const int nx = K / 8;  // 16-byte chunks of a row of x
+    for (int m = 0; m < M; ++m) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K);
+        typename Pack2<TX>::type m2 = {};
+        for (int c = threadIdx.x; c < nx; c += kSmallThreads) m2 = absmax8<TX>(__ldg(xr + c), m2);
+        float amax = absmax_to_f32<TX>(m2);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0) s_red[m][warp] = amax;
+    }
+    __syncthreads();
+    for (int m = 0; m < M; ++m) {
+        float amax = s_red[m][0];
+#pragma unroll
+        for (int i = 1; i < kSmallWarps; ++i) amax = fmaxf(amax, s_red[m][i]);
         const float s = act_scale(amax);
         const float rs = act_rcp(s);
-        if (lane == 0) s_sx[m] = s;
-        for (int c = lane; c < K / 8; c += 32) {
+        if (threadIdx.x == 0) s_sx[m] = s;
+        const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K);
+        for (int c = threadIdx.x; c < nx; c += kSmallThreads) {
             float f[8];
             unpack8_f32<TX>(__ldg(xr + c), f);
             *reinterpret_cast<uint2*>(s_q + static_cast<int64_t>(m) * K + 8 * c) = quant8_codes(f, s, rs);
@@ -117,8 +126,7 @@ __global__ void __launch_bounds__(kSmallThreads) k_small_m(const TX* __restrict_
     __syncthreads();
 
     const int lpg = PG ? gs / KC : 32;  // lanes per group: 2, 4 or 8
-    for (; blk < geo.nblocks; blk += gridDim.x) {
-        load(nxt, blk + gridDim.x);
+    auto step = [&](const uint4 (&cur)[PPW], int blk) {
         const int n = blk * geo.R + r_in_blk;
         int iacc[MAXM];
         float facc[MAXM];
@@ -126,10 +134,9 @@ __global__ void __launch_bounds__(kSmallThreads) k_small_m(const TX* __restrict_
         for (int m = 0; m < MAXM; ++m) { iacc[m] = 0; facc[m] = 0.0f; }
         if (n < N) {
 #pragma unroll
-            for (int p = 0; p < kMaxPass; ++p) {
-                if (p >= geo.ppw) break;  // warp-uniform
+            for (int p = 0; p < PPW; ++p) {
+                if (p >= geo.ppw || (pass0 + p) * 32 >= nch) break;  // warp-uniform
                 const int c = (pass0 + p) * 32 + lane;
-                if ((pass0 + p) * 32 >= nch) break;  // warp-uniform
                 const bool valid = c < nch;
                 const int k0 = c * KC;
                 if (!PG) {
@@ -150,44 +157,73 @@ __global__ void __launch_bounds__(kSmallThreads) k_small_m(const TX* __restrict_
                 }
             }
         }
-        // warp reduction, then across the S slices of each row
+        // reduce over the warp; one warp per row (S == 1) stores directly,
+        // otherwise the S slices of a row combine through shared memory
 #pragma unroll
         for (int m = 0; m < MAXM; ++m) {
             if (m < M) {
+                float v;
                 if (!PG) {
                     int a = iacc[m];
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-                    if (lane == 0) s_part[warp][m] = __int_as_float(a);
+                    v = __int_as_float(a);
                 } else {
                     float a = facc[m];
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-                    if (lane == 0) s_part[warp][m] = a;
+                    v = a;
+                }
+                if (geo.S == 1) {
+                    if (lane == 0 && n < N) {
+                        const float out = PG ? v * s_sx[m] : static_cast<float>(__float_as_int(v)) * s_sx[m] * __ldg(sw + n);
+                        if (ydt == 1)
+                            static_cast<__nv_bfloat16*>(y)[static_cast<int64_t>(m) * N + n] = __float2bfloat16_rn(out);
+                        else
+                            static_cast<__half*>(y)[static_cast<int64_t>(m) * N + n] = __float2half_rn(out);
+                    }
+                } else if (lane == 0) {
+                    s_part[warp][m] = v;
                 }
             }
         }
-        __syncthreads();
-        for (int t = threadIdx.x; t < geo.R * M; t += kSmallThreads) {
-            const int rr = t / M, m = t % M;
-            const int nn = blk * geo.R + rr;
-            if (nn < N) {
-                float v;
-                if (!PG) {
-                    int a = 0;
-                    for (int sl = 0; sl < geo.S; ++sl) a += __float_as_int(s_part[rr * geo.S + sl][m]);
-                    v = static_cast<float>(a) * s_sx[m] * __ldg(sw + nn);
-                } else {
-                    float a = 0.0f;
-                    for (int sl = 0; sl < geo.S; ++sl) a += s_part[rr * geo.S + sl][m];
-                    v = a * s_sx[m];
+        if (geo.S > 1) {
+            __syncthreads();
+            for (int t = threadIdx.x; t < geo.R * M; t += kSmallThreads) {
+                const int rr = t / M, m = t % M;
+                const int nn = blk * geo.R + rr;
+                if (nn < N) {
+                    float out;
+                    if (!PG) {
+                        int a = 0;
+                        for (int sl = 0; sl < geo.S; ++sl) a += __float_as_int(s_part[rr * geo.S + sl][m]);
+                        out = static_cast<float>(a) * s_sx[m] * __ldg(sw + nn);
+                    } else {
+                        float a = 0.0f;
+                        for (int sl = 0; sl < geo.S; ++sl) a += s_part[rr * geo.S + sl][m];
+                        out = a * s_sx[m];
+                    }
+                    if (ydt == 1)
+                        static_cast<__nv_bfloat16*>(y)[static_cast<int64_t>(m) * N + nn] = __float2bfloat16_rn(out);
+                    else
+                        static_cast<__half*>(y)[static_cast<int64_t>(m) * N + nn] = __float2half_rn(out);
                 }
-                y[static_cast<int64_t>(m) * N + nn] = from_f32<TY>(v);
             }
+            __syncthreads();
         }
-        __syncthreads();
+    };
+    // The ring is walked with compile-time slot indices (the loop is unrolled
+    // by the ring depth) so that it stays in registers.
+    int blk = blockIdx.x;
+    while (blk < geo.nblocks) {
 #pragma unroll
-        for (int p = 0; p < kMaxPass; ++p) cur[p] = nxt[p];
+        for (int r = 0; r < kRing; ++r) {
+            if (blk < geo.nblocks) {
+                load(ring[(r + kRing - 1) % kRing], blk + (kRing - 1) * gridDim.x);
+                step(ring[r], blk);
+            }
+            blk += gridDim.x;
+        }
     }
 }
 
@@ -205,46 +241,46 @@ static SmallGeom small_geom(int K, int N, bool w4) {
     return g;
 }
 
-template <typename TX, typename TY, bool PG, bool W4, int MAXM>
-static cudaError_t launch_small_t(const void* x, int M, int K, const void* w, const float* sw,
-                                  int N, int gs, void* y, int num_sms, cudaStream_t st) {
-    const SmallGeom geo = small_geom(K, N, W4);
-    if (geo.ppw > kMaxPass) return cudaErrorInvalidValue;  // K too large for this kernel
+template <typename TX, bool PG, bool W4, int MAXM, int PPW>
+static cudaError_t launch_small_t(const void* x, int M, int K, const void* w, const float* sw, int N, int gs,
+                                  void* y, int ydt, const SmallGeom& geo, int num_sms, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(M) * K;
-    auto kern = k_small_m<TX, TY, PG, W4, MAXM>;
+    auto kern = k_small_m<TX, PG, W4, MAXM, PPW>;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
     const int grid = geo.nblocks < 2 * num_sms ? geo.nblocks : 2 * num_sms;
-    kern<<<grid, kSmallThreads, smem, st>>>(static_cast<const TX*>(x), M, K, static_cast<const uint8_t*>(w), sw, N,
-                                             gs, static_cast<TY*>(y), geo);
+    kern<<<grid, kSmallThreads, smem, st>>>(static_cast<const TX*>(x), M, K, static_cast<const uint8_t*>(w), sw, N, gs,
+                                             y, ydt, geo);
     return cudaGetLastError();
 }
 
-bool small_m_supported(int K, bool w4) { return small_geom(K, 8, w4).ppw <= kMaxPass; }
+template <typename TX, bool PG, bool W4, int MAXM>
+static cudaError_t launch_small_ppw(const void* x, int M, int K, const void* w, const float* sw, int N, int gs,
+                                   void* y, int ydt, int num_sms, cudaStream_t st) {
+    const SmallGeom geo = small_geom(K, N, W4);
+    if (geo.ppw <= 2) return launch_small_t<TX, PG, W4, MAXM, 2>(x, M, K, w, sw, N, gs, y, ydt, geo, num_sms, st);
+    if (geo.ppw <= 4) return launch_small_t<TX, PG, W4, MAXM, 4>(x, M, K, w, sw, N, gs, y, ydt, geo, num_sms, st);
+    if (geo.ppw <= 5) return launch_small_t<TX, PG, W4, MAXM, 5>(x, M, K, w, sw, N, gs, y, ydt, geo, num_sms, st);
+    if (geo.ppw <= 8) return launch_small_t<TX, PG, W4, MAXM, 8>(x, M, K, w, sw, N, gs, y, ydt, geo, num_sms, st);
+    return cudaErrorInvalidValue;  // K beyond the small-M kernel: the host sends such calls to the GEMM path
+}
 
-template <typename TX, typename TY, bool PG, bool W4>
-static cudaError_t launch_small_m_tt(const void* x, int M, int K, const void* w, const float* sw,
-                                     int N, int gs, void* y, int num_sms, cudaStream_t st) {
-    if (M <= 1) return launch_small_t<TX, TY, PG, W4, 1>(x, M, K, w, sw, N, gs, y, num_sms, st);
-    if (M <= 4) return launch_small_t<TX, TY, PG, W4, 4>(x, M, K, w, sw, N, gs, y, num_sms, st);
-    if (M <= 8) return launch_small_t<TX, TY, PG, W4, 8>(x, M, K, w, sw, N, gs, y, num_sms, st);
-    return launch_small_t<TX, TY, PG, W4, 16>(x, M, K, w, sw, N, gs, y, num_sms, st);
+template <typename TX, bool PG, bool W4>
+static cudaError_t launch_small_m_t(const void* x, int M, int K, const void* w, const float* sw, int N, int gs,
+                                    void* y, int ydt, int num_sms, cudaStream_t st) {
+    if (M <= 1) return launch_small_ppw<TX, PG, W4, 1>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
+    if (M <= 4) return launch_small_ppw<TX, PG, W4, 4>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
+    if (M <= 8) return launch_small_ppw<TX, PG, W4, 8>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
+    return launch_small_ppw<TX, PG, W4, 16>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
 }
 
 template <bool PG, bool W4>
-static cudaError_t launch_small_m_v(const void* x, int xdt, int M, int K, const void* w,
-                                    const float* sw, int N, int gs, void* y, int ydt, int num_sms,
-                                    cudaStream_t st) {
-    if (xdt == 0 && ydt == 0)
-        return launch_small_m_tt<__half, __half, PG, W4>(x, M, K, w, sw, N, gs, y, num_sms, st);
-    if (xdt == 0 && ydt == 1)
-        return launch_small_m_tt<__half, __nv_bfloat16, PG, W4>(x, M, K, w, sw, N, gs, y, num_sms, st);
-    if (xdt == 1 && ydt == 0)
-        return launch_small_m_tt<__nv_bfloat16, __half, PG, W4>(x, M, K, w, sw, N, gs, y, num_sms, st);
-    return launch_small_m_tt<__nv_bfloat16, __nv_bfloat16, PG, W4>(x, M, K, w, sw, N, gs, y, num_sms, st);
+static cudaError_t launch_small_m_v(const void* x, int xdt, int M, int K, const void* w, const float* sw, int N,
+                                    int gs, void* y, int ydt, int num_sms, cudaStream_t st) {
+    if (xdt == 1) return launch_small_m_t<__nv_bfloat16, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
+    return launch_small_m_t<__half, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
 }
 
 cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const void* w,
