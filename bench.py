@@ -458,7 +458,26 @@ def bench_rows(device, pk, steps, warmup):
     sb = torch.empty((M,), dtype=torch.float32, device=device)
     ms = graph_time(lambda i: cider.cider_silu_mul_quantize(gts[i % 3], uts[i % 3], q=qb[i % 3], scale_x=sb), steps, warmup)
     record("silu_mul_quantize", ms, 0, M * F * 5 + M * 4, M=M, F=F)
+    out.append(bench_stack(device, pk, steps=max(3, steps // 20), warmup=warmup))
     return out
+
+
+def bench_stack(device, pk, steps, warmup, layers=36, M=2048):
+    """The linear stack of an 8B-class decoder: `layers` layers x 7 W8A8
+    per-channel linears with SiLU(gate)*up fused into down_proj's quantize."""
+    from w8a8_activation_quantized_b200 import stack, synth
+    int8_peak = pk["bf16"] * INT8_PER_BF16
+    stk = stack.DecoderLinearStack(layers, device=device)
+    H = torch.from_numpy(synth.activations(M, stack.HIDDEN, seed=4000 + M, outlier_frac=0.005,
+                                           outlier_scale=100.0)).to(device)
+    ms = graph_time(lambda i: stk.forward(H), steps, warmup)
+    ops = layers * stack.ops_per_layer(M)
+    wbytes = layers * sum(n * k for _, n, k in stack.LINEARS)
+    tops = ops / (ms * 1e-3) / 1e12
+    del stk
+    return dict(row="decoder_linear_stack", layers=layers, M=M, ms=ms, TOPS=tops,
+                **{"GB/s": wbytes / (ms * 1e-3) / 1e9}, bound="tensor", frac=tops / int8_peak,
+                launches_per_step=layers * 11, weight_bytes=wbytes)
 
 
 ROW_CASES = {
@@ -469,6 +488,7 @@ ROW_CASES = {
     "pg128_m1": ("pg", 1, 2560, 10240, 128), "pg128_m4096": ("pg", 4096, 2560, 10240, 128),
     "pg64_m1": ("pg", 1, 2560, 10240, 64), "pg64_m4096": ("pg", 4096, 2560, 10240, 64),
     "w4a8_m2048": ("w4", 2048, 12288, 4096, 64),
+    "stack_8b": ("stack", 2048, 0, 0, 0),
 }
 
 
@@ -476,6 +496,10 @@ def run_row(args):
     """One hot-path row alone (for profiling): device time per call, one JSON line."""
     import w8a8_activation_quantized_b200 as cider
     from w8a8_activation_quantized_b200 import synth
+    if args.row == "stack_8b":
+        torch.cuda.set_device(0)
+        print(json.dumps(bench_stack(torch.device("cuda", 0), peaks(), args.steps, args.warmup)), flush=True)
+        return 0
     kind, M, N, K, gs = ROW_CASES[args.row]
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)

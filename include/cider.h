@@ -217,6 +217,11 @@ CIDER_API cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8
  * 2 = single-CTA 128x256 tiles, 3 = CTA-pair 256x256 tiles.  Lets tests cover
  * every variant on small shapes. */
 CIDER_API cider_status_t cider_test_set_gemm_variant(int variant);
+/* Exercises the bounded-wait path of the kernels without a fault: one warp
+ * waits on an mbarrier that nothing arrives on and gives up after limit_ns
+ * (1 .. 1e8).  The next cider_device_status() then returns CIDER_ERR_TIMEOUT
+ * and clears the status word. */
+CIDER_API cider_status_t cider_test_bounded_wait(int64_t limit_ns, void* stream);
 /* The W4A8 load path's unpack: w[n][k] = nibble(n, k) - 8. */
 CIDER_API cider_status_t cider_test_unpack_int4(const uint8_t* w_packed, int64_t N, int64_t K, int8_t* w,
                                       void* stream);

@@ -149,3 +149,26 @@ def test_linear_is_composition(act, ydt):
     w4 = oracle.unpack_int4(packed, 512)
     np.testing.assert_array_equal(oracle.w4a8_linear_pg(act, packed, s4, 64, ydt=ydt),
                                   oracle.linear_pg(act, w4, s4, 64, ydt=ydt))
+
+
+def test_silu_mul_against_numpy():
+    """SiLU(g) * u of the decoder MLP: the oracle's fp64 evaluation rounded once
+    equals numpy's own fp64 expression rounded by numpy (nearest even), and
+    SiLU's closed-form special values hold."""
+    rng = np.random.default_rng(21)
+    g = (rng.standard_normal(100_000) * 4).astype(np.float16)
+    u = (rng.standard_normal(100_000) * 2).astype(np.float16)
+    a = oracle.silu_mul(g, u).view(np.float16)
+    gd, ud = g.astype(np.float64), u.astype(np.float64)
+    np.testing.assert_array_equal(a, (gd / (1.0 + np.exp(-gd)) * ud).astype(np.float16))
+    # silu(0) = 0, silu(g) -> g for large g, silu(g) -> 0 for very negative g
+    sp = oracle.silu_mul(np.float16([0.0, 20.0, -30.0]), np.float16([1.0, 1.0, 1.0])).view(np.float16)
+    assert sp[0] == 0 and sp[1] == np.float16(20.0) and abs(float(sp[2])) < 1e-6
+    # bf16 path: values exact in bf16, checked against torch's rounding of the fp64 result
+    import torch
+    gb = torch.tensor([0.5, -1.0, 3.0, -7.5], dtype=torch.bfloat16)
+    ub = torch.tensor([2.0, 1.5, -0.25, 4.0], dtype=torch.bfloat16)
+    got = oracle.silu_mul(gb.view(torch.int16).numpy().view(np.uint16), ub.view(torch.int16).numpy().view(np.uint16),
+                          oracle.BF16)
+    ref = (gb.double() * torch.sigmoid(gb.double()) * ub.double()).float().to(torch.bfloat16)
+    np.testing.assert_array_equal(got, ref.view(torch.int16).numpy().view(np.uint16))

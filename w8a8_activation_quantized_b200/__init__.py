@@ -57,6 +57,7 @@ _SIGNATURES = {
     "cider_test_gemm_i32_grouped": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _P, _P]),
     "cider_test_unpack_int4": (_INT, [_P, _I64, _I64, _P, _P]),
     "cider_test_set_gemm_variant": (_INT, [_INT]),
+    "cider_test_bounded_wait": (_INT, [_I64, _P]),
 }
 EXPORTS = tuple(_SIGNATURES)
 
@@ -297,6 +298,11 @@ def cider_test_gemm_i32_grouped(q, w, gs, acc_g=None, stream=None):
 def cider_test_set_gemm_variant(variant: int):
     """0 automatic, 1 single-CTA 128x128, 2 single-CTA 128x256, 3 CTA-pair 256x256."""
     _check("cider_test_set_gemm_variant", lib().cider_test_set_gemm_variant(variant))
+
+
+def cider_test_bounded_wait(limit_ns: int, stream=None, device=None):
+    """Runs the bounded-wait self-test kernel (see include/cider.h)."""
+    _check("cider_test_bounded_wait", lib().cider_test_bounded_wait(limit_ns, _stream(stream, device)))
 
 
 def cider_test_unpack_int4(w_packed, K, w=None, stream=None):

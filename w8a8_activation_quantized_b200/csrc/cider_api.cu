@@ -456,6 +456,18 @@ cider_status_t cider_test_set_gemm_variant(int variant) {
     return CIDER_OK;
 }
 
+cider_status_t cider_test_bounded_wait(int64_t limit_ns, void* stream) {
+    t_last_error[0] = '\0';
+    if (limit_ns < 1 || limit_ns > 100000000)
+        return fail(CIDER_ERR_INVALID_ARG, "limit_ns = %lld outside [1, 1e8]", (long long)limit_ns);
+    DeviceInfo* d = nullptr;
+    cider_status_t s = device_info(&d);
+    if (s != CIDER_OK) return s;
+    cudaError_t e = launch_wait_selftest(d->status, static_cast<unsigned long long>(limit_ns),
+                                         static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "wait self-test launch");
+}
+
 cider_status_t cider_test_unpack_int4(const uint8_t* w_packed, int64_t N, int64_t K, int8_t* w, void* stream) {
     t_last_error[0] = '\0';
     if (N < 1 || K < 1 || K % 32) return fail(CIDER_ERR_INVALID_ARG, "N >= 1, K >= 1, K %% 32 == 0 required");

@@ -56,23 +56,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up (returns
-// false, sets the status word) after kWaitLimitNs, or as soon as another
-// thread has recorded a failure in *abort_flag.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status,
-                                          volatile int* abort_flag) {
+// false, sets the status word) after limit_ns, or as soon as another thread
+// has recorded a failure in *abort_flag.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned* status,
+                                              volatile int* abort_flag, unsigned long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     unsigned long long t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 255u) == 0u) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 atomicOr(status, kStatusTimeout);
                 *abort_flag = 1;
                 return false;
             }
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status,
+                                          volatile int* abort_flag) {
+    return mbar_wait_for(bar, parity, status, abort_flag, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------------------

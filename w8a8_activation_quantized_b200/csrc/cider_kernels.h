@@ -54,6 +54,7 @@ cudaError_t launch_silu_mul_quantize(const void* g, const void* u, int dt, int64
 // mode 0: per channel (out = int8 [N][K]); 1: per group int8; 2: per group int4 packed
 cudaError_t launch_quantize_weight(int mode, const float* W, int64_t N, int K, int gs, void* out,
                                    float* sw, cudaStream_t st);
+cudaError_t launch_wait_selftest(unsigned* status, unsigned long long limit_ns, cudaStream_t st);
 cudaError_t launch_unpack_int4(const uint8_t* packed, int64_t N, int K, int8_t* w, cudaStream_t st);
 cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const void* w,
                            const float* sw, int N, int gs, void* y, int ydt, int num_sms,

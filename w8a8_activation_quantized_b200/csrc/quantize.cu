@@ -332,4 +332,24 @@ cudaError_t launch_unpack_int4(const uint8_t* packed, int64_t N, int K, int8_t* 
     return cudaGetLastError();
 }
 
+// ---- self-test of the bounded wait ------------------------------------------
+// One warp waits on an mbarrier that nothing ever arrives on; the wait must
+// give up after limit_ns and record the timeout in the status word.
+__global__ void k_wait_selftest(unsigned* status, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait_for(&bar, 0, status, &abort_flag, limit_ns);
+}
+
+cudaError_t launch_wait_selftest(unsigned* status, unsigned long long limit_ns, cudaStream_t st) {
+    k_wait_selftest<<<1, 32, 0, st>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+
 }  // namespace cider

@@ -59,6 +59,16 @@ def weights(N: int, K: int, seed: int, std: float = 0.02) -> np.ndarray:
     return _rng(seed + 1_000_003).normal(0.0, std, size=(N, K)).astype(np.float32)
 
 
+def weights_device(N: int, K: int, seed: int, std: float = 0.02, device="cuda"):
+    """fp32 [N, K] ~ N(0, std) drawn on `device` by torch's seeded generator
+    (for weight sets too large to draw on the host; the same seed and device
+    give the same numbers, which a CPU check can copy back)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randn((N, K), generator=g, device=device, dtype=torch.float32) * std
+
+
 # Named workloads (sizes of the Cider single-op tables and of an 8B-class
 # decoder's linear stack).  Each entry: kind, M list, N, K, extra.
 WORKLOADS = {
