@@ -22,6 +22,13 @@ __device__ __forceinline__ unsigned long long global_timer_ns() {
     return t;
 }
 
+// Programmatic dependent launch: every kernel of this library is launched so
+// that it may start while the previous kernel on the stream finishes.  It
+// must call pdl_wait() before its first read of global memory another kernel
+// may have written; pdl_trigger() lets the next kernel begin its own launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

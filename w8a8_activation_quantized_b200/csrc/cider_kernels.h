@@ -39,6 +39,25 @@ struct GemmLaunch {
     unsigned* status;  // device status word
 };
 
+// Launches `kern` with programmatic stream serialisation allowed, so that its
+// setup overlaps the tail of the previous kernel on the stream (each kernel
+// waits with griddepcontrol.wait before reading global memory).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // Records a message for cider_last_error() on this thread and returns `s`.
 cider_status_t set_error(cider_status_t s, const char* fmt, ...);
 

@@ -200,6 +200,8 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     volatile int* abort_flag = &s_abort;
+    pdl_wait();  // inputs of the previous kernel on the stream are complete
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
@@ -464,8 +466,7 @@ static cudaError_t launch_grouped_t(const GemmLaunch& L, cudaStream_t st) {
     auto kern = k_gemm_grouped<MODE, TY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, tmY, a);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, C::THREADS, C::SMEM_BYTES, st, tmA, tmB, tmY, a);
 }
 
 cudaError_t launch_gemm_grouped(const GemmLaunch& L, cudaStream_t st) {

@@ -129,6 +129,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     volatile int* abort_flag = &s_abort;
+    pdl_wait();  // inputs of the previous kernel on the stream are complete
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
@@ -333,6 +335,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     volatile int* abort_flag = &s_abort;
+    pdl_wait();  // inputs of the previous kernel on the stream are complete
+    pdl_trigger();
 
     if (warp == 0) {
         // ---------------- TMA producer (both CTAs): own A rows, own half of B ----------------
@@ -479,8 +483,7 @@ static cudaError_t launch_gemm_cfg(const GemmLaunch& L, cudaStream_t st) {
     auto kern = k_gemm_sm100<Cfg, TY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(tmA, tmB, a);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, Cfg::THREADS, Cfg::SMEM_BYTES, st, tmA, tmB, a);
 }
 
 template <int MODE, typename TY>
@@ -510,8 +513,7 @@ static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
     auto kern = k_gemm_pair<MODE, TY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<2 * clusters, PairCfg::THREADS, PairCfg::SMEM_BYTES, st>>>(tmA, tmB, tmY, a);
-    return cudaGetLastError();
+    return launch_pdl(kern, 2 * clusters, PairCfg::THREADS, PairCfg::SMEM_BYTES, st, tmA, tmB, tmY, a);
 }
 
 template <int MODE, typename TY>

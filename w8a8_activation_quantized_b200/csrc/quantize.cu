@@ -38,6 +38,8 @@ template <typename T, int NV>
 __global__ void __launch_bounds__(128, (NV <= 10 ? 6 : 4)) k_quantize_warp(const T* __restrict__ x, int64_t M, int K,
                                                        int8_t* __restrict__ q,
                                                        float* __restrict__ sx) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (row >= M) return;
@@ -77,6 +79,8 @@ __global__ void __launch_bounds__(256) k_quantize_cta(const T* __restrict__ x, i
                                                       int8_t* __restrict__ q,
                                                       float* __restrict__ sx) {
     __shared__ float red[8];
+    pdl_wait();
+    pdl_trigger();
     const int64_t row = blockIdx.x;
     const int tid = threadIdx.x;
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
@@ -136,25 +140,26 @@ static cudaError_t launch_quantize_t(const void* x, int64_t M, int K, int8_t* q,
                                      cudaStream_t st) {
     const T* xt = static_cast<const T*>(x);
     if (M == 0) return cudaSuccess;
+    cudaError_t e = cudaSuccess;
     if (K <= 4096) {
         const unsigned grid = static_cast<unsigned>((M + 3) / 4);
         const int nv = (K + 255) / 256;
-        if (nv <= 1) k_quantize_warp<T, 1><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
-        else if (nv <= 2) k_quantize_warp<T, 2><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
-        else if (nv <= 4) k_quantize_warp<T, 4><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
-        else if (nv <= 6) k_quantize_warp<T, 6><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
-        else if (nv <= 8) k_quantize_warp<T, 8><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
-        else if (nv <= 10) k_quantize_warp<T, 10><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
-        else if (nv <= 12) k_quantize_warp<T, 12><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
-        else k_quantize_warp<T, 16><<<grid, 128, 0, st>>>(xt, M, K, q, sx);
+        if (nv <= 1) e = launch_pdl(k_quantize_warp<T, 1>, grid, 128, 0, st, xt, M, K, q, sx);
+        else if (nv <= 2) e = launch_pdl(k_quantize_warp<T, 2>, grid, 128, 0, st, xt, M, K, q, sx);
+        else if (nv <= 4) e = launch_pdl(k_quantize_warp<T, 4>, grid, 128, 0, st, xt, M, K, q, sx);
+        else if (nv <= 6) e = launch_pdl(k_quantize_warp<T, 6>, grid, 128, 0, st, xt, M, K, q, sx);
+        else if (nv <= 8) e = launch_pdl(k_quantize_warp<T, 8>, grid, 128, 0, st, xt, M, K, q, sx);
+        else if (nv <= 10) e = launch_pdl(k_quantize_warp<T, 10>, grid, 128, 0, st, xt, M, K, q, sx);
+        else if (nv <= 12) e = launch_pdl(k_quantize_warp<T, 12>, grid, 128, 0, st, xt, M, K, q, sx);
+        else e = launch_pdl(k_quantize_warp<T, 16>, grid, 128, 0, st, xt, M, K, q, sx);
     } else {
         const unsigned grid = static_cast<unsigned>(M);
         const int nv = (K / 8 + 255) / 256;
-        if (nv <= 4) k_quantize_cta<T, 4><<<grid, 256, 0, st>>>(xt, K, q, sx);
-        else if (nv <= 8) k_quantize_cta<T, 8><<<grid, 256, 0, st>>>(xt, K, q, sx);
-        else k_quantize_cta<T, 0><<<grid, 256, 0, st>>>(xt, K, q, sx);
+        if (nv <= 4) e = launch_pdl(k_quantize_cta<T, 4>, grid, 256, 0, st, xt, K, q, sx);
+        else if (nv <= 8) e = launch_pdl(k_quantize_cta<T, 8>, grid, 256, 0, st, xt, K, q, sx);
+        else e = launch_pdl(k_quantize_cta<T, 0>, grid, 256, 0, st, xt, K, q, sx);
     }
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_quantize_act(const void* x, int xdt, int64_t M, int K, int8_t* q, float* sx,
@@ -173,6 +178,8 @@ __global__ void __launch_bounds__(256) k_silu_mul_quantize(const T* __restrict__
                                                            float* __restrict__ sx,
                                                            T* __restrict__ a_out) {
     __shared__ float red[8];
+    pdl_wait();
+    pdl_trigger();
     const int64_t row = blockIdx.x;
     const int tid = threadIdx.x;
     const uint4* gr = reinterpret_cast<const uint4*>(gate + row * F);
@@ -236,11 +243,10 @@ static cudaError_t launch_silu_t(const void* g, const void* u, int64_t M, int F,
     const T* ut = static_cast<const T*>(u);
     T* at = static_cast<T*>(a_out);
     const unsigned grid = static_cast<unsigned>(M);
-    if (nv <= 2) k_silu_mul_quantize<T, 2><<<grid, 256, 0, st>>>(gt, ut, F, q, sx, at);
-    else if (nv <= 8) k_silu_mul_quantize<T, 8><<<grid, 256, 0, st>>>(gt, ut, F, q, sx, at);
-    else if (nv <= 16) k_silu_mul_quantize<T, 16><<<grid, 256, 0, st>>>(gt, ut, F, q, sx, at);
-    else return cudaErrorInvalidValue;  // F > 32768: rejected by the host checks first
-    return cudaGetLastError();
+    if (nv <= 2) return launch_pdl(k_silu_mul_quantize<T, 2>, grid, 256, 0, st, gt, ut, F, q, sx, at);
+    else if (nv <= 8) return launch_pdl(k_silu_mul_quantize<T, 8>, grid, 256, 0, st, gt, ut, F, q, sx, at);
+    else if (nv <= 16) return launch_pdl(k_silu_mul_quantize<T, 16>, grid, 256, 0, st, gt, ut, F, q, sx, at);
+    return cudaErrorInvalidValue;  // F > 32768: rejected by the host checks first
 }
 
 cudaError_t launch_silu_mul_quantize(const void* g, const void* u, int dt, int64_t M, int F,
@@ -255,6 +261,8 @@ __global__ void __launch_bounds__(256) k_quantize_weight_pc(const float* __restr
                                                             int8_t* __restrict__ w,
                                                             float* __restrict__ sw) {
     __shared__ float red[8];
+    pdl_wait();
+    pdl_trigger();
     const int64_t n = blockIdx.x;
     const float* wr = W + n * K;
     float amax = 0.0f;
@@ -275,6 +283,8 @@ __global__ void __launch_bounds__(256) k_quantize_weight_group(const float* __re
                                                                int64_t N, int K, int gs,
                                                                void* __restrict__ out,
                                                                float* __restrict__ sw) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     const int G = K / gs;
@@ -305,21 +315,18 @@ __global__ void __launch_bounds__(256) k_quantize_weight_group(const float* __re
 
 cudaError_t launch_quantize_weight(int mode, const float* W, int64_t N, int K, int gs, void* out,
                                    float* sw, cudaStream_t st) {
-    if (mode == 0) {
-        k_quantize_weight_pc<<<static_cast<unsigned>(N), 256, 0, st>>>(W, K, static_cast<int8_t*>(out), sw);
-    } else {
-        const int64_t items = N * (K / gs);
-        const unsigned grid = static_cast<unsigned>((items + 7) / 8);
-        if (mode == 1)
-            k_quantize_weight_group<false><<<grid, 256, 0, st>>>(W, N, K, gs, out, sw);
-        else
-            k_quantize_weight_group<true><<<grid, 256, 0, st>>>(W, N, K, gs, out, sw);
-    }
-    return cudaGetLastError();
+    if (mode == 0)
+        return launch_pdl(k_quantize_weight_pc, static_cast<unsigned>(N), 256, 0, st, W, K, static_cast<int8_t*>(out), sw);
+    const int64_t items = N * (K / gs);
+    const unsigned grid = static_cast<unsigned>((items + 7) / 8);
+    if (mode == 1) return launch_pdl(k_quantize_weight_group<false>, grid, 256, 0, st, W, N, K, gs, out, sw);
+    return launch_pdl(k_quantize_weight_group<true>, grid, 256, 0, st, W, N, K, gs, out, sw);
 }
 
 // ---- INT4 unpack (the W4A8 load path's conversion), standalone ---------------
 __global__ void k_unpack_int4(const uint32_t* __restrict__ packed, int64_t words, uint2* __restrict__ w) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i < words) w[i] = unpack_int4x8(packed[i]);
 }
@@ -327,9 +334,8 @@ __global__ void k_unpack_int4(const uint32_t* __restrict__ packed, int64_t words
 cudaError_t launch_unpack_int4(const uint8_t* packed, int64_t N, int K, int8_t* w, cudaStream_t st) {
     const int64_t words = N * (K / 8);  // K % 32 == 0 keeps rows whole words
     if (words == 0) return cudaSuccess;
-    k_unpack_int4<<<static_cast<unsigned>((words + 255) / 256), 256, 0, st>>>(
-        reinterpret_cast<const uint32_t*>(packed), words, reinterpret_cast<uint2*>(w));
-    return cudaGetLastError();
+    return launch_pdl(k_unpack_int4, static_cast<unsigned>((words + 255) / 256), 256, 0, st,
+                      reinterpret_cast<const uint32_t*>(packed), words, reinterpret_cast<uint2*>(w));
 }
 
 // ---- self-test of the bounded wait ------------------------------------------

@@ -30,7 +30,12 @@ namespace cider {
 
 constexpr int kSmallThreads = 256;
 constexpr int kSmallWarps = kSmallThreads / 32;
-constexpr int kRing = 3;  // row blocks per warp: one being used, two loading
+// Row blocks per warp in the register ring: one being used and the rest
+// loading; two for the widest slices (8 passes) to stay within registers.
+template <int PPW>
+struct RingDepth {
+    static constexpr int value = PPW <= 5 ? 3 : 2;
+};
 
 __device__ __forceinline__ int dp4a(uint32_t a, uint32_t b, int c) {
     return __dp4a(static_cast<int>(a), static_cast<int>(b), c);
@@ -82,20 +87,31 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
     const int nch = K / KC;
     const int r_in_blk = warp / geo.S, slice = warp % geo.S;
     const int pass0 = slice * geo.ppw;
+    pdl_wait();
+    pdl_trigger();
 
+    // Ring slot: the block's weight chunks and the scales they need (per-channel:
+    // scale_w[n]; per-group: this lane's group scale for each pass), all loaded
+    // ahead so no scale load sits on the critical path.
+    constexpr int kRing = RingDepth<PPW>::value;
     uint4 ring[kRing][PPW];
-    auto load = [&](uint4 (&dst)[PPW], int blk) {
+    float ring_s[kRing][PG ? PPW : 1];
+    auto load = [&](uint4 (&dst)[PPW], float (&ds)[PG ? PPW : 1], int blk) {
         const int n = blk * geo.R + r_in_blk;
+        const bool row_ok = blk < geo.nblocks && n < N;
         const uint4* wr = reinterpret_cast<const uint4*>(w + static_cast<int64_t>(n) * row_bytes);
 #pragma unroll
         for (int p = 0; p < PPW; ++p) {
             const int c = (pass0 + p) * 32 + lane;
-            dst[p] = (p < geo.ppw && blk < geo.nblocks && n < N && c < nch) ? __ldcs(wr + c) : make_uint4(0, 0, 0, 0);
+            const bool ok = p < geo.ppw && row_ok && c < nch;
+            dst[p] = ok ? __ldcs(wr + c) : make_uint4(0, 0, 0, 0);
+            if (PG) ds[p] = ok ? __ldg(sw + static_cast<int64_t>(c * KC / gs) * N + n) : 0.0f;
         }
+        if (!PG) ds[0] = row_ok ? __ldg(sw + n) : 0.0f;
     };
     // weight traffic starts before the activations are quantized
 #pragma unroll
-    for (int i = 0; i < kRing - 1; ++i) load(ring[i], blockIdx.x + i * gridDim.x);
+    for (int i = 0; i < kRing - 1; ++i) load(ring[i], ring_s[i], blockIdx.x + i * gridDim.x);
 
     // Quantize the M activation rows into shared memory, all warps on every row.
     const int nx = K / 8;  // 16-byte chunks of a row of x
@@ -126,7 +142,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
     __syncthreads();
 
     const int lpg = PG ? gs / KC : 32;  // lanes per group: 2, 4 or 8
-    auto step = [&](const uint4 (&cur)[PPW], int blk) {
+    auto step = [&](const uint4 (&cur)[PPW], const float (&cs)[PG ? PPW : 1], int blk) {
         const int n = blk * geo.R + r_in_blk;
         int iacc[MAXM];
         float facc[MAXM];
@@ -144,8 +160,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
                     for (int m = 0; m < MAXM; ++m)
                         if (m < M && valid) iacc[m] = chunk_dot<W4>(cur[p], s_q + static_cast<int64_t>(m) * K, k0) + iacc[m];
                 } else {
-                    const int g = valid ? k0 / gs : 0;
-                    const float s = valid ? __ldg(sw + static_cast<int64_t>(g) * N + n) : 0.0f;
+                    const float s = cs[p];  // this lane's group scale (0 for invalid chunks)
 #pragma unroll
                     for (int m = 0; m < MAXM; ++m) {
                         if (m < M) {
@@ -176,7 +191,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
                 }
                 if (geo.S == 1) {
                     if (lane == 0 && n < N) {
-                        const float out = PG ? v * s_sx[m] : static_cast<float>(__float_as_int(v)) * s_sx[m] * __ldg(sw + n);
+                        const float out = PG ? v * s_sx[m] : static_cast<float>(__float_as_int(v)) * s_sx[m] * cs[0];
                         if (ydt == 1)
                             static_cast<__nv_bfloat16*>(y)[static_cast<int64_t>(m) * N + n] = __float2bfloat16_rn(out);
                         else
@@ -219,8 +234,8 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
 #pragma unroll
         for (int r = 0; r < kRing; ++r) {
             if (blk < geo.nblocks) {
-                load(ring[(r + kRing - 1) % kRing], blk + (kRing - 1) * gridDim.x);
-                step(ring[r], blk);
+                load(ring[(r + kRing - 1) % kRing], ring_s[(r + kRing - 1) % kRing], blk + (kRing - 1) * gridDim.x);
+                step(ring[r], ring_s[r], blk);
             }
             blk += gridDim.x;
         }
@@ -251,9 +266,8 @@ static cudaError_t launch_small_t(const void* x, int M, int K, const void* w, co
         if (e != cudaSuccess) return e;
     }
     const int grid = geo.nblocks < 2 * num_sms ? geo.nblocks : 2 * num_sms;
-    kern<<<grid, kSmallThreads, smem, st>>>(static_cast<const TX*>(x), M, K, static_cast<const uint8_t*>(w), sw, N, gs,
-                                             y, ydt, geo);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, kSmallThreads, smem, st, static_cast<const TX*>(x), M, K,
+                      static_cast<const uint8_t*>(w), sw, N, gs, y, ydt, geo);
 }
 
 template <typename TX, bool PG, bool W4, int MAXM>
