@@ -10,27 +10,32 @@
 // Design.  One CTA per SM, persistent over 128 x 128 output tiles.
 //  * warp 0 issues TMA loads of A = q [M][K] and B = w [N][K] (or, for W4A8,
 //    packed [N][K/2] bytes) into a ring of 128-wide K stages;
-//  * warp 1 issues tcgen05.mma.kind::i8, one INT32 partial per group into a
-//    ring of four 128-column TMEM buffers;
+//  * warp 1 issues the MMAs: one INT32 partial per group into a ring of four
+//    128-column TMEM buffers.  Each group starts with one kind::f16 MMA of
+//    constant operands (16 products 64 * 12288, exact in fp32) that
+//    overwrites the buffer with the bits of 1.5 * 2^23 (0x4B400000); the
+//    group's kind::i8 MMAs then accumulate onto those bits, so the 32-bit
+//    word of a partial p (|p| < 2^22) read as a float is exactly
+//    1.5 * 2^23 + p.  The tensor core writes the bias itself (64 MMA cycles
+//    per group), so the epilogue never stores to TMEM;
 //  * for W4A8, two converter warps expand each packed stage to int8
 //    (nibble - 8) in the 128-byte-swizzled layout the MMA reads, then fence the
 //    writes to the async proxy and hand the stage to the MMA warp;
-//  * eight epilogue warps rescale every partial.  Each TMEM buffer is preset
-//    with the bit pattern of 1.5 * 2^23 (0x4B400000) and the MMA accumulates
-//    on top of it, so the 32-bit word of a partial p (|p| < 2^22) read as a
-//    float is exactly 1.5 * 2^23 + p: one packed f32x2 add recovers p exactly
-//    and one packed f32x2 FMA adds p * scale to the running sum, two elements
-//    per instruction.  The reader restores the preset (tcgen05.st) before
-//    handing the buffer back.  Group scales reach shared memory ahead of use
-//    through a per-warp cp.async ring; the finished tile leaves through
-//    swizzled staging boxes and TMA stores.
+//  * eight epilogue warps rescale every partial: one packed f32x2 add
+//    recovers p exactly and one packed f32x2 FMA adds p * scale to the running
+//    sum, two elements per instruction.  A warp hands a buffer back as soon as
+//    its last TMEM load of it has completed.  Group scales reach shared memory
+//    ahead of use through a per-warp cp.async ring; the finished tile leaves
+//    through swizzled staging boxes and TMA stores.
+// Cost model (measured on B200): per group and 128 x 128 tile the epilogue
+// moves every partial TMEM -> registers once and issues two fp32 operations
+// per partial; these do not overlap, which puts the floor near 384 cycles
+// per group per SM sub-partition -- the epilogue, not the tensor core, bounds
+// this kernel at gs = 64 and gs = 128.
 // Every mbarrier wait is bounded.
-#include "gemm_common.cuh"
+#include "grouped_common.cuh"
 
 namespace cider {
-
-constexpr uint32_t kPartialBias = 0x4B400000u;  // bits of 1.5 * 2^23
-constexpr int kScaleSlots = 4;                   // per-warp scale ring depth
 
 template <int MODE>
 struct GroupedCfg {
@@ -48,7 +53,10 @@ struct GroupedCfg {
     static constexpr int STG_BYTES = 32 * 32 * 2;  // one 32 x 32 output box
     static constexpr int STG_PER_WARP = 2;
     static constexpr int SCL_BYTES = EPI_COLS * 4;  // one group's scales for one warp
-    static constexpr int EXTRA = EPI_WARPS * (STG_PER_WARP * STG_BYTES + kScaleSlots * SCL_BYTES);
+    // constant f16 operands of the bias MMA (128 x 16 elements each), filled to
+    // twice their extent so any reading of the descriptor strides stays inside
+    static constexpr int BIAS_BYTES = 2 * 128 * 16 * 2;
+    static constexpr int EXTRA = EPI_WARPS * (STG_PER_WARP * STG_BYTES + kScaleSlots * SCL_BYTES) + 2 * BIAS_BYTES;
     static constexpr int NB = 4;                     // TMEM partial buffers
     static constexpr int TMEM_COLS = NB * BN;        // 512
     static constexpr int BAR_BYTES = 8 * (3 * 8 + 2 * NB) + 16;
@@ -59,94 +67,8 @@ struct GroupedCfg {
     static_assert(SMEM_BYTES <= kSmemMax, "shared memory");
 };
 
-__device__ __forceinline__ uint64_t pack_u32x2(uint32_t lo, uint32_t hi) {
-    return (static_cast<uint64_t>(hi) << 32) | lo;
-}
-__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
-__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, uint32_t v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
-        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
-        "r"(v)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, uint32_t v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
-        "r"(v)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// 16 bytes global -> shared, zero-filled when `bytes` is 0.
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint32_t bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // 10 or 12 warps: three of them share a 16K-register SM sub-partition, so
 // the launch bound caps registers at 168 per thread.
-// Scales of 4 consecutive columns as two packed pairs; the load is ordered
-// (volatile) so the compiler keeps scale registers short-lived.
-__device__ __forceinline__ void lds_scale4(const uint8_t* p, uint64_t& a, uint64_t& b) {
-    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(smem_u32(p)) : "memory");
-}
-
-// sum += (partial - preset) * scale for 16 columns, two per instruction; the
-// next 16 bytes of scales are loaded while the current ones are used.
-__device__ __forceinline__ void rescale16(uint64_t* sum2, const uint32_t (&r)[16], const uint8_t* scales,
-                                          uint64_t neg_bias2) {
-    uint64_t a0, a1, b0, b1;
-    lds_scale4(scales, a0, a1);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        if (j + 1 < 4) lds_scale4(scales + 16 * (j + 1), b0, b1);
-        sum2[2 * j] = f32x2_fma(f32x2_add(pack_u32x2(r[4 * j], r[4 * j + 1]), neg_bias2), a0, sum2[2 * j]);
-        sum2[2 * j + 1] = f32x2_fma(f32x2_add(pack_u32x2(r[4 * j + 2], r[4 * j + 3]), neg_bias2), a1, sum2[2 * j + 1]);
-        a0 = b0;
-        a1 = b1;
-    }
-}
-
-// Test mode: 16 per-group INT32 partials of one row (preset removed).
-__device__ __forceinline__ void store_partial16(const GemmArgs& p, const uint32_t (&r)[16], int g, int m, bool mvalid,
-                                                int n0) {
-    if (!mvalid) return;
-    int32_t* out = static_cast<int32_t*>(p.y) + (static_cast<int64_t>(g) * p.M + m) * p.N;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        if (n0 + 4 * j < p.N)
-            *reinterpret_cast<int4*>(out + n0 + 4 * j) =
-                make_int4(static_cast<int>(r[4 * j] - kPartialBias), static_cast<int>(r[4 * j + 1] - kPartialBias),
-                          static_cast<int>(r[4 * j + 2] - kPartialBias), static_cast<int>(r[4 * j + 3] - kPartialBias));
-}
-
 template <int MODE, typename TY>
 __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
     k_gemm_grouped(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -162,7 +84,9 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
     uint8_t* sBP = sB + S * C::B_BYTES;
     uint8_t* sStg = sBP + S * C::BP_BYTES;                                 // [8 warps][2] boxes
     uint8_t* sScl = sStg + C::EPI_WARPS * C::STG_PER_WARP * C::STG_BYTES;  // [8 warps][slots][64 floats]
-    uint64_t* full = reinterpret_cast<uint64_t*>(sScl + C::EPI_WARPS * kScaleSlots * C::SCL_BYTES);
+    uint8_t* sBiasA = sScl + C::EPI_WARPS * kScaleSlots * C::SCL_BYTES;   // 128 x 16 f16 of 64.0
+    uint8_t* sBiasB = sBiasA + C::BIAS_BYTES;                            // 128 x 16 f16 of 12288.0
+    uint64_t* full = reinterpret_cast<uint64_t*>(sBiasB + C::BIAS_BYTES);
     uint64_t* empty = full + 8;
     uint64_t* conv = empty + 8;
     uint64_t* accf = conv + 8;
@@ -180,7 +104,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&conv[s], C::CONV_WARPS * 32);
+            if (C::W4) mbar_init(&conv[s], C::CONV_WARPS * 32);
         }
         for (int b = 0; b < NB; ++b) {
             mbar_init(&accf[b], 1);
@@ -195,6 +119,15 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
         if (MODE != kModeI32G) tma_prefetch_desc(&tmY);
     }
     if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    // Operands of the bias MMA: every element of A is 64 (f16 0x5400) and of B
+    // 12288 (f16 0x7200), so each output is a sum of 16 products
+    // 64 * 12288 = 12582912 = 1.5 * 2^23 (all exact in fp32), whatever the
+    // operand layout.
+    for (int i = threadIdx.x; i < 2 * C::BIAS_BYTES / 16; i += C::THREADS) {
+        const uint32_t v = i < C::BIAS_BYTES / 16 ? 0x54005400u : 0x72007200u;
+        reinterpret_cast<uint4*>(sBiasA)[i] = make_uint4(v, v, v, v);
+    }
+    fence_async_smem();  // visible to the tensor core
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -229,6 +162,10 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_i8(C::BM, BN);
+            constexpr uint32_t idesc_bias = umma_idesc_f16(C::BM, BN);
+            // unswizzled K-major 16-column f16 tiles: core matrices 128 B, 2 along K, 256 B apart along rows
+            const uint64_t bias_adesc = umma_desc_plain(smem_u32(sBiasA), 128, 256);
+            const uint64_t bias_bdesc = umma_desc_plain(smem_u32(sBiasB), 128, 256);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t acc_i = 0;  // partial-buffer uses so far
@@ -245,13 +182,14 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
                     const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
                     for (int j = 0; j < gpk && g < G; ++j, ++g) {
                         const uint32_t b = acc_i % NB;
-                        // use u of buffer b waits for phase u: the preset after use u-1 (or the initial preset)
+                        // use u of buffer b waits for phase u: use u-1 read out (or the initial release)
                         if (!mbar_wait(&acce[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t d = tmem_base + b * BN;
+                        umma_f16_overwrite(d, bias_adesc, bias_bdesc, idesc_bias);  // D = bits of 1.5 * 2^23
                         for (int kk = 0; kk < steps; ++kk) {
                             const int off = (j * steps + kk) * kUmmaK;
-                            umma_i8(d, adesc + (off >> 4), bdesc + (off >> 4), idesc, 1u);  // onto the preset
+                            umma_i8(d, adesc + (off >> 4), bdesc + (off >> 4), idesc, 1u);  // onto the bias
                         }
                         umma_commit(&accf[b]);
                         ++acc_i;
@@ -270,16 +208,9 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         uint8_t* stg = sStg + ew * C::STG_PER_WARP * C::STG_BYTES;
         uint8_t* scl = sScl + ew * kScaleSlots * C::SCL_BYTES;
-        // preset every partial buffer, then report it free (phase 0 of acce)
-        for (int b = 0; b < NB; ++b) {
-            tmem_st_32x32b_x32(tmem_base + lane_addr + b * BN + half * C::EPI_COLS, kPartialBias);
-            tmem_st_32x32b_x32(tmem_base + lane_addr + b * BN + half * C::EPI_COLS + 32, kPartialBias);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
+        // every partial buffer starts free (phase 0 of acce)
         if (lane == 0)
-            for (int b = 0; b < NB; ++b) mbar_arrive(&acce[b]);
+            for (int b = 0; b < NB; ++b) mbar_arrive_relaxed(&acce[b]);
 
         // Scale prefetch runs kScaleSlots-1 groups ahead of the rescale along this
         // CTA's (tile, group) sequence; a running pointer avoids divisions.
@@ -344,10 +275,14 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     tmem_ld_wait();  // rr[c & 1] = columns 16c .. 16c+15 of group g
-                    tmem_st_32x32b_x16(taddr + 16 * c, kPartialBias);
                     if (c < 3) {
                         tmem_ld_32x32b_x16(taddr + 16 * (c + 1), rr[(c + 1) & 1]);
-                    } else if (g + 1 < G) {  // first step of the next group
+                    } else {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_relaxed(&acce[b]);  // buffer b read out
+                    }
+                    if (c == 3 && g + 1 < G) {  // first step of the next group
                         const uint32_t bn = (acc_i + 1) % NB;
                         if (!mbar_wait(&accf[bn], ((acc_i + 1) / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
                         tc_fence_after();
@@ -359,10 +294,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
                         rescale16(sum2 + 8 * c, rr[c & 1], slot + 64 * c, neg_bias2);
                 }
                 if (!ok) break;
-                tmem_st_wait();  // buffer b holds the preset again
-                tc_fence_before();
-                __syncwarp();  // also: every lane has read the scale slot before it is refilled
-                if (lane == 0) mbar_arrive(&acce[b]);
+                __syncwarp();  // every lane has read the scale slot before it is refilled
                 ++acc_i;
             }
             if (!ok) break;
