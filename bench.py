@@ -424,7 +424,7 @@ def bench_rows(device, pk, steps, warmup):
             n = rotating(N * K + M * K * 3 + M * N * 2)
             wgs = [wg] + [wg.roll(i, 0).contiguous() for i in range(1, n)]
             ys = [torch.empty((M, N), dtype=torch.float16, device=device) for _ in range(n)]
-            wsp = torch.empty((max(1, cider.cider_workspace_bytes(M, K)),), dtype=torch.uint8, device=device)
+            wsp = torch.empty((max(1, cider.cider_workspace_bytes_mnk(M, N, K)),), dtype=torch.uint8, device=device)
             ms = graph_time(lambda i: cider.cider_w8a8_linear_pg(x, wgs[i % n], sg, gs, y=ys[i % n], workspace=wsp),
                             steps, warmup)
             record("w8a8_linear_pg", ms, 2.0 * M * N * K, N * K + sg.numel() * 4 + M * K * 2 + M * N * 2,
@@ -439,7 +439,7 @@ def bench_rows(device, pk, steps, warmup):
     n = rotating(N * K // 2 + M * K * 3 + M * N * 2)
     p4s = [p4] + [p4.roll(i, 0).contiguous() for i in range(1, n)]
     ys = [torch.empty((M, N), dtype=torch.float16, device=device) for _ in range(n)]
-    wsp = torch.empty((cider.cider_workspace_bytes(M, K),), dtype=torch.uint8, device=device)
+    wsp = torch.empty((cider.cider_workspace_bytes_mnk(M, N, K),), dtype=torch.uint8, device=device)
     ms = graph_time(lambda i: cider.cider_w4a8_linear_pg(x, p4s[i % n], s4, gs, y=ys[i % n], workspace=wsp), steps, warmup)
     record("w4a8_linear_pg", ms, 2.0 * M * N * K, N * K // 2 + s4.numel() * 4 + M * K * 2 + M * N * 2, gs=gs, M=M, N=N, K=K)
     del p4s, ys
@@ -487,6 +487,8 @@ ROW_CASES = {
     "pc_m8192": ("pc", 8192, 10240, 2560, 0),
     "pg128_m1": ("pg", 1, 2560, 10240, 128), "pg128_m4096": ("pg", 4096, 2560, 10240, 128),
     "pg64_m1": ("pg", 1, 2560, 10240, 64), "pg64_m4096": ("pg", 4096, 2560, 10240, 64),
+    "pg128_m128": ("pg", 128, 2560, 10240, 128), "pg64_m128": ("pg", 128, 2560, 10240, 64),
+    "pg64_m1024": ("pg", 1024, 2560, 10240, 64), 
     "w4a8_m2048": ("w4", 2048, 12288, 4096, 64),
     "stack_8b": ("stack", 2048, 0, 0, 0),
 }
@@ -516,7 +518,7 @@ def run_row(args):
         call = lambda y, ws_: cider.cider_w4a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)
     del W
     y = torch.empty((M, N), dtype=torch.float16, device=device)
-    wsp = torch.empty((max(1, cider.cider_workspace_bytes(M, K)),), dtype=torch.uint8, device=device)
+    wsp = torch.empty((max(1, cider.cider_workspace_bytes_mnk(M, N, K)),), dtype=torch.uint8, device=device)
     ms = graph_time(lambda i: call(y, wsp), args.steps, args.warmup)
     cider.cider_device_status()
     print(json.dumps({"row": args.row, "kind": kind, "M": M, "N": N, "K": K, "gs": gs, "ms": ms,

@@ -96,6 +96,14 @@ CIDER_API cider_status_t cider_device_status(void* stream);
  * (M <= cider_get_small_m_threshold()), which keeps q in shared memory. */
 CIDER_API size_t cider_workspace_bytes(int64_t M, int64_t K);
 
+/* Workspace that lets a linear of shape M x N x K take its fastest path on
+ * the current device: cider_workspace_bytes(M, K), plus, for the per-group
+ * linears when their 128 x 128 output tiles would leave at least half of the
+ * SMs idle, room for split-K partial sums (fp32 [splits][M][N], 256-byte
+ * aligned, after scale_x).  A per-group linear given less than this (but at
+ * least cider_workspace_bytes(M, K)) runs without splitting K. */
+CIDER_API size_t cider_workspace_bytes_mnk(int64_t M, int64_t N, int64_t K);
+
 /* Calls with 1 <= M <= threshold use the fused small-M (decode-shaped) kernel;
  * larger M use quantize + the tcgen05 GEMM.  The threshold is process-wide;
  * 0 sends every call to the GEMM path.  Values above 16 are rejected.  The
@@ -126,7 +134,9 @@ CIDER_API cider_status_t cider_w8a8_linear_pc(const void* x, cider_dtype_t xdt, 
 /* W8A8 linear, per-group weight scales along K (gs = 64 or 128; Cider README,
  * table "W8A8 量化粒度"; juejin post, section "三种量化粒度的实现").
  * scale_w: [K/gs][N] fp32 (group-major).  The INT32 partial sum of each group
- * is rescaled by its scale in fp32 and the rescaled partials are summed. */
+ * is rescaled by its scale in fp32 and the rescaled partials are summed.
+ * With a workspace of cider_workspace_bytes_mnk(M, N, K) bytes, small tile
+ * counts split K into pieces whose fp32 sums are added by a second kernel. */
 CIDER_API cider_status_t cider_w8a8_linear_pg(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
                                     const int8_t* w, const float* scale_w, int64_t N, int64_t gs,
                                     void* y, cider_dtype_t ydt,
@@ -217,6 +227,13 @@ CIDER_API cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8
  * 2 = single-CTA 128x256 tiles, 3 = CTA-pair 256x256 tiles.  Lets tests cover
  * every variant on small shapes. */
 CIDER_API cider_status_t cider_test_set_gemm_variant(int variant);
+/* Forces the split-K piece count of the per-group GEMM for later calls
+ * (process-wide): 0 = automatic (default), 1 = never split, 2 .. 16 = that
+ * many K pieces per tile (fewer when K has fewer 128-wide blocks).  The INT32
+ * test export honours it without a workspace (it writes per-group partials);
+ * the per-group linears need cider_workspace_bytes_mnk(M, N, K) bytes, read
+ * after setting it, or they do not split. */
+CIDER_API cider_status_t cider_test_set_split_k(int splits);
 /* Exercises the bounded-wait path of the kernels without a fault: one warp
  * waits on an mbarrier that nothing arrives on and gives up after limit_ns
  * (1 .. 1e8).  The next cider_device_status() then returns CIDER_ERR_TIMEOUT

@@ -77,3 +77,73 @@ def test_w4a8_linear_ragged(M, N, K, gs):
     wp, sw = oracle.quantize_weight_int4_pg(synth.weights(N, K, seed=K + 7), gs)
     y = cider.cider_w4a8_linear_pg(dev_bits(x, oracle.F16), dev(wp), _gmajor(sw), gs)
     check_y(y, oracle.w4a8_linear_pg(x, wp, sw, gs), oracle.F16)
+
+
+# ---------------------------------------------------------------- split K
+
+@pytest.fixture
+def split_k():
+    yield cider.cider_test_set_split_k
+    cider.cider_test_set_split_k(0)
+
+
+@pytest.mark.parametrize("splits", [2, 3, 7])
+@pytest.mark.parametrize("gs", [64, 128])
+@pytest.mark.parametrize("M,N,K", [(130, 264, 1280), (64, 136, 192), (257, 8, 2560)])
+def test_gemm_i32_grouped_split_pieces(split_k, splits, gs, M, N, K):
+    """Forced K pieces: every (tile, piece) unit writes its own groups'
+    partials, so the result is the same bit for bit (K = 192 at gs = 64 leaves
+    the last 128-wide block with one group; K = 192 has only 2 blocks, so 3
+    and 7 pieces collapse to 2)."""
+    if K % gs:
+        pytest.skip("gs must divide K")
+    split_k(splits)
+    q, w = _codes(M, N, K, seed=7 * M + N + K + gs + splits)
+    acc_g = cider.cider_test_gemm_i32_grouped(dev(q), dev(w), gs)
+    np.testing.assert_array_equal(acc_g.cpu().numpy(), oracle.gemm_i32_grouped(q, w, gs))
+
+
+@pytest.mark.parametrize("splits", [0, 2, 5])
+@pytest.mark.parametrize("gs", [64, 128])
+@pytest.mark.parametrize("M,N,K", [(128, 2560, 10240), (40, 264, 2560), (300, 520, 1280), (1024, 2560, 4096)])
+def test_linear_pg_split(split_k, splits, gs, M, N, K):
+    """Per-group linear with automatic (0) or forced K pieces: fp32 piece sums
+    added by the reduce kernel, then scale_x and rounding.  At 1024 x 2560 the
+    automatic plan runs 148 whole tiles and splits the 12 tiles of the tail
+    round (rows 512.., columns 2304..), so both kinds of unit are checked."""
+    cider.cider_set_small_m_threshold(4)
+    split_k(splits)
+    x = act(M, K, seed=M + N + K + gs + splits)
+    qw, sw = oracle.quantize_weight_pg(synth.weights(N, K, seed=N + K), gs)
+    y = cider.cider_w8a8_linear_pg(dev_bits(x, oracle.F16), dev(qw), _gmajor(sw), gs)
+    rows = np.arange(0, M, max(1, M // 40))
+    check_y(y, oracle.linear_pg(x[rows], qw, sw, gs), oracle.F16, rows=rows)
+
+
+@pytest.mark.parametrize("dt", [oracle.F16, oracle.BF16])
+def test_w4a8_linear_split(split_k, dt):
+    M, N, K, gs = 128, 1032, 4096, 64
+    split_k(0)
+    x = act(M, K, seed=77, dt=dt)
+    wp, sw = oracle.quantize_weight_int4_pg(synth.weights(N, K, seed=78), gs)
+    y = cider.cider_w4a8_linear_pg(dev_bits(x, dt), dev(wp), _gmajor(sw), gs)
+    check_y(y, oracle.w4a8_linear_pg(x, wp, sw, gs, xdt=dt, ydt=dt), dt)
+
+
+def test_split_needs_the_larger_workspace(split_k):
+    """A workspace of cider_workspace_bytes(M, K) runs the unsplit kernel; one
+    of cider_workspace_bytes_mnk(M, N, K) splits K; both give the oracle's
+    answer, and the automatic split is > 1 for this shape (20 tiles)."""
+    M, N, K, gs = 128, 2560, 10240, 128
+    assert cider.cider_workspace_bytes_mnk(M, N, K) > cider.cider_workspace_bytes(M, K)
+    x = act(M, K, seed=5)
+    qw, sw = oracle.quantize_weight_pg(synth.weights(N, K, seed=6), gs)
+    xd, wd, sd = dev_bits(x, oracle.F16), dev(qw), _gmajor(sw)
+    small = torch.empty((cider.cider_workspace_bytes(M, K),), dtype=torch.uint8, device="cuda")
+    big = torch.empty((cider.cider_workspace_bytes_mnk(M, N, K),), dtype=torch.uint8, device="cuda")
+    y_plain = cider.cider_w8a8_linear_pg(xd, wd, sd, gs, workspace=small)
+    y_split = cider.cider_w8a8_linear_pg(xd, wd, sd, gs, workspace=big)
+    rows = np.arange(0, M, 5)
+    ref = oracle.linear_pg(x[rows], qw, sw, gs)
+    check_y(y_plain, ref, oracle.F16, rows=rows)
+    check_y(y_split, ref, oracle.F16, rows=rows)

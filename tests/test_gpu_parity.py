@@ -246,6 +246,18 @@ def test_grouped_small_m_and_tensor_core_paths_agree(mode, M, small_m):
 
 
 def test_gemm_q_entry_points_match_linears():
+    """The pre-quantized entry points run the same arithmetic as the linears,
+    bit for bit.  The per-group linears would split K here (6 tiles), which
+    adds fp32 piece sums in another order, so splitting is turned off; the
+    split path has its own tests against the oracle."""
+    cider.cider_test_set_split_k(1)
+    try:
+        _gemm_q_entry_points_match_linears()
+    finally:
+        cider.cider_test_set_split_k(0)
+
+
+def _gemm_q_entry_points_match_linears():
     M, N, K, gs = 200, 264, 1024, 128
     x = act(M, K, seed=1)
     xd = dev_bits(x, F16)

@@ -39,6 +39,7 @@ _SIGNATURES = {
     "cider_last_error": (ctypes.c_char_p, []),
     "cider_device_status": (_INT, [_P]),
     "cider_workspace_bytes": (_SZ, [_I64, _I64]),
+    "cider_workspace_bytes_mnk": (_SZ, [_I64, _I64, _I64]),
     "cider_set_small_m_threshold": (_INT, [_I64]),
     "cider_get_small_m_threshold": (_I64, []),
     "cider_quantize_act": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P]),
@@ -57,6 +58,7 @@ _SIGNATURES = {
     "cider_test_gemm_i32_grouped": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _P, _P]),
     "cider_test_unpack_int4": (_INT, [_P, _I64, _I64, _P, _P]),
     "cider_test_set_gemm_variant": (_INT, [_INT]),
+    "cider_test_set_split_k": (_INT, [_INT]),
     "cider_test_bounded_wait": (_INT, [_I64, _P]),
 }
 EXPORTS = tuple(_SIGNATURES)
@@ -116,6 +118,10 @@ def cider_workspace_bytes(M: int, K: int) -> int:
     return int(lib().cider_workspace_bytes(M, K))
 
 
+def cider_workspace_bytes_mnk(M: int, N: int, K: int) -> int:
+    return int(lib().cider_workspace_bytes_mnk(M, N, K))
+
+
 def cider_set_small_m_threshold(threshold: int):
     _check("cider_set_small_m_threshold", lib().cider_set_small_m_threshold(threshold))
 
@@ -137,8 +143,8 @@ def cider_quantize_act(x, q=None, scale_x=None, stream=None):
     return q, scale_x
 
 
-def _workspace(M, K, device, workspace):
-    need = cider_workspace_bytes(M, K)
+def _workspace(M, K, device, workspace, N=0):
+    need = cider_workspace_bytes_mnk(M, N, K) if N else cider_workspace_bytes(M, K)
     if workspace is None and need:
         workspace = torch.empty((need,), dtype=torch.uint8, device=device)
     return workspace, (0 if workspace is None else workspace.numel() * workspace.element_size())
@@ -167,7 +173,7 @@ def cider_w8a8_linear_pg(x, w, scale_w, gs, y=None, out_dtype=None, workspace=No
     M, K = x.shape
     N = w.shape[0]
     y = _out(y, M, N, out_dtype or x.dtype, x.device)
-    ws, ws_bytes = _workspace(M, K, x.device, workspace)
+    ws, ws_bytes = _workspace(M, K, x.device, workspace, N)
     _check("cider_w8a8_linear_pg", lib().cider_w8a8_linear_pg(
         _ptr(x), _DT[x.dtype], M, K, _ptr(w), _ptr(scale_w), N, gs, _ptr(y), _DT[y.dtype],
         _ptr(ws), ws_bytes, _stream(stream, x.device)))
@@ -180,7 +186,7 @@ def cider_w4a8_linear_pg(x, w_packed, scale_w, gs, y=None, out_dtype=None, works
     M, K = x.shape
     N = w_packed.shape[0]
     y = _out(y, M, N, out_dtype or x.dtype, x.device)
-    ws, ws_bytes = _workspace(M, K, x.device, workspace)
+    ws, ws_bytes = _workspace(M, K, x.device, workspace, N)
     _check("cider_w4a8_linear_pg", lib().cider_w4a8_linear_pg(
         _ptr(x), _DT[x.dtype], M, K, _ptr(w_packed), _ptr(scale_w), N, gs, _ptr(y), _DT[y.dtype],
         _ptr(ws), ws_bytes, _stream(stream, x.device)))
@@ -298,6 +304,11 @@ def cider_test_gemm_i32_grouped(q, w, gs, acc_g=None, stream=None):
 def cider_test_set_gemm_variant(variant: int):
     """0 automatic, 1 single-CTA 128x128, 2 single-CTA 128x256, 3 CTA-pair 256x256."""
     _check("cider_test_set_gemm_variant", lib().cider_test_set_gemm_variant(variant))
+
+
+def cider_test_set_split_k(splits: int):
+    """0 automatic split-K of the per-group GEMM, 1 never, 2..16 forced pieces."""
+    _check("cider_test_set_split_k", lib().cider_test_set_split_k(splits))
 
 
 def cider_test_bounded_wait(limit_ns: int, stream=None, device=None):

@@ -129,6 +129,35 @@ cider_status_t check_gs(int64_t K, int64_t gs, bool w4) {
 }
 
 std::atomic<int> g_gemm_variant{kGemmAuto};  // test override
+std::atomic<int> g_split_override{0};         // test override of the split-K piece count (0 = automatic)
+constexpr int kMaxSplits = 16;
+
+// Split-K plan of the per-group GEMM (128 x 128 tiles on a persistent grid of
+// one CTA per SM): the tiles that fill whole rounds run over all of K; the
+// R tiles of the last, partial round are cut into S K pieces so that their
+// R * S units fill that round (S <= SMs / R, >= 4 k-blocks per piece, <= 16).
+// A forced piece count (test override) splits every tile.
+struct SplitPlan {
+    int full_tiles, splits;
+    int64_t tail_tiles;
+};
+SplitPlan grouped_split_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
+    const int64_t tiles = ((M + 127) / 128) * ((N + 127) / 128);
+    const int forced = g_split_override.load();
+    if (forced > 1) return {0, forced, tiles};
+    if (forced == 1 || num_sms <= 0) return {static_cast<int>(tiles), 1, 0};
+    const int64_t full = tiles / num_sms * num_sms, tail = tiles - full;
+    if (tail == 0) return {static_cast<int>(tiles), 1, 0};
+    int64_t s = std::min<int64_t>(num_sms / tail, ((K + 127) / 128) / 4);
+    s = std::min<int64_t>(s, kMaxSplits);
+    if (s < 2) return {static_cast<int>(tiles), 1, 0};
+    return {static_cast<int>(full), static_cast<int>(s), tail};
+}
+
+// Bytes of fp32 partial sums: one 128 x 128 slot per K piece of a tail tile.
+size_t part_bytes(const SplitPlan& sp) {
+    return sp.splits > 1 ? align256(static_cast<size_t>(sp.tail_tiles) * sp.splits * 128 * 128 * 4) : 0;
+}
 
 // Per-channel GEMM variant: the CTA-pair 256x256 tile when it still gives
 // every pair of SMs a tile, else single-CTA tiles of 128x256 or 128x128.
@@ -143,7 +172,7 @@ int pick_variant(int64_t M, int64_t N, int num_sms) {
 
 cider_status_t run_gemm(int mode, const int8_t* q, const float* sx, int64_t M, int64_t K,
                         const void* w, const float* sw, int64_t N, int64_t gs, void* y, int ydt,
-                        const DeviceInfo* d, cudaStream_t st) {
+                        const DeviceInfo* d, cudaStream_t st, SplitPlan sp = {0, 1, 0}, float* part = nullptr) {
     GemmLaunch L;
     L.mode = mode;
     L.q = q;
@@ -157,6 +186,9 @@ cider_status_t run_gemm(int mode, const int8_t* q, const float* sx, int64_t M, i
     L.gs = static_cast<int>(gs);
     L.ydt = ydt;
     L.variant = (mode == kModePC || mode == kModeI32) ? pick_variant(M, N, d->num_sms) : kGemmSingle128;
+    L.full_tiles = sp.full_tiles;
+    L.splits = sp.splits;
+    L.part = part;
     L.num_sms = d->num_sms;
     L.status = d->status;
     cudaError_t e = launch_gemm(L, st);
@@ -194,12 +226,25 @@ cider_status_t linear(int mode, const void* x, int xdt, int64_t M, int64_t K, co
     if (!ws || ws_bytes < need)
         return fail(CIDER_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, ws ? ws_bytes : 0);
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(CIDER_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    if (overlap(ry, rng(ws, need))) return fail(CIDER_ERR_INVALID_ARG, "y overlaps the workspace");
+    // split-K partial sums of the per-group GEMM, when the workspace holds them
+    SplitPlan plan{0, 1, 0};
+    float* part = nullptr;
+    size_t used = need;
+    if (mode != kModePC) {
+        const SplitPlan sp = grouped_split_plan(M, N, K, d->num_sms);
+        const size_t pb = part_bytes(sp);
+        if (sp.splits > 1 && ws_bytes >= need + pb) {
+            plan = sp;
+            part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + need);
+            used = need + pb;
+        }
+    }
+    if (overlap(ry, rng(ws, used))) return fail(CIDER_ERR_INVALID_ARG, "y overlaps the workspace");
     int8_t* q = static_cast<int8_t*>(ws);
     float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(static_cast<size_t>(M) * K));
     cudaError_t e = launch_quantize_act(x, xdt, M, static_cast<int>(K), q, sx, st);
     if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
-    return run_gemm(mode, q, sx, M, K, w, sw, N, gs, y, ydt, d, st);
+    return run_gemm(mode, q, sx, M, K, w, sw, N, gs, y, ydt, d, st, plan, part);
 }
 
 cider_status_t gemm_q(int mode, const int8_t* q, const float* sx, int64_t M, int64_t K, const void* w,
@@ -301,6 +346,21 @@ cider_status_t cider_device_status(void* stream) {
 size_t cider_workspace_bytes(int64_t M, int64_t K) {
     if (M <= 0 || K <= 0 || small_m_path(M, K)) return 0;
     return align256(static_cast<size_t>(M) * K) + align256(static_cast<size_t>(M) * 4);
+}
+
+size_t cider_workspace_bytes_mnk(int64_t M, int64_t N, int64_t K) {
+    const size_t need = cider_workspace_bytes(M, K);
+    if (need == 0 || N <= 0) return need;
+    DeviceInfo* d = nullptr;
+    if (device_info(&d) != CIDER_OK) return need;
+    return need + part_bytes(grouped_split_plan(M, N, K, d->num_sms));
+}
+
+cider_status_t cider_test_set_split_k(int splits) {
+    if (splits < 0 || splits > kMaxSplits)
+        return fail(CIDER_ERR_INVALID_ARG, "splits %d outside [0, %d]", splits, kMaxSplits);
+    g_split_override.store(splits);
+    return CIDER_OK;
 }
 
 cider_status_t cider_set_small_m_threshold(int64_t threshold) {
@@ -446,7 +506,10 @@ cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8_t* w, int
     if (M == 0) return CIDER_OK;
     DeviceInfo* d = nullptr;
     if ((s = device_info(&d)) != CIDER_OK) return s;
-    return run_gemm(kModeI32G, q, nullptr, M, K, w, nullptr, N, gs, acc_g, 0, d, static_cast<cudaStream_t>(stream));
+    const int forced = g_split_override.load();
+    const SplitPlan sp{0, forced > 1 ? forced : 1, 0};
+    return run_gemm(kModeI32G, q, nullptr, M, K, w, nullptr, N, gs, acc_g, 0, d, static_cast<cudaStream_t>(stream),
+                    sp, nullptr);
 }
 
 cider_status_t cider_test_set_gemm_variant(int variant) {

@@ -35,6 +35,9 @@ struct GemmLaunch {
     int M, N, K, gs;
     int ydt;           // 0 fp16, 1 bf16
     int variant;       // per-channel modes: kGemmSingle128, kGemmSingle256 or kGemmPair
+    int full_tiles;    // grouped modes: tiles that run over all of K (the rest are split)
+    int splits;        // grouped modes: K pieces of each later tile (1 = no split)
+    float* part;       // grouped modes with splits > 1: fp32 partial sums, [piece slot][128][128]
     int num_sms;
     unsigned* status;  // device status word
 };

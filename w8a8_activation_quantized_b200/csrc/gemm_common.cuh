@@ -18,6 +18,9 @@ struct GemmArgs {
     int M, N, K;
     int gs;             // group size (grouped modes)
     int num_m_blocks, num_n_blocks, num_k_blocks;
+    // grouped modes: tiles [0, full_tiles) run over all of K; every later tile
+    // is cut into `splits` K pieces of kb_per_split k-blocks
+    int full_tiles, splits, kb_per_split;
     const float* sx;    // [M]
     const float* sw;    // [N] or [G][N]
     void* y;            // [M][N] output (fp16/bf16), or int32 acc / acc_g in test modes
@@ -62,6 +65,16 @@ __device__ __forceinline__ void stage_row32_f(uint8_t* box, int r, const float (
     for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(row + ((j ^ sw) << 4)) = pack8_out<TY>(v + 8 * j);
 }
 
+// Row `r` of a 32 x 16 staging box of fp32 values, in the same 64-byte swizzle
+// (a row is 64 bytes either way).
+__device__ __forceinline__ void stage_row16_f32(uint8_t* box, int r, const float* v) {
+    uint8_t* row = box + r * 64;
+    const int sw = (r >> 1) & 3;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<float4*>(row + ((j ^ sw) << 4)) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+}
+
 // ---------------------------------------------------------------------------
 // Host-side tensor maps
 // ---------------------------------------------------------------------------
@@ -85,6 +98,17 @@ inline bool make_map_out(CUtensorMap* map, void* y, int M, int N, int ydt) {
     cuuint32_t estr[2] = {1, 1};
     return encode_tensor_map(map, ydt == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, y,
                              dims, strides, box, estr, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// Map of split-K partial sums: `slots` tile-local blocks of rows x cols fp32,
+// for TMA stores of 32-row x 16-column boxes.
+inline bool make_map_part(CUtensorMap* map, float* part, int rows, int cols, int slots) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slots)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 4, static_cast<cuuint64_t>(rows) * cols * 4};
+    cuuint32_t box[3] = {16, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return encode_tensor_map(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, part, dims, strides, box, estr,
+                             CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 }  // namespace cider

@@ -27,12 +27,21 @@
 //    its last TMEM load of it has completed.  Group scales reach shared memory
 //    ahead of use through a per-warp cp.async ring; the finished tile leaves
 //    through swizzled staging boxes and TMA stores.
+// Split K of the tail.  The tiles that fill whole rounds of the persistent
+// grid run over all of K; the tiles of the last, partial round are cut into
+// `splits` K pieces so that their units fill that round.  A piece's running
+// sum covers its own groups only and goes out as fp32 partial sums into a
+// tile-local 128 x 128 slot (3-D TMA store); k_splitk_reduce adds a tile's
+// pieces in order, multiplies by scale_x and rounds.  With few tiles (small
+// M) every tile is a tail tile.
 // Cost model (measured on B200): per group and 128 x 128 tile the epilogue
 // moves every partial TMEM -> registers once and issues two fp32 operations
 // per partial; these do not overlap, which puts the floor near 384 cycles
 // per group per SM sub-partition -- the epilogue, not the tensor core, bounds
 // this kernel at gs = 64 and gs = 128.
 // Every mbarrier wait is bounded.
+#include <algorithm>
+
 #include "grouped_common.cuh"
 
 namespace cider {
@@ -67,12 +76,38 @@ struct GroupedCfg {
     static_assert(SMEM_BYTES <= kSmemMax, "shared memory");
 };
 
+// Work unit u: a whole tile (u < full_tiles) or one K piece of a tail tile;
+// its tile coordinates, k-blocks [kb0, kb1), groups [g0, g1) and, for a
+// piece, the slot of its partial sums (-1 for a whole tile).
+struct GroupUnit {
+    int mb, nb, kb0, kb1, g0, g1, slot;
+};
+__device__ __forceinline__ GroupUnit group_unit(const GemmArgs& p, int u, int G, int gpk) {
+    GroupUnit w;
+    int t, piece;
+    if (u < p.full_tiles) {
+        t = u;
+        piece = -1;
+    } else {
+        const int v = u - p.full_tiles;
+        t = p.full_tiles + v / p.splits;
+        piece = v % p.splits;
+    }
+    tile_coords(t, p.num_m_blocks, p.num_n_blocks, w.mb, w.nb);
+    w.slot = piece < 0 ? -1 : (t - p.full_tiles) * p.splits + piece;
+    w.kb0 = piece < 0 ? 0 : piece * p.kb_per_split;
+    w.kb1 = piece < 0 ? p.num_k_blocks : min(w.kb0 + p.kb_per_split, p.num_k_blocks);
+    w.g0 = w.kb0 * gpk;
+    w.g1 = min(w.kb1 * gpk, G);
+    return w;
+}
+
 // 10 or 12 warps: three of them share a 16K-register SM sub-partition, so
 // the launch bound caps registers at 168 per thread.
 template <int MODE, typename TY>
 __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
     k_gemm_grouped(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
+                   const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmP, GemmArgs p) {
     using C = GroupedCfg<MODE>;
     constexpr int S = C::STAGES;
     constexpr int NB = C::NB;
@@ -96,8 +131,9 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int num_tiles = p.num_m_blocks * p.num_n_blocks;
+    const int num_units = p.full_tiles + (p.num_m_blocks * p.num_n_blocks - p.full_tiles) * p.splits;
     const int G = p.K / p.gs;
+    const int gpk = kBK / p.gs;  // groups per k-block: 1 or 2
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -143,17 +179,16 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
             uint32_t phase = 0;
             const uint32_t tx = C::A_BYTES + (C::W4 ? C::BP_BYTES : C::B_BYTES);
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                int mb, nb;
-                tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+                const GroupUnit w = group_unit(p, u, G, gpk);
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full[stage], tx);
-                    tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * kBK, mb * C::BM);
+                    tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * kBK, w.mb * C::BM);
                     if (C::W4)
-                        tma_load_2d(sBP + stage * C::BP_BYTES, &tmB, &full[stage], kb * (kBK / 2), nb * BN);
+                        tma_load_2d(sBP + stage * C::BP_BYTES, &tmB, &full[stage], kb * (kBK / 2), w.nb * BN);
                     else
-                        tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * kBK, nb * BN);
+                        tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * kBK, w.nb * BN);
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -171,16 +206,16 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
             uint32_t acc_i = 0;  // partial-buffer uses so far
             bool ok = true;
             const int steps = p.gs / kUmmaK;
-            const int gpk = kBK / p.gs;  // groups per stage: 1 or 2
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                int g = 0;
-                for (int kb = 0; kb < p.num_k_blocks && ok; ++kb) {
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+                const GroupUnit w = group_unit(p, u, G, gpk);
+                int g = w.g0;
+                for (int kb = w.kb0; kb < w.kb1 && ok; ++kb) {
                     if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
                     if (C::W4 && !mbar_wait(&conv[stage], phase, p.status, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
                     const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
-                    for (int j = 0; j < gpk && g < G; ++j, ++g) {
+                    for (int j = 0; j < gpk && g < w.g1; ++j, ++g) {
                         const uint32_t b = acc_i % NB;
                         // use u of buffer b waits for phase u: use u-1 read out (or the initial release)
                         if (!mbar_wait(&acce[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
@@ -213,28 +248,28 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
             for (int b = 0; b < NB; ++b) mbar_arrive_relaxed(&acce[b]);
 
         // Scale prefetch runs kScaleSlots-1 groups ahead of the rescale along this
-        // CTA's (tile, group) sequence; a running pointer avoids divisions.
-        int pf_t = blockIdx.x, pf_g = 0, pf_slot = 0, pf_col = 0;
-        auto pf_tile = [&]() {
-            if (pf_t < num_tiles) {
-                int mb, nb;
-                tile_coords(pf_t, p.num_m_blocks, p.num_n_blocks, mb, nb);
-                pf_col = nb * BN + half * C::EPI_COLS + 4 * lane;
+        // CTA's (unit, group) sequence; a running pointer avoids divisions.
+        int pf_u = blockIdx.x, pf_g = 0, pf_g1 = 0, pf_slot = 0, pf_col = 0;
+        auto pf_unit = [&]() {
+            if (pf_u < num_units) {
+                const GroupUnit w = group_unit(p, pf_u, G, gpk);
+                pf_g = w.g0;
+                pf_g1 = w.g1;
+                pf_col = w.nb * BN + half * C::EPI_COLS + 4 * lane;
             }
         };
-        pf_tile();
+        pf_unit();
         auto prefetch = [&]() {
-            if (MODE != kModeI32G && pf_t < num_tiles && lane < C::EPI_COLS / 4) {
+            if (MODE != kModeI32G && pf_u < num_units && lane < C::EPI_COLS / 4) {
                 const bool in = pf_col < p.N;
                 const float* src = p.sw + static_cast<int64_t>(pf_g) * p.N + (in ? pf_col : 0);
                 cp_async16(scl + pf_slot * C::SCL_BYTES + 16 * lane, src, in ? 16u : 0u);
             }
             cp_async_commit();
             pf_slot = (pf_slot + 1) % kScaleSlots;
-            if (++pf_g == G) {
-                pf_g = 0;
-                pf_t += gridDim.x;
-                pf_tile();
+            if (++pf_g == pf_g1) {
+                pf_u += gridDim.x;
+                pf_unit();
             }
         };
         for (int i = 0; i < kScaleSlots - 1; ++i) prefetch();
@@ -242,13 +277,12 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
         const uint64_t neg_bias2 = pack_u32x2(__float_as_uint(-12582912.0f), __float_as_uint(-12582912.0f));
         uint32_t acc_i = 0, nstore = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-            int mb, nb;
-            tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
-            const int m0 = mb * C::BM + quarter * 32;
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const GroupUnit w = group_unit(p, u, G, gpk);
+            const int m0 = w.mb * C::BM + quarter * 32;
             const int m = m0 + lane;
             const bool mvalid = m < p.M;
-            const int nw = nb * BN + half * C::EPI_COLS;
+            const int nw = w.nb * BN + half * C::EPI_COLS;
             uint64_t sum2[C::EPI_COLS / 2];
 #pragma unroll
             for (int j = 0; j < C::EPI_COLS / 2; ++j) sum2[j] = 0;
@@ -263,7 +297,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
                 tc_fence_after();
                 tmem_ld_32x32b_x16(tmem_base + lane_addr + b0 * BN + half * C::EPI_COLS, rr[0]);
             }
-            for (int g = 0; g < G && ok; ++g) {
+            for (int g = w.g0; g < w.g1 && ok; ++g) {
                 prefetch();
                 const uint32_t b = acc_i % NB;
                 const uint32_t taddr = tmem_base + lane_addr + b * BN + half * C::EPI_COLS;
@@ -282,7 +316,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive_relaxed(&acce[b]);  // buffer b read out
                     }
-                    if (c == 3 && g + 1 < G) {  // first step of the next group
+                    if (c == 3 && g + 1 < w.g1) {  // first step of the next group
                         const uint32_t bn = (acc_i + 1) % NB;
                         if (!mbar_wait(&accf[bn], ((acc_i + 1) / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
                         tc_fence_after();
@@ -298,7 +332,29 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
                 ++acc_i;
             }
             if (!ok) break;
-            if (MODE != kModeI32G) {
+            if (MODE != kModeI32G && w.slot >= 0) {
+                // this piece's fp32 sums: four 32 x 16 boxes into its tile-local slot
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float v[16];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        v[2 * j] = __uint_as_float(static_cast<uint32_t>(sum2[8 * c + j]));
+                        v[2 * j + 1] = __uint_as_float(static_cast<uint32_t>(sum2[8 * c + j] >> 32));
+                    }
+                    uint8_t* box = stg + (nstore & 1) * C::STG_BYTES;
+                    if (lane == 0) bulk_wait_read<1>();
+                    __syncwarp();
+                    stage_row16_f32(box, lane, v);
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tmP, box, half * C::EPI_COLS + 16 * c, quarter * 32, w.slot);
+                        bulk_commit();
+                    }
+                    ++nstore;
+                }
+            } else if (MODE != kModeI32G) {
                 const float sxm = mvalid ? __ldg(p.sx + m) : 0.0f;
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
@@ -333,8 +389,9 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+                const GroupUnit w = group_unit(p, u, G, gpk);
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
                     const uint8_t* src = sBP + stage * C::BP_BYTES;  // [BN][64] packed, row-major
                     uint8_t* dst = sB + stage * C::B_BYTES;          // [BN][128] int8, 128B swizzle
@@ -366,10 +423,63 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
     }
 }
 
+// The end of a split tail tile: y[m,n] = fp16/bf16(scale_x[m] * (sum over
+// its pieces, ascending, of the piece's fp32 partial sum)).  kReduceSlices
+// CTAs per tail tile, each 8 rows x 128 columns; a thread owns 8 outputs and
+// issues the loads of four pieces before adding them.
+constexpr int kReduceSlices = 16;
+template <typename TY>
+__global__ void __launch_bounds__(128) k_splitk_reduce(const float* __restrict__ part, GemmArgs p, TY* __restrict__ y) {
+    pdl_wait();  // the partial sums of the GEMM before it are complete
+    pdl_trigger();
+    constexpr int T = 128;  // tile edge
+    const int ti = blockIdx.x / kReduceSlices;  // tail tile index
+    const int r = (blockIdx.x % kReduceSlices) * (T / kReduceSlices) + threadIdx.x / (T / 8);
+    const int c = (threadIdx.x % (T / 8)) * 8;
+    int mb, nb;
+    tile_coords(p.full_tiles + ti, p.num_m_blocks, p.num_n_blocks, mb, nb);
+    const int m = mb * T + r, n = nb * T + c;
+    if (m >= p.M || n >= p.N) return;
+    const float* src = part + (static_cast<int64_t>(ti) * p.splits * T + r) * T + c;  // piece 0
+    const int64_t piece = static_cast<int64_t>(T) * T;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int s = 0;
+    for (; s + 4 <= p.splits; s += 4) {
+        float4 x[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            x[2 * j] = __ldg(reinterpret_cast<const float4*>(src + (s + j) * piece));
+            x[2 * j + 1] = __ldg(reinterpret_cast<const float4*>(src + (s + j) * piece) + 1);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[0] += x[2 * j].x; v[1] += x[2 * j].y; v[2] += x[2 * j].z; v[3] += x[2 * j].w;
+            v[4] += x[2 * j + 1].x; v[5] += x[2 * j + 1].y; v[6] += x[2 * j + 1].z; v[7] += x[2 * j + 1].w;
+        }
+    }
+    for (; s < p.splits; ++s) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(src + s * piece));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(src + s * piece) + 1);
+        v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+        v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
+    const float sxm = __ldg(p.sx + m);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] *= sxm;
+    *reinterpret_cast<uint4*>(y + static_cast<int64_t>(m) * p.N + n) = pack8_out<TY>(v);
+}
+
 template <int MODE, typename TY>
 static cudaError_t launch_grouped_t(const GemmLaunch& L, cudaStream_t st) {
     using C = GroupedCfg<MODE>;
-    CUtensorMap tmA, tmB, tmY;
+    CUtensorMap tmA, tmB, tmY, tmP;
+    const int tiles = ((L.M + C::BM - 1) / C::BM) * ((L.N + C::BN - 1) / C::BN);
+    int splits = L.splits > 1 ? L.splits : 1;
+    int full = splits > 1 ? std::min(std::max(L.full_tiles, 0), tiles) : tiles;
+    if (MODE != kModeI32G && L.part == nullptr) {  // nowhere to put partial sums
+        splits = 1;
+        full = tiles;
+    }
     if (!make_map_2d(&tmA, L.q, L.K, L.M, kBK, C::BM, true)) return cudaErrorInvalidValue;
     if (C::W4) {
         if (!make_map_2d(&tmB, L.w, L.K / 2, L.N, kBK / 2, C::BN, false)) return cudaErrorInvalidValue;
@@ -381,6 +491,11 @@ static cudaError_t launch_grouped_t(const GemmLaunch& L, cudaStream_t st) {
     } else {
         tmY = tmA;  // unused by the INT32 test epilogue
     }
+    if (MODE != kModeI32G && splits > 1) {
+        if (!make_map_part(&tmP, L.part, C::BM, C::BN, (tiles - full) * splits)) return cudaErrorInvalidValue;
+    } else {
+        tmP = tmA;  // unused without split partial sums
+    }
     GemmArgs a;
     a.M = L.M;
     a.N = L.N;
@@ -389,16 +504,24 @@ static cudaError_t launch_grouped_t(const GemmLaunch& L, cudaStream_t st) {
     a.num_m_blocks = (L.M + C::BM - 1) / C::BM;
     a.num_n_blocks = (L.N + C::BN - 1) / C::BN;
     a.num_k_blocks = (L.K + kBK - 1) / kBK;
+    // every piece gets at least one k-block: the piece count is recomputed
+    // from the k-blocks per piece (never above the count the slots were sized for)
+    a.kb_per_split = (a.num_k_blocks + splits - 1) / splits;
+    a.splits = (a.num_k_blocks + a.kb_per_split - 1) / a.kb_per_split;
+    a.full_tiles = a.splits > 1 ? full : tiles;
     a.sx = L.sx;
     a.sw = L.sw;
     a.y = L.y;
     a.status = L.status;
-    const int tiles = a.num_m_blocks * a.num_n_blocks;
-    const int grid = tiles < L.num_sms ? tiles : L.num_sms;
+    const int units = a.full_tiles + (tiles - a.full_tiles) * a.splits;
+    const int grid = units < L.num_sms ? units : L.num_sms;
     auto kern = k_gemm_grouped<MODE, TY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, grid, C::THREADS, C::SMEM_BYTES, st, tmA, tmB, tmY, a);
+    e = launch_pdl(kern, grid, C::THREADS, C::SMEM_BYTES, st, tmA, tmB, tmY, tmP, a);
+    if (e != cudaSuccess || MODE == kModeI32G || a.splits == 1 || a.full_tiles == tiles) return e;
+    return launch_pdl(k_splitk_reduce<TY>, (tiles - a.full_tiles) * kReduceSlices, 128, 0, st,
+                      static_cast<const float*>(L.part), a, static_cast<TY*>(L.y));
 }
 
 cudaError_t launch_gemm_grouped(const GemmLaunch& L, cudaStream_t st) {

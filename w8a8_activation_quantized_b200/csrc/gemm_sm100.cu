@@ -478,6 +478,9 @@ static cudaError_t launch_gemm_cfg(const GemmLaunch& L, cudaStream_t st) {
     a.sw = L.sw;
     a.y = L.y;
     a.status = L.status;
+    a.full_tiles = a.num_m_blocks * a.num_n_blocks;
+    a.splits = 1;
+    a.kb_per_split = a.num_k_blocks;
     const int tiles = a.num_m_blocks * a.num_n_blocks;
     const int grid = tiles < L.num_sms ? tiles : L.num_sms;
     auto kern = k_gemm_sm100<Cfg, TY>;
@@ -508,6 +511,9 @@ static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
     a.sw = L.sw;
     a.y = L.y;
     a.status = L.status;
+    a.full_tiles = a.num_m_blocks * a.num_n_blocks;
+    a.splits = 1;
+    a.kb_per_split = a.num_k_blocks;
     const int tiles = a.num_m_blocks * a.num_n_blocks;
     const int clusters = tiles < L.num_sms / 2 ? tiles : L.num_sms / 2;
     auto kern = k_gemm_pair<MODE, TY>;
