@@ -376,26 +376,63 @@ __device__ __forceinline__ int quant_code(float x, float scale) {
     return static_cast<int>(r);
 }
 
+// Packed fp32 arithmetic: two IEEE operations (round to nearest) per instruction.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // Eight codes at once, bit-identical to quant_code but mostly without a
 // division.  With r = 1/scale correctly rounded (__frcp_rn) and |x/scale| <= 127
 // (+ one ulp), the product t = x * r lies within 2^-15 of the correctly rounded
 // quotient fl(x/scale): each of the two roundings adds at most 2^-24 relative
 // error on a value below 128.  Whenever t is more than 2^-14 away from the
 // nearest halfway point k + 1/2, both t and fl(x/scale) round to the same
-// integer, so rint(t) is the code; within that margin (or if r is not finite)
-// the code is recomputed exactly with quant_code.  rint is taken by adding
-// 1.5 * 2^23: the sum has spacing 1, so it rounds t to an integer, and its low
-// byte is that integer's two's-complement byte.  Returns the eight code bytes.
+// integer, so rint(t) is the code.  rint is taken by adding 1.5 * 2^23: the sum
+// has spacing 1, so it rounds t to an integer, and its low byte is that
+// integer's two's-complement byte; d = t - (sum - 1.5 * 2^23) is exact and
+// measures the distance to that integer.  The eight values go two per packed
+// instruction and are checked together: if any of them is within the margin
+// of a halfway point (or r is not finite, which makes d NaN), all eight are
+// recomputed exactly with quant_code -- one rarely taken branch per eight
+// codes.  Returns the eight code bytes.
 __device__ __forceinline__ uint2 quant8_codes(const float (&f)[8], float scale, float rcp) {
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    constexpr float kMargin = 0.5f - 0x1p-14f;
+    const uint64_t r2 = pack_f32x2(rcp, rcp);
+    const uint64_t m2 = pack_f32x2(kMagic, kMagic), nm2 = pack_f32x2(-kMagic, -kMagic);
+    const uint64_t neg1 = pack_f32x2(-1.0f, -1.0f);
     uint32_t b[8];
+    bool near_tie = false;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float t = f[i] * rcp;
-        float v = t + kMagic;
-        const float d = t - (v - kMagic);
-        if (!(fabsf(d) < 0.5f - 0x1p-14f)) v = static_cast<float>(quant_code(f[i], scale)) + kMagic;
-        b[i] = __float_as_uint(v);
+    for (int i = 0; i < 4; ++i) {
+        const uint64_t t2 = f32x2_mul(pack_f32x2(f[2 * i], f[2 * i + 1]), r2);
+        const uint64_t v2 = f32x2_add(t2, m2);
+        const uint64_t d2 = f32x2_fma(f32x2_add(v2, nm2), neg1, t2);  // t - (v - 1.5 * 2^23)
+        near_tie |= !(fabsf(lo_f32(d2)) < kMargin);
+        near_tie |= !(fabsf(hi_f32(d2)) < kMargin);
+        b[2 * i] = static_cast<uint32_t>(v2);
+        b[2 * i + 1] = static_cast<uint32_t>(v2 >> 32);
+    }
+    if (near_tie) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) b[i] = __float_as_uint(static_cast<float>(quant_code(f[i], scale)) + kMagic);
     }
     uint2 o;
     o.x = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);

@@ -10,11 +10,10 @@
 // section "底层 API" (quantize_weight_int8, pack_weight_int4) and table "量化".
 //
 // Layout: a token row is read with 16-byte vector loads (8 fp16/bf16 values),
-// lane-strided so that each warp load covers 512 contiguous bytes; codes are
-// written as 8-byte vectors.  Rows up to 4096 wide are handled by one warp
-// (the row stays in registers between the max and the quantize pass); wider
-// rows by one 256-thread CTA, which keeps up to 16384 values in registers
-// and re-reads beyond that.
+// thread-strided so that each warp load covers 512 contiguous bytes; codes are
+// written as 8-byte vectors.  Rows up to 12288 wide are spread over 32 to 256
+// threads and stay in registers between the max and the quantize pass; wider
+// rows go to one 256-thread CTA that re-reads the row.
 #include "cider_device.cuh"
 #include "cider_kernels.h"
 
@@ -31,38 +30,53 @@ __device__ __forceinline__ void quant_store8(const float (&f)[8], float scale, f
     *reinterpret_cast<uint2*>(dst) = quant8_codes(f, scale, rcp);
 }
 
-// ---- one warp per token row, row kept in registers (K <= 256 * NV) -------
-// 128-thread CTAs (4 rows each) and NV sized to K keep registers low, so many
-// warps per SM have loads in flight while others quantize.
+// ---- tpr threads per token row, row kept in registers -------------------
+// A 256-thread CTA holds 256 / tpr rows (tpr = 32, 64, 128 or 256); thread j
+// of a row loads the row's 16-byte chunks j, j + tpr, ... (at most NV of
+// them), so each warp load still covers 512 contiguous bytes.  The row max
+// is a warp shuffle reduction, then (tpr > 32) a shared-memory max over the
+// row's warps.  The per-thread chain (loads, max, codes, stores) is short:
+// the launcher picks tpr so that NV <= 6 and, for few rows, so that the grid
+// still fills the GPU -- one row per warp with long chains was bound by the
+// latency of that chain, not by memory.
 template <typename T, int NV>
-__global__ void __launch_bounds__(128, (NV <= 10 ? 6 : 4)) k_quantize_warp(const T* __restrict__ x, int64_t M, int K,
-                                                       int8_t* __restrict__ q,
-                                                       float* __restrict__ sx) {
+__global__ void __launch_bounds__(256) k_quantize_rows(const T* __restrict__ x, int64_t M, int K, int tpr,
+                                                       int8_t* __restrict__ q, float* __restrict__ sx) {
+    __shared__ float red[8];
     pdl_wait();
     pdl_trigger();
-    const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (row >= M) return;
-    const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
+    const int tid = threadIdx.x;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * (256 / tpr) + tid / tpr;
+    const int j = tid % tpr;
+    const bool live = row < M;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (live ? row : 0) * K);
     const int nch = K >> 3;
     uint4 v[NV];
-    // all loads of the row in flight before any of them is used
+    // all loads of the thread in flight before any of them is used
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-        const int c = lane + 32 * i;
-        v[i] = c < nch ? __ldcs(xr + c) : make_uint4(0, 0, 0, 0);
+        const int c = j + tpr * i;
+        v[i] = (live && c < nch) ? __ldcs(xr + c) : make_uint4(0, 0, 0, 0);
     }
     typename Pack2<T>::type m2 = {};
 #pragma unroll
     for (int i = 0; i < NV; ++i) m2 = absmax8<T>(v[i], m2);
-    const float amax = warp_max(absmax_to_f32<T>(m2));
+    float amax = warp_max(absmax_to_f32<T>(m2));
+    if (tpr > 32) {  // uniform across the CTA
+        if ((tid & 31) == 0) red[tid >> 5] = amax;
+        __syncthreads();
+        const int w0 = (tid / tpr) * (tpr >> 5);
+        amax = red[w0];
+        for (int w = 1; w < (tpr >> 5); ++w) amax = fmaxf(amax, red[w0 + w]);
+    }
+    if (!live) return;
     const float s = act_scale(amax);
     const float rs = act_rcp(s);
-    if (lane == 0) sx[row] = s;
+    if (j == 0) sx[row] = s;
     int8_t* qr = q + row * K;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-        const int c = lane + 32 * i;
+        const int c = j + tpr * i;
         if (c < nch) {
             float f[8];
             unpack8_f32<T>(v[i], f);
@@ -71,7 +85,7 @@ __global__ void __launch_bounds__(128, (NV <= 10 ? 6 : 4)) k_quantize_warp(const
     }
 }
 
-// ---- one CTA (256 threads) per token row ---------------------------------
+// ---- one CTA (256 threads) per token row, any width -------------------------
 // NV > 0: up to NV 16-byte chunks per thread stay in registers; NV == 0:
 // any width, the quantize pass re-reads the row (L1/L2 hits).
 template <typename T, int NV>
@@ -140,26 +154,25 @@ static cudaError_t launch_quantize_t(const void* x, int64_t M, int K, int8_t* q,
                                      cudaStream_t st) {
     const T* xt = static_cast<const T*>(x);
     if (M == 0) return cudaSuccess;
-    cudaError_t e = cudaSuccess;
-    if (K <= 4096) {
-        const unsigned grid = static_cast<unsigned>((M + 3) / 4);
-        const int nv = (K + 255) / 256;
-        if (nv <= 1) e = launch_pdl(k_quantize_warp<T, 1>, grid, 128, 0, st, xt, M, K, q, sx);
-        else if (nv <= 2) e = launch_pdl(k_quantize_warp<T, 2>, grid, 128, 0, st, xt, M, K, q, sx);
-        else if (nv <= 4) e = launch_pdl(k_quantize_warp<T, 4>, grid, 128, 0, st, xt, M, K, q, sx);
-        else if (nv <= 6) e = launch_pdl(k_quantize_warp<T, 6>, grid, 128, 0, st, xt, M, K, q, sx);
-        else if (nv <= 8) e = launch_pdl(k_quantize_warp<T, 8>, grid, 128, 0, st, xt, M, K, q, sx);
-        else if (nv <= 10) e = launch_pdl(k_quantize_warp<T, 10>, grid, 128, 0, st, xt, M, K, q, sx);
-        else if (nv <= 12) e = launch_pdl(k_quantize_warp<T, 12>, grid, 128, 0, st, xt, M, K, q, sx);
-        else e = launch_pdl(k_quantize_warp<T, 16>, grid, 128, 0, st, xt, M, K, q, sx);
-    } else {
-        const unsigned grid = static_cast<unsigned>(M);
-        const int nv = (K / 8 + 255) / 256;
-        if (nv <= 4) e = launch_pdl(k_quantize_cta<T, 4>, grid, 256, 0, st, xt, K, q, sx);
-        else if (nv <= 8) e = launch_pdl(k_quantize_cta<T, 8>, grid, 256, 0, st, xt, K, q, sx);
-        else e = launch_pdl(k_quantize_cta<T, 0>, grid, 256, 0, st, xt, K, q, sx);
+    const int nch = K / 8;
+    if (nch > 6 * 256) {  // wider than 12288: one CTA per row, re-reading the row
+        return launch_pdl(k_quantize_cta<T, 0>, static_cast<unsigned>(M), 256, 0, st, xt, K, q, sx);
     }
-    return e;
+    // threads per row: the fewest with <= 6 chunks each, then more while the
+    // grid would hold fewer than ~4 warps per SM sub-partition
+    int tpr = 32;
+    while (tpr < 256 && (nch + tpr - 1) / tpr > 6) tpr *= 2;
+    while (tpr < 256 && M * tpr < 148LL * 512 && nch >= 2 * tpr) tpr *= 2;
+    const int nv = (nch + tpr - 1) / tpr;
+    const unsigned grid = static_cast<unsigned>((M * tpr + 255) / 256);
+    switch (nv) {
+        case 1: return launch_pdl(k_quantize_rows<T, 1>, grid, 256, 0, st, xt, M, K, tpr, q, sx);
+        case 2: return launch_pdl(k_quantize_rows<T, 2>, grid, 256, 0, st, xt, M, K, tpr, q, sx);
+        case 3: return launch_pdl(k_quantize_rows<T, 3>, grid, 256, 0, st, xt, M, K, tpr, q, sx);
+        case 4: return launch_pdl(k_quantize_rows<T, 4>, grid, 256, 0, st, xt, M, K, tpr, q, sx);
+        case 5: return launch_pdl(k_quantize_rows<T, 5>, grid, 256, 0, st, xt, M, K, tpr, q, sx);
+        default: return launch_pdl(k_quantize_rows<T, 6>, grid, 256, 0, st, xt, M, K, tpr, q, sx);
+    }
 }
 
 cudaError_t launch_quantize_act(const void* x, int xdt, int64_t M, int K, int8_t* q, float* sx,
