@@ -291,7 +291,7 @@ def run_cider(args):
     sets = [(x0, w0, sw0)] + [(x0.roll(i, 0).contiguous(), w0.roll(i, 0).contiguous(), sw0.roll(i, 0).contiguous())
                               for i in range(1, n_sets)]
     ys = [torch.empty((M, N), dtype=torch.float16, device=device) for _ in range(n_sets)]
-    wsb = cider.cider_workspace_bytes(M, K)
+    wsb = cider.cider_workspace_bytes_mnk(M, N, K)
     wss = [torch.empty((wsb,), dtype=torch.uint8, device=device) for _ in range(n_sets)]
 
     def step(i):
@@ -407,7 +407,7 @@ def bench_rows(device, pk, steps, warmup):
         n = rotating(N * K + M * K * 3 + M * N * 2)
         ws_ = [w8] + [w8.roll(i, 0).contiguous() for i in range(1, n)]
         ys = [torch.empty((M, N), dtype=torch.float16, device=device) for _ in range(n)]
-        wsp = torch.empty((max(1, cider.cider_workspace_bytes(M, K)),), dtype=torch.uint8, device=device)
+        wsp = torch.empty((max(1, cider.cider_workspace_bytes_mnk(M, N, K)),), dtype=torch.uint8, device=device)
         ms = graph_time(lambda i: cider.cider_w8a8_linear_pc(x, ws_[i % n], s8, y=ys[i % n], workspace=wsp),
                         steps, warmup)
         record("w8a8_linear_pc", ms, 2.0 * M * N * K, N * K + N * 4 + M * K * 2 + M * N * 2, M=M, N=N, K=K,

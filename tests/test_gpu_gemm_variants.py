@@ -73,3 +73,51 @@ def test_pair_is_chosen_for_large_m():
     assert torch.equal(y_pair, y_single) and torch.equal(y_auto, y_pair)
     rows = np.arange(0, M, 97)
     check_y(y_auto, oracle.linear_pc(x[rows], qw, sw), oracle.F16, rows=rows)
+
+
+# ---------------------------------------------------------------- split K of the pair kernel
+
+@pytest.mark.parametrize("splits", [2, 3, 5])
+@pytest.mark.parametrize("M,N,K", [(300, 520, 2560), (513, 1032, 1280), (256, 256, 512)])
+def test_linear_pc_pair_split_equals_unsplit(splits, M, N, K):
+    """K pieces of the CTA-pair kernel add INT32 partial sums exactly and then
+    dequantize with the fused epilogue's expression, so the split result equals
+    the unsplit one bit for bit (and the oracle within tolerance)."""
+    cider.cider_set_small_m_threshold(4)
+    x = act(M, K, seed=M + N + K + splits)
+    qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed=N + splits))
+    xd, wd, sd = dev_bits(x, oracle.F16), dev(qw), dev(sw)
+    cider.cider_test_set_gemm_variant(3)
+    try:
+        cider.cider_test_set_split_k(1)
+        y_plain = cider.cider_w8a8_linear_pc(xd, wd, sd)
+        cider.cider_test_set_split_k(splits)
+        y_split = cider.cider_w8a8_linear_pc(xd, wd, sd)
+    finally:
+        cider.cider_test_set_split_k(0)
+        cider.cider_test_set_gemm_variant(0)
+    torch.cuda.synchronize()
+    assert torch.equal(y_split, y_plain)
+    rows = np.arange(0, M, 7)
+    check_y(y_split, oracle.linear_pc(x[rows], qw, sw), oracle.F16, rows=rows)
+
+
+@pytest.mark.parametrize("dt", [oracle.F16, oracle.BF16])
+def test_linear_pc_tail_split_automatic(dt):
+    """M=2048, N=2560, K=10240: 80 pair tiles on 74 SM pairs, so the automatic
+    plan runs 74 whole tiles and cuts the 6 tiles of the last round into K
+    pieces (80 k-blocks, enough to pay for the partial sums); the result
+    equals the unsplit kernel's bit for bit."""
+    M, N, K = 2048, 2560, 10240
+    x = act(M, K, seed=31, dt=dt)
+    qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed=32))
+    xd, wd, sd = dev_bits(x, dt), dev(qw), dev(sw)
+    big = torch.empty((cider.cider_workspace_bytes_mnk(M, N, K),), dtype=torch.uint8, device="cuda")
+    assert big.numel() > cider.cider_workspace_bytes(M, K)
+    y_auto = cider.cider_w8a8_linear_pc(xd, wd, sd, workspace=big)
+    small = torch.empty((cider.cider_workspace_bytes(M, K),), dtype=torch.uint8, device="cuda")
+    y_plain = cider.cider_w8a8_linear_pc(xd, wd, sd, workspace=small)
+    torch.cuda.synchronize()
+    assert torch.equal(y_auto, y_plain)
+    rows = np.arange(0, M, 37)
+    check_y(y_auto, oracle.linear_pc(x[rows], qw, sw, xdt=dt, ydt=dt), dt, rows=rows)

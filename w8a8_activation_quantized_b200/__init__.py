@@ -160,7 +160,7 @@ def cider_w8a8_linear_pc(x, w, scale_w, y=None, out_dtype=None, workspace=None, 
     M, K = x.shape
     N = w.shape[0]
     y = _out(y, M, N, out_dtype or x.dtype, x.device)
-    ws, ws_bytes = _workspace(M, K, x.device, workspace)
+    ws, ws_bytes = _workspace(M, K, x.device, workspace, N)
     _check("cider_w8a8_linear_pc", lib().cider_w8a8_linear_pc(
         _ptr(x), _DT[x.dtype], M, K, _ptr(w), _ptr(scale_w), N, _ptr(y), _DT[y.dtype],
         _ptr(ws), ws_bytes, _stream(stream, x.device)))

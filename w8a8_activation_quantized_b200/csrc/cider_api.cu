@@ -132,31 +132,48 @@ std::atomic<int> g_gemm_variant{kGemmAuto};  // test override
 std::atomic<int> g_split_override{0};         // test override of the split-K piece count (0 = automatic)
 constexpr int kMaxSplits = 16;
 
-// Split-K plan of the per-group GEMM (128 x 128 tiles on a persistent grid of
-// one CTA per SM): the tiles that fill whole rounds run over all of K; the
-// R tiles of the last, partial round are cut into S K pieces so that their
-// R * S units fill that round (S <= SMs / R, >= 4 k-blocks per piece, <= 16).
-// A forced piece count (test override) splits every tile.
+int pick_variant(int64_t M, int64_t N, int num_sms);
+
+// Split-K plan of a persistent GEMM with `slots` resident tiles (SMs, or SM
+// pairs): the tiles that fill whole rounds run over all of K; the R tiles of
+// the last, partial round are cut into S K pieces so that their R * S units
+// fill that round (S <= slots / R, >= 4 k-blocks per piece, <= 16), provided
+// the cut saves at least min_saved k-blocks on the critical path (the partial
+// sums and the reduce kernel cost a few microseconds).  A forced piece count
+// (test override) splits every tile.  Partial sums take one tile-sized slot
+// of 32-bit values per piece.
 struct SplitPlan {
     int full_tiles, splits;
-    int64_t tail_tiles;
+    int64_t tail_tiles, tile_elems;
 };
-SplitPlan grouped_split_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
-    const int64_t tiles = ((M + 127) / 128) * ((N + 127) / 128);
+SplitPlan split_plan(int64_t tiles, int64_t tile_elems, int slots, int64_t K, int64_t min_saved) {
     const int forced = g_split_override.load();
-    if (forced > 1) return {0, forced, tiles};
-    if (forced == 1 || num_sms <= 0) return {static_cast<int>(tiles), 1, 0};
-    const int64_t full = tiles / num_sms * num_sms, tail = tiles - full;
-    if (tail == 0) return {static_cast<int>(tiles), 1, 0};
-    int64_t s = std::min<int64_t>(num_sms / tail, ((K + 127) / 128) / 4);
+    if (forced > 1) return {0, forced, tiles, tile_elems};
+    if (forced == 1 || slots <= 0) return {static_cast<int>(tiles), 1, 0, tile_elems};
+    const int64_t full = tiles / slots * slots, tail = tiles - full;
+    if (tail == 0) return {static_cast<int>(tiles), 1, 0, tile_elems};
+    const int64_t nkb = (K + 127) / 128;
+    int64_t s = std::min<int64_t>(slots / tail, nkb / 4);
     s = std::min<int64_t>(s, kMaxSplits);
-    if (s < 2) return {static_cast<int>(tiles), 1, 0};
-    return {static_cast<int>(full), static_cast<int>(s), tail};
+    if (s < 2 || nkb - (nkb + s - 1) / s < min_saved) return {static_cast<int>(tiles), 1, 0, tile_elems};
+    return {static_cast<int>(full), static_cast<int>(s), tail, tile_elems};
+}
+// Per-group GEMM: 128 x 128 tiles, one CTA per SM; a k-block costs ~0.5-1 us
+// of epilogue time, so any cut of >= 4 k-blocks pays.
+SplitPlan grouped_split_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
+    return split_plan(((M + 127) / 128) * ((N + 127) / 128), 128 * 128, num_sms, K, 4);
+}
+// Per-channel GEMM: only on the CTA-pair 256 x 256 tile, whose k-block takes
+// ~0.27 us; measured at K = 2560 (M = 1024 and 8192) the split does not pay,
+// so it needs >= 32 saved k-blocks (K of roughly 5120 and more).
+SplitPlan pc_split_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
+    if (pick_variant(M, N, num_sms) != kGemmPair) return {0, 1, 0, 0};
+    return split_plan(((M + 255) / 256) * ((N + 255) / 256), 256 * 256, num_sms / 2, K, 32);
 }
 
-// Bytes of fp32 partial sums: one 128 x 128 slot per K piece of a tail tile.
+// Bytes of 32-bit partial sums: one tile-sized slot per K piece of a tail tile.
 size_t part_bytes(const SplitPlan& sp) {
-    return sp.splits > 1 ? align256(static_cast<size_t>(sp.tail_tiles) * sp.splits * 128 * 128 * 4) : 0;
+    return sp.splits > 1 ? align256(static_cast<size_t>(sp.tail_tiles) * sp.splits * sp.tile_elems * 4) : 0;
 }
 
 // Per-channel GEMM variant: the CTA-pair 256x256 tile when it still gives
@@ -172,7 +189,7 @@ int pick_variant(int64_t M, int64_t N, int num_sms) {
 
 cider_status_t run_gemm(int mode, const int8_t* q, const float* sx, int64_t M, int64_t K,
                         const void* w, const float* sw, int64_t N, int64_t gs, void* y, int ydt,
-                        const DeviceInfo* d, cudaStream_t st, SplitPlan sp = {0, 1, 0}, float* part = nullptr) {
+                        const DeviceInfo* d, cudaStream_t st, SplitPlan sp = {0, 1, 0, 0}, float* part = nullptr) {
     GemmLaunch L;
     L.mode = mode;
     L.q = q;
@@ -227,11 +244,12 @@ cider_status_t linear(int mode, const void* x, int xdt, int64_t M, int64_t K, co
         return fail(CIDER_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, ws ? ws_bytes : 0);
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(CIDER_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     // split-K partial sums of the per-group GEMM, when the workspace holds them
-    SplitPlan plan{0, 1, 0};
+    SplitPlan plan{0, 1, 0, 0};
     float* part = nullptr;
     size_t used = need;
-    if (mode != kModePC) {
-        const SplitPlan sp = grouped_split_plan(M, N, K, d->num_sms);
+    {
+        const SplitPlan sp = mode == kModePC ? pc_split_plan(M, N, K, d->num_sms)
+                                             : grouped_split_plan(M, N, K, d->num_sms);
         const size_t pb = part_bytes(sp);
         if (sp.splits > 1 && ws_bytes >= need + pb) {
             plan = sp;
@@ -353,7 +371,8 @@ size_t cider_workspace_bytes_mnk(int64_t M, int64_t N, int64_t K) {
     if (need == 0 || N <= 0) return need;
     DeviceInfo* d = nullptr;
     if (device_info(&d) != CIDER_OK) return need;
-    return need + part_bytes(grouped_split_plan(M, N, K, d->num_sms));
+    return need + std::max(part_bytes(grouped_split_plan(M, N, K, d->num_sms)),
+                           part_bytes(pc_split_plan(M, N, K, d->num_sms)));
 }
 
 cider_status_t cider_test_set_split_k(int splits) {
@@ -507,7 +526,7 @@ cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8_t* w, int
     DeviceInfo* d = nullptr;
     if ((s = device_info(&d)) != CIDER_OK) return s;
     const int forced = g_split_override.load();
-    const SplitPlan sp{0, forced > 1 ? forced : 1, 0};
+    const SplitPlan sp{0, forced > 1 ? forced : 1, 0, 0};
     return run_gemm(kModeI32G, q, nullptr, M, K, w, nullptr, N, gs, acc_g, 0, d, static_cast<cudaStream_t>(stream),
                     sp, nullptr);
 }

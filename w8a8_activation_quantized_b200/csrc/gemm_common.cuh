@@ -39,6 +39,33 @@ __device__ __forceinline__ void tile_coords(int t, int nm, int nn, int& mb, int&
     nb = r / gm;
 }
 
+// Work unit u of a GEMM with a split tail: a whole tile (u < full_tiles) or
+// one K piece of a tail tile.  Tile coordinates, k-blocks [kb0, kb1) and, for
+// a piece, the slot of its partial sums (-1 for a whole tile).
+struct TileUnit {
+    int mb, nb, kb0, kb1, slot;
+};
+__device__ __forceinline__ TileUnit tile_unit(const GemmArgs& p, int u) {
+    TileUnit w;
+    int t, piece;
+    if (u < p.full_tiles) {
+        t = u;
+        piece = -1;
+    } else {
+        const int v = u - p.full_tiles;
+        t = p.full_tiles + v / p.splits;
+        piece = v % p.splits;
+    }
+    tile_coords(t, p.num_m_blocks, p.num_n_blocks, w.mb, w.nb);
+    w.slot = piece < 0 ? -1 : (t - p.full_tiles) * p.splits + piece;
+    w.kb0 = piece < 0 ? 0 : piece * p.kb_per_split;
+    w.kb1 = piece < 0 ? p.num_k_blocks : min(w.kb0 + p.kb_per_split, p.num_k_blocks);
+    return w;
+}
+__device__ __forceinline__ int num_units(const GemmArgs& p) {
+    return p.full_tiles + (p.num_m_blocks * p.num_n_blocks - p.full_tiles) * p.splits;
+}
+
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

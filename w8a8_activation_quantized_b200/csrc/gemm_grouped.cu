@@ -76,30 +76,13 @@ struct GroupedCfg {
     static_assert(SMEM_BYTES <= kSmemMax, "shared memory");
 };
 
-// Work unit u: a whole tile (u < full_tiles) or one K piece of a tail tile;
-// its tile coordinates, k-blocks [kb0, kb1), groups [g0, g1) and, for a
-// piece, the slot of its partial sums (-1 for a whole tile).
+// A work unit (tile_unit) plus its groups [g0, g1).
 struct GroupUnit {
     int mb, nb, kb0, kb1, g0, g1, slot;
 };
 __device__ __forceinline__ GroupUnit group_unit(const GemmArgs& p, int u, int G, int gpk) {
-    GroupUnit w;
-    int t, piece;
-    if (u < p.full_tiles) {
-        t = u;
-        piece = -1;
-    } else {
-        const int v = u - p.full_tiles;
-        t = p.full_tiles + v / p.splits;
-        piece = v % p.splits;
-    }
-    tile_coords(t, p.num_m_blocks, p.num_n_blocks, w.mb, w.nb);
-    w.slot = piece < 0 ? -1 : (t - p.full_tiles) * p.splits + piece;
-    w.kb0 = piece < 0 ? 0 : piece * p.kb_per_split;
-    w.kb1 = piece < 0 ? p.num_k_blocks : min(w.kb0 + p.kb_per_split, p.num_k_blocks);
-    w.g0 = w.kb0 * gpk;
-    w.g1 = min(w.kb1 * gpk, G);
-    return w;
+    const TileUnit t = tile_unit(p, u);
+    return GroupUnit{t.mb, t.nb, t.kb0, t.kb1, t.kb0 * gpk, min(t.kb1 * gpk, G), t.slot};
 }
 
 // 10 or 12 warps: three of them share a 16K-register SM sub-partition, so
@@ -131,7 +114,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int num_units = p.full_tiles + (p.num_m_blocks * p.num_n_blocks - p.full_tiles) * p.splits;
+    const int nunits = num_units(p);
     const int G = p.K / p.gs;
     const int gpk = kBK / p.gs;  // groups per k-block: 1 or 2
 
@@ -179,7 +162,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
             uint32_t phase = 0;
             const uint32_t tx = C::A_BYTES + (C::W4 ? C::BP_BYTES : C::B_BYTES);
             bool ok = true;
-            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
                 const GroupUnit w = group_unit(p, u, G, gpk);
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) { ok = false; break; }
@@ -206,7 +189,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
             uint32_t acc_i = 0;  // partial-buffer uses so far
             bool ok = true;
             const int steps = p.gs / kUmmaK;
-            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
                 const GroupUnit w = group_unit(p, u, G, gpk);
                 int g = w.g0;
                 for (int kb = w.kb0; kb < w.kb1 && ok; ++kb) {
@@ -251,7 +234,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
         // CTA's (unit, group) sequence; a running pointer avoids divisions.
         int pf_u = blockIdx.x, pf_g = 0, pf_g1 = 0, pf_slot = 0, pf_col = 0;
         auto pf_unit = [&]() {
-            if (pf_u < num_units) {
+            if (pf_u < nunits) {
                 const GroupUnit w = group_unit(p, pf_u, G, gpk);
                 pf_g = w.g0;
                 pf_g1 = w.g1;
@@ -260,7 +243,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
         };
         pf_unit();
         auto prefetch = [&]() {
-            if (MODE != kModeI32G && pf_u < num_units && lane < C::EPI_COLS / 4) {
+            if (MODE != kModeI32G && pf_u < nunits && lane < C::EPI_COLS / 4) {
                 const bool in = pf_col < p.N;
                 const float* src = p.sw + static_cast<int64_t>(pf_g) * p.N + (in ? pf_col : 0);
                 cp_async16(scl + pf_slot * C::SCL_BYTES + 16 * lane, src, in ? 16u : 0u);
@@ -277,7 +260,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
         const uint64_t neg_bias2 = pack_u32x2(__float_as_uint(-12582912.0f), __float_as_uint(-12582912.0f));
         uint32_t acc_i = 0, nstore = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
             const GroupUnit w = group_unit(p, u, G, gpk);
             const int m0 = w.mb * C::BM + quarter * 32;
             const int m = m0 + lane;
@@ -389,7 +372,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
                 const GroupUnit w = group_unit(p, u, G, gpk);
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }

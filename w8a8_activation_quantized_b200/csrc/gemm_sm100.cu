@@ -23,6 +23,8 @@
 // The pages' own tiles (BM128 BN128 BK512 on Apple TensorOps) are prior art;
 // the sizes here follow from TMEM (512 columns x 128 lanes x 32 bit per SM),
 // the 256x256x32 kind::i8 pair MMA shape and 227 KB of shared memory.
+#include <algorithm>
+
 #include "gemm_common.cuh"
 
 namespace cider {
@@ -287,7 +289,7 @@ __device__ __forceinline__ void load_scales32(const float* sw, int n0, int N, fl
 template <int MODE, typename TY>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmY, GemmArgs p) {
+                const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmP, GemmArgs p) {
     using C = PairCfg;
     constexpr int S = C::STAGES;
     constexpr int NB = C::ACC_BUFS;
@@ -309,7 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     const bool leader = (rank == 0);
     const int cid = static_cast<int>(cluster_id_x());
     const int ncl = static_cast<int>(cluster_count_x());
-    const int num_tiles = p.num_m_blocks * p.num_n_blocks;
+    const int nunits = num_units(p);  // whole tiles, then K pieces of the tail tiles
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -344,15 +346,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int t = cid; t < num_tiles && ok; t += ncl) {
-                int mb, nb;
-                tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+            for (int u = cid; u < nunits && ok; u += ncl) {
+                const TileUnit w = tile_unit(p, u);
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, p.status, abort_flag)) { ok = false; break; }
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
                     const uint32_t bar = map_to_rank(&full[stage], 0);
-                    tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, bar, kb * kBK, mb * C::BM + static_cast<int>(rank) * 128);
-                    tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, bar, kb * kBK, nb * C::BN + static_cast<int>(rank) * (C::BN / 2));
+                    tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, bar, kb * kBK, w.mb * C::BM + static_cast<int>(rank) * 128);
+                    tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, bar, kb * kBK, w.nb * C::BN + static_cast<int>(rank) * (C::BN / 2));
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -365,12 +366,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             uint32_t phase = 0;
             uint32_t acc_i = 0;
             bool ok = true;
-            for (int t = cid; t < num_tiles && ok; t += ncl) {
+            for (int u = cid; u < nunits && ok; u += ncl) {
+                const TileUnit w = tile_unit(p, u);
                 const uint32_t b = acc_i % NB;
                 if (!mbar_wait_cluster(&acce[b], ((acc_i / NB) & 1u) ^ 1u, p.status, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem_base + b * C::BN;
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait_cluster(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
@@ -378,7 +380,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBK / kUmmaK; ++kk)
                         umma_i8_pair(d, adesc + (kk * kUmmaK >> 4), bdesc + (kk * kUmmaK >> 4), idesc,
-                                     (kb > 0 || kk > 0) ? 1u : 0u);
+                                     (kb > w.kb0 || kk > 0) ? 1u : 0u);
                     umma_commit_pair(&empty[stage]);
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
@@ -401,17 +403,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         constexpr int NCH = C::EPI_COLS / 32;
         uint32_t acc_i = 0, nstore = 0;
         bool ok = true;
-        for (int t = cid; t < num_tiles && ok; t += ncl) {
-            int mb, nb;
-            tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
-            const int m0 = mb * C::BM + static_cast<int>(rank) * 128 + quarter * 32;  // first row of this warp
+        for (int u = cid; u < nunits && ok; u += ncl) {
+            const TileUnit w = tile_unit(p, u);
+            const int m0 = w.mb * C::BM + static_cast<int>(rank) * 128 + quarter * 32;  // first row of this warp
             const int m = m0 + lane;
             const bool mvalid = m < p.M;
-            const int nw = nb * C::BN + half * C::EPI_COLS;  // first column of this warp
+            const int nw = w.nb * C::BN + half * C::EPI_COLS;  // first column of this warp
             const uint32_t b = acc_i % NB;
+            const bool piece = w.slot >= 0;  // K piece of a tail tile: INT32 partial sums out
             const float sxm = (MODE == kModePC && mvalid) ? __ldg(p.sx + m) : 0.0f;
             float ws[2][32];
-            if (MODE == kModePC) load_scales32(p.sw, nw, p.N, ws[0]);
+            if (MODE == kModePC && !piece) load_scales32(p.sw, nw, p.N, ws[0]);
             if (!mbar_wait_cluster(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
             tc_fence_after();
             uint32_t r[2][32];
@@ -422,7 +424,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                 tmem_ld_wait();
                 if (c + 1 < NCH) {
                     tmem_ld_32x32b_x32(tbase + (c + 1) * 32, r[(c + 1) & 1]);
-                    if (MODE == kModePC) load_scales32(p.sw, nw + (c + 1) * 32, p.N, ws[(c + 1) & 1]);
+                    if (MODE == kModePC && !piece) load_scales32(p.sw, nw + (c + 1) * 32, p.N, ws[(c + 1) & 1]);
                 } else {
                     tc_fence_before();
                     __syncwarp();
@@ -431,6 +433,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                 const int n0 = nw + c * 32;
                 if (MODE == kModeI32) {
                     if (mvalid) store_chunk_pc<MODE, TY>(p, r[c & 1], m, n0, sxm);
+                } else if (piece) {
+                    // this piece's INT32 sums, two 32 x 16 boxes into the tile-local slot
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint8_t* box = stg + (nstore & 1) * C::STG_BYTES;
+                        if (lane == 0) bulk_wait_read<1>();
+                        __syncwarp();
+                        float v[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(r[c & 1][16 * h + e]);
+                        stage_row16_f32(box, lane, v);
+                        fence_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_3d(&tmP, box, half * C::EPI_COLS + c * 32 + 16 * h,
+                                         static_cast<int>(rank) * 128 + quarter * 32, w.slot);
+                            bulk_commit();
+                        }
+                        ++nstore;
+                    }
                 } else {
                     uint8_t* box = stg + (nstore & 1) * C::STG_BYTES;
                     if (lane == 0) bulk_wait_read<1>();  // the store issued two boxes ago has read `box`
@@ -489,9 +511,61 @@ static cudaError_t launch_gemm_cfg(const GemmLaunch& L, cudaStream_t st) {
     return launch_pdl(kern, grid, Cfg::THREADS, Cfg::SMEM_BYTES, st, tmA, tmB, a);
 }
 
+// The end of a split tail tile of the per-channel pair GEMM: the pieces'
+// INT32 sums add exactly, then y = fp16/bf16((acc * scale_x[m]) * scale_w[n])
+// -- the same expression as the fused epilogue, so split and unsplit results
+// are equal bit for bit.  32 CTAs per 256 x 256 tail tile (8 rows each), eight
+// outputs per thread.
+template <typename TY>
+__global__ void __launch_bounds__(256) k_splitk_reduce_pc(const int32_t* __restrict__ part, GemmArgs p,
+                                                          TY* __restrict__ y) {
+    pdl_wait();  // the partial sums of the GEMM before it are complete
+    pdl_trigger();
+    constexpr int T = PairCfg::BM;  // 256 x 256 tiles
+    static_assert(PairCfg::BM == PairCfg::BN, "square pair tiles");
+    const int ti = blockIdx.x / (T / 8);
+    const int r = (blockIdx.x % (T / 8)) * 8 + threadIdx.x / 32;
+    const int c = (threadIdx.x % 32) * 8;
+    int mb, nb;
+    tile_coords(p.full_tiles + ti, p.num_m_blocks, p.num_n_blocks, mb, nb);
+    const int m = mb * T + r, n = nb * T + c;
+    if (m >= p.M || n >= p.N) return;
+    const int32_t* src = part + (static_cast<int64_t>(ti) * p.splits * T + r) * T + c;
+    int acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    constexpr int64_t piece = static_cast<int64_t>(T) * T;
+    int s = 0;
+    for (; s + 4 <= p.splits; s += 4) {  // four pieces' loads in flight, then the adds
+        int4 x[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            x[2 * j] = __ldg(reinterpret_cast<const int4*>(src + (s + j) * piece));
+            x[2 * j + 1] = __ldg(reinterpret_cast<const int4*>(src + (s + j) * piece) + 1);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            acc[0] += x[2 * j].x; acc[1] += x[2 * j].y; acc[2] += x[2 * j].z; acc[3] += x[2 * j].w;
+            acc[4] += x[2 * j + 1].x; acc[5] += x[2 * j + 1].y; acc[6] += x[2 * j + 1].z; acc[7] += x[2 * j + 1].w;
+        }
+    }
+    for (; s < p.splits; ++s) {
+        const int4 a = __ldg(reinterpret_cast<const int4*>(src + s * piece));
+        const int4 b = __ldg(reinterpret_cast<const int4*>(src + s * piece) + 1);
+        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    const float sxm = __ldg(p.sx + m);
+    const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.sw + n));
+    const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.sw + n) + 1);
+    const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = (static_cast<float>(acc[e]) * sxm) * ws[e];
+    store_row8<TY>(y + static_cast<int64_t>(m) * p.N + n, v);
+}
+
 template <int MODE, typename TY>
 static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
-    CUtensorMap tmA, tmB, tmY;
+    CUtensorMap tmA, tmB, tmY, tmP;
     if (!make_map_2d(&tmA, L.q, L.K, L.M, kBK, 128, true)) return cudaErrorInvalidValue;
     if (!make_map_2d(&tmB, L.w, L.K, L.N, kBK, PairCfg::BN / 2, true)) return cudaErrorInvalidValue;
     if (MODE == kModePC) {
@@ -511,15 +585,29 @@ static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
     a.sw = L.sw;
     a.y = L.y;
     a.status = L.status;
-    a.full_tiles = a.num_m_blocks * a.num_n_blocks;
-    a.splits = 1;
-    a.kb_per_split = a.num_k_blocks;
     const int tiles = a.num_m_blocks * a.num_n_blocks;
-    const int clusters = tiles < L.num_sms / 2 ? tiles : L.num_sms / 2;
+    // split K of the tail tiles (per-channel with a partial-sum buffer only)
+    int splits = (MODE == kModePC && L.part != nullptr && L.splits > 1) ? L.splits : 1;
+    const int full = splits > 1 ? std::min(std::max(L.full_tiles, 0), tiles) : tiles;
+    a.kb_per_split = (a.num_k_blocks + splits - 1) / splits;
+    a.splits = (a.num_k_blocks + a.kb_per_split - 1) / a.kb_per_split;
+    a.full_tiles = a.splits > 1 ? full : tiles;
+    if (a.splits > 1 && a.full_tiles < tiles) {
+        if (!make_map_part(&tmP, L.part, PairCfg::BM, PairCfg::BN, (tiles - full) * splits)) return cudaErrorInvalidValue;
+    } else {
+        a.splits = 1;
+        a.full_tiles = tiles;
+        tmP = tmA;  // unused without split partial sums
+    }
+    const int units = a.full_tiles + (tiles - a.full_tiles) * a.splits;
+    const int clusters = units < L.num_sms / 2 ? units : L.num_sms / 2;
     auto kern = k_gemm_pair<MODE, TY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, 2 * clusters, PairCfg::THREADS, PairCfg::SMEM_BYTES, st, tmA, tmB, tmY, a);
+    e = launch_pdl(kern, 2 * clusters, PairCfg::THREADS, PairCfg::SMEM_BYTES, st, tmA, tmB, tmY, tmP, a);
+    if (e != cudaSuccess || a.splits == 1) return e;
+    return launch_pdl(k_splitk_reduce_pc<TY>, (tiles - a.full_tiles) * (PairCfg::BM / 8), 256, 0, st,
+                      reinterpret_cast<const int32_t*>(L.part), a, static_cast<TY*>(L.y));
 }
 
 template <int MODE, typename TY>
