@@ -19,10 +19,12 @@
 // group (64 or 128 values) never straddles warps.  Each warp keeps a ring of
 // three row blocks in registers -- all loads of a slice issued at once, two
 // blocks ahead of the one being used -- and its first two blocks start
-// loading before the activations are quantized.  Per-group: the lanes of one
-// group reduce its INT32 partial with shuffles and one lane rescales it by
-// scale_w[g][n] in fp32.  With one warp per row (S = 1) a warp writes its
-// outputs directly; otherwise the slices combine through shared memory.
+// loading before the activations are quantized.  Per-group: each lane scales
+// its chunk's exact INT32 dot by the chunk's group scale scale_w[g][n] and
+// adds it to an fp32 sum (scale_w[g] * acc_g, summed in another order); the
+// warp's final shuffle reduction adds the lanes.  With one warp per row
+// (S = 1) a warp writes its outputs directly; otherwise the slices combine
+// through shared memory.
 #include "cider_device.cuh"
 #include "cider_kernels.h"
 
@@ -141,7 +143,6 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
     }
     __syncthreads();
 
-    const int lpg = PG ? gs / KC : 32;  // lanes per group: 2, 4 or 8
     auto step = [&](const uint4 (&cur)[PPW], const float (&cs)[PG ? PPW : 1], int blk) {
         const int n = blk * geo.R + r_in_blk;
         int iacc[MAXM];
@@ -160,13 +161,15 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
                     for (int m = 0; m < MAXM; ++m)
                         if (m < M && valid) iacc[m] = chunk_dot<W4>(cur[p], s_q + static_cast<int64_t>(m) * K, k0) + iacc[m];
                 } else {
+                    // Each lane scales its own chunk's exact INT32 dot by the chunk's
+                    // group scale: summed over the group's lanes that is
+                    // scale_w[g] * acc_g, with the fp32 additions in another order.
                     const float s = cs[p];  // this lane's group scale (0 for invalid chunks)
 #pragma unroll
                     for (int m = 0; m < MAXM; ++m) {
                         if (m < M) {
-                            int pp = valid ? chunk_dot<W4>(cur[p], s_q + static_cast<int64_t>(m) * K, k0) : 0;
-                            for (int o = 1; o < lpg; o <<= 1) pp += __shfl_xor_sync(0xffffffffu, pp, o);
-                            if ((lane & (lpg - 1)) == 0) facc[m] = fmaf(static_cast<float>(pp), s, facc[m]);
+                            const int pp = valid ? chunk_dot<W4>(cur[p], s_q + static_cast<int64_t>(m) * K, k0) : 0;
+                            facc[m] = fmaf(static_cast<float>(pp), s, facc[m]);
                         }
                     }
                 }
