@@ -358,7 +358,7 @@ def run_cider(args):
                    "launch": "K steps captured in one CUDA graph, replayed once in the timed region"},
         "tops_per_gpu": value / ws, "pct_int8_peak": 100.0 * (value / ws) / int8_peak,
         "breakdown_ms": {"quantize_act": ms_quant, "gemm_pc": ms_gemm},
-        "roofline": {"bound": "tensor", "kernel": "k_gemm_sm100 per-channel (tcgen05.mma kind::i8)",
+        "roofline": {"bound": "tensor", "kernel": "k_gemm_pair per-channel (tcgen05.mma.cta_group::2 kind::i8)",
                      "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
                      "traffic": gemm_traffic(), "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "algorithmic_bytes": M * K + N * K + M * N * 2 + 4 * (M + N),
