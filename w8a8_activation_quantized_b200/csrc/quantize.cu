@@ -219,8 +219,12 @@ __global__ void __launch_bounds__(256) k_silu_mul_quantize(const T* __restrict__
             for (int j = 0; j < 8; ++j) {
                 // sigmoid(g) = 1/(1+e^-g) for g >= 0 and e^g/(1+e^g) for g < 0:
                 // e^-|g| never overflows, so large negative g keep their tiny value.
+                // The quotient's denominator lies in [1, 2], where __fdividef is
+                // within 2 ulp of fp32: far below the one unit of fp16/bf16 that
+                // a is rounded to (the IEEE division cost more than the rest of
+                // the element's work).
                 const float e = expf(-fabsf(g[j]));
-                const float sig = __fdiv_rn(g[j] >= 0.0f ? 1.0f : e, 1.0f + e);
+                const float sig = __fdividef(g[j] >= 0.0f ? 1.0f : e, 1.0f + e);
                 ah[j] = from_f32<T>((g[j] * sig) * u[j]);
                 amax = fmaxf(amax, fabsf(to_f32<T>(ah[j])));
             }
@@ -257,6 +261,8 @@ static cudaError_t launch_silu_t(const void* g, const void* u, int64_t M, int F,
     T* at = static_cast<T*>(a_out);
     const unsigned grid = static_cast<unsigned>(M);
     if (nv <= 2) return launch_pdl(k_silu_mul_quantize<T, 2>, grid, 256, 0, st, gt, ut, F, q, sx, at);
+    else if (nv <= 4) return launch_pdl(k_silu_mul_quantize<T, 4>, grid, 256, 0, st, gt, ut, F, q, sx, at);
+    else if (nv <= 6) return launch_pdl(k_silu_mul_quantize<T, 6>, grid, 256, 0, st, gt, ut, F, q, sx, at);
     else if (nv <= 8) return launch_pdl(k_silu_mul_quantize<T, 8>, grid, 256, 0, st, gt, ut, F, q, sx, at);
     else if (nv <= 16) return launch_pdl(k_silu_mul_quantize<T, 16>, grid, 256, 0, st, gt, ut, F, q, sx, at);
     return cudaErrorInvalidValue;  // F > 32768: rejected by the host checks first
