@@ -6,8 +6,8 @@ import torch
 import oracle
 
 # fp16 output: |y_gpu - y_oracle| <= 1e-3 * max_n |y_oracle[m, n]| per row (the
-# spec tolerance; one fp16 ulp is at most 2^-10 |y| < 1e-3 |y|, so any
-# single-rounding difference passes).  bf16 keeps 8 significant bits, so one
+# workload's stated tolerance; one fp16 ulp is at most 2^-10 |y| < 1e-3 |y|, so
+# any single-rounding difference passes).  bf16 keeps 8 significant bits, so one
 # bf16 ulp is up to 2^-7 |y|: its tolerance is 2^-7 * row max, derived the same way.
 TOL = {oracle.F16: 1e-3, oracle.BF16: 2.0 ** -7}
 
