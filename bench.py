@@ -440,6 +440,15 @@ def bench_rows(device, pk, steps, warmup):
         record("w8a8_linear_pc", ms, 2.0 * M * N * K, N * K + N * 4 + M * K * 2 + M * N * 2, M=M, N=N, K=K,
                path="small-M fused kernel" if cider.cider_workspace_bytes(M, K) == 0 else "quantize + tcgen05 GEMM")
         del ws_, ys
+    # W8A16 decode product (no activation quantization), M=1, N=10240 K=2560
+    x1 = torch.from_numpy(synth.activations(1, K, 1001)).to(device)
+    n = rotating(N * K)
+    ws_ = [w8] + [w8.roll(i, 0).contiguous() for i in range(1, n)]
+    y1 = torch.empty((1, N), dtype=torch.float16, device=device)
+    ms = graph_time(lambda i: cider.cider_w8a16_mv_pc(x1, ws_[i % n], s8, y=y1), steps, warmup)
+    record("w8a16_mv_pc", ms, 2.0 * N * K, N * K + N * 4 + K * 2 + N * 2, M=1, N=N, K=K,
+           path="W8A16 decode kernel (no activation quantization)")
+    del ws_
     del w8
     # per-group, N=2560 K=10240, gs 128 and 64
     N, K = 2560, 10240
@@ -513,6 +522,7 @@ ROW_CASES = {
     "pc_m1024": ("pc", 1024, 10240, 2560, 0), "pc_m4096": ("pc", 4096, 10240, 2560, 0),
     "pc_m8192": ("pc", 8192, 10240, 2560, 0),
     "pg128_m1": ("pg", 1, 2560, 10240, 128), "pg128_m4096": ("pg", 4096, 2560, 10240, 128),
+    "mv_m1": ("mv", 1, 10240, 2560, 0),
     "pg64_m1": ("pg", 1, 2560, 10240, 64), "pg64_m4096": ("pg", 4096, 2560, 10240, 64),
     "pg128_m128": ("pg", 128, 2560, 10240, 128), "pg64_m128": ("pg", 128, 2560, 10240, 64),
     "pg64_m1024": ("pg", 1024, 2560, 10240, 64), 
@@ -537,6 +547,9 @@ def run_row(args):
     if kind == "pc":
         w, s = cider.cider_quantize_weight_pc(W)
         call = lambda y, ws_: cider.cider_w8a8_linear_pc(x, w, s, y=y, workspace=ws_)
+    elif kind == "mv":
+        w, s = cider.cider_quantize_weight_pc(W)
+        call = lambda y, ws_: cider.cider_w8a16_mv_pc(x, w, s, y=y)
     elif kind == "pg":
         w, s = cider.cider_quantize_weight_pg(W, gs)
         call = lambda y, ws_: cider.cider_w8a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)

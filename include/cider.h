@@ -131,6 +131,19 @@ CIDER_API cider_status_t cider_w8a8_linear_pc(const void* x, cider_dtype_t xdt, 
                                     void* y, cider_dtype_t ydt,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* W8A16 decode matrix-vector product, per-output-channel weight scales: the
+ * pages' decode kernel (Cider README, section "Metal Kernel 流水线", Decode:
+ * a direct INT8 matrix-vector product, weights dequantized on the fly, no
+ * activation quantization).  y[m,n] = round_ydt(scale_w[n] * sum_k x[m,k] *
+ * w[n,k]), x widened to fp32 and the products summed in fp32; the activations
+ * are NOT quantized, unlike cider_w8a8_linear_pc, whose small-M path keeps the
+ * W8A8 semantics.  x: [M][K] (xdt), 1 <= M <= 4 and M * ceil(K / 512) * 2048
+ * <= 160 KiB (the rows are staged in shared memory as fp32), K <= 32768; w: [N][K] int8;
+ * scale_w: [N] fp32; y: [M][N] (ydt).  No workspace. */
+CIDER_API cider_status_t cider_w8a16_mv_pc(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
+                                 const int8_t* w, const float* scale_w, int64_t N,
+                                 void* y, cider_dtype_t ydt, void* stream);
+
 /* W8A8 linear, per-group weight scales along K (gs = 64 or 128; Cider README,
  * table "W8A8 量化粒度"; juejin post, section "三种量化粒度的实现").
  * scale_w: [K/gs][N] fp32 (group-major).  The INT32 partial sum of each group

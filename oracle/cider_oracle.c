@@ -21,7 +21,10 @@
  *           W4A8 weights symmetric INT4 "zp=8"; activations symmetric INT8
  *           per-token; INT32 accumulation; C_fp16 = C_int32 * s_act * s_weight),
  *           table "模式" (W4A8: INT4 packed in uint8, unpack -> TensorOps),
- *           section "底层 API" (quantize_weight_int8, pack_weight_int4).
+ *           section "底层 API" (quantize_weight_int8, pack_weight_int4),
+ *           section "Metal Kernel 流水线" (Decode: INT8 matrix-vector
+ *           product, weights dequantized on the fly, no activation
+ *           quantization).
  *
  * Readings where the pages are silent (each one is listed in the design notes):
  *  - round() is round-half-away-from-zero;
@@ -344,6 +347,26 @@ int oracle_linear_pc(const uint16_t* x, int xdt, int64_t M, int64_t K, const int
         }
     }
     return bad ? -1 : 0;
+}
+
+/* W8A16 decode product, per-channel weight scales ([README] section
+ * "Metal Kernel 流水线", Decode: a direct INT8 matrix-vector product with the
+ * weights dequantized on the fly and no activation quantization):
+ * y[m,n] = round(sw[n] * sum_k x[m,k] * w[n,k]) -- x widened exactly, the
+ * products and their sum in fp64, one rounding to the output type. */
+int oracle_w8a16_linear_pc(const uint16_t* x, int xdt, int64_t M, int64_t K, const int8_t* w,
+                           const float* sw, int64_t N, int ydt, uint16_t* y)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double a = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                a += (double)widen(x, m * K + k, xdt) * (double)w[n * K + k];
+            y[m * N + n] = narrow(a * (double)sw[n], ydt);
+        }
+    }
+    return 0;
 }
 
 /* W8A8, per-group weight scales sw[n][K/gs]. */

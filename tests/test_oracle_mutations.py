@@ -16,6 +16,7 @@ import oracle
 from oracle.build import CFLAGS, SRC
 from tests import test_oracle_golden as golden_tests
 from tests import test_oracle_invariants as inv_tests
+from tests import test_oracle_w8a16 as w8a16_tests
 
 MUTATIONS = {
     "round_half_to_even_codes": ("if (fabsf(d) >= 0.5f)", "if (fabsf(d) > 0.5f || (fabsf(d) == 0.5f && fmodf(r, 2.0f) != 0.0f))"),
@@ -29,6 +30,9 @@ MUTATIONS = {
                           "a -= (int64_t)qrow[k] * (int64_t)w[n * K + k];\n            if (a > INT32_MAX"),
     "weight_scale_divisor_128": ("quantize_slab(W + n * K, K, 127.0f,", "quantize_slab(W + n * K, K, 128.0f,"),
     "pg_group_offset_dropped": ("quantize_slab(W + n * K + g * gs, gs,", "quantize_slab(W + n * K, gs,"),
+    "w8a16_scale_dropped": ("y[m * N + n] = narrow(a * (double)sw[n], ydt);", "y[m * N + n] = narrow(a, ydt);"),
+    "w8a16_weight_sign_dropped": ("(double)widen(x, m * K + k, xdt) * (double)w[n * K + k];",
+                                  "(double)widen(x, m * K + k, xdt) * fabs((double)w[n * K + k]);"),
 }
 
 PINS = [
@@ -36,6 +40,7 @@ PINS = [
     golden_tests.test_pg_worked_example,
     golden_tests.test_w4a8_worked_example,
     lambda _golden: inv_tests.test_nibble_round_trip_all_bytes(),
+    lambda _golden: w8a16_tests.test_w8a16_worked_example(),
 ]
 
 

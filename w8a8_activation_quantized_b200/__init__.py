@@ -44,6 +44,7 @@ _SIGNATURES = {
     "cider_get_small_m_threshold": (_I64, []),
     "cider_quantize_act": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P]),
     "cider_w8a8_linear_pc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P, _SZ, _P]),
+    "cider_w8a16_mv_pc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_w8a8_linear_pg": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P, _SZ, _P]),
     "cider_w4a8_linear_pg": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P, _SZ, _P]),
     "cider_w8a8_linear_pc_noalloc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
@@ -164,6 +165,18 @@ def cider_w8a8_linear_pc(x, w, scale_w, y=None, out_dtype=None, workspace=None, 
     _check("cider_w8a8_linear_pc", lib().cider_w8a8_linear_pc(
         _ptr(x), _DT[x.dtype], M, K, _ptr(w), _ptr(scale_w), N, _ptr(y), _DT[y.dtype],
         _ptr(ws), ws_bytes, _stream(stream, x.device)))
+    return y
+
+
+def cider_w8a16_mv_pc(x, w, scale_w, y=None, out_dtype=None, stream=None):
+    """W8A16 decode product (1 <= M <= 4): y = scale_w[n] * sum_k x[m,k] * w[n,k]
+    with fp16/bf16 x used as is (no activation quantization)."""
+    _contig(x, "x"), _contig(w, "w")
+    M, K = x.shape
+    N = w.shape[0]
+    y = _out(y, M, N, out_dtype or x.dtype, x.device)
+    _check("cider_w8a16_mv_pc", lib().cider_w8a16_mv_pc(
+        _ptr(x), _DT[x.dtype], M, K, _ptr(w), _ptr(scale_w), N, _ptr(y), _DT[y.dtype], _stream(stream, x.device)))
     return y
 
 

@@ -25,6 +25,8 @@ constexpr int64_t kMaxK = 131072;            // 127 * 128 * K < 2^31 keeps INT32
 constexpr int64_t kMaxSmallM = 16;
 constexpr int64_t kSmallSmemLimit = 160 * 1024;  // q rows of the small-M kernel in shared memory
 constexpr int64_t kSmallMaxK = 32768;
+constexpr int kMaxMvM = 4;                        // rows of the W8A16 decode kernel
+constexpr int kMaxSmallXBytes = 160 * 1024;       // its fp32 activation rows in shared memory
 
 struct DeviceInfo {
     int ready = 0;     // 1 = filled in
@@ -418,6 +420,29 @@ cider_status_t cider_w8a8_linear_pc(const void* x, cider_dtype_t xdt, int64_t M,
                                     const float* scale_w, int64_t N, void* y, cider_dtype_t ydt,
                                     void* workspace, size_t workspace_bytes, void* stream) {
     return linear(kModePC, x, xdt, M, K, w, scale_w, N, 0, y, ydt, workspace, workspace_bytes, stream);
+}
+
+cider_status_t cider_w8a16_mv_pc(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, const int8_t* w,
+                                 const float* scale_w, int64_t N, void* y, cider_dtype_t ydt, void* stream) {
+    t_last_error[0] = '\0';
+    cider_status_t s = check_common(x, M, K, w, scale_w, N, y, xdt, ydt);
+    if (s != CIDER_OK) return s;
+    if (M == 0) return CIDER_OK;
+    if (M > kMaxMvM) return fail(CIDER_ERR_INVALID_ARG, "M = %lld exceeds %d (decode shapes only)", (long long)M, kMaxMvM);
+    const int64_t xbytes = M * ((K / 16 + 31) / 32) * 2048;  // fp32 activations, whole 512-wide passes
+    if (xbytes > kMaxSmallXBytes)
+        return fail(CIDER_ERR_INVALID_ARG, "%lld bytes of staged activations exceed %d", (long long)xbytes,
+                    kMaxSmallXBytes);
+    if (K > kSmallMaxK) return fail(CIDER_ERR_INVALID_ARG, "K = %lld exceeds %lld", (long long)K, (long long)kSmallMaxK);
+    const Range ry = rng(y, static_cast<size_t>(M) * N * 2);
+    if (overlap(ry, rng(x, static_cast<size_t>(M) * K * 2)) || overlap(ry, rng(w, static_cast<size_t>(N) * K)) ||
+        overlap(ry, rng(scale_w, N * 4)))
+        return fail(CIDER_ERR_INVALID_ARG, "y overlaps an input");
+    DeviceInfo* d = nullptr;
+    if ((s = device_info(&d)) != CIDER_OK) return s;
+    cudaError_t e = launch_mv_w8a16(x, xdt, static_cast<int>(M), static_cast<int>(K), w, scale_w, static_cast<int>(N),
+                                    y, ydt, d->num_sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "W8A16 decode kernel launch");
 }
 
 cider_status_t cider_w8a8_linear_pg(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, const int8_t* w,

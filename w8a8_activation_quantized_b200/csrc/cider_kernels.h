@@ -81,6 +81,8 @@ cudaError_t launch_unpack_int4(const uint8_t* packed, int64_t N, int K, int8_t* 
 cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const void* w,
                            const float* sw, int N, int gs, void* y, int ydt, int num_sms,
                            cudaStream_t st);
+cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* w, const float* sw, int N,
+                            void* y, int ydt, int num_sms, cudaStream_t st);
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t st);
 cudaError_t launch_gemm_grouped(const GemmLaunch& L, cudaStream_t st);
 

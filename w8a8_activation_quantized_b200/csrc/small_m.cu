@@ -245,6 +245,162 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
     }
 }
 
+// ---- W8A16 decode matrix-vector product ----------------------------------
+// The pages' decode kernel (Cider README, section "Metal Kernel 流水线",
+// Decode): a direct INT8 matrix-vector product with the weights dequantized
+// on the fly and NO activation quantization.  y[m,n] = round(scale_w[n] *
+// sum_k x[m,k] * w[n,k]) with x widened to fp32 (exact) and the products
+// summed in fp32.  Same streaming layout as k_small_m (persistent grid, R rows
+// x S K-slices, a register ring of 16-byte weight chunks); the M <= 4
+// activation rows are staged once into shared memory as fp32 pairs laid out
+// [pass][pair][lane], so that the lanes of a warp, each holding a different
+// 16-weight chunk, read 32 consecutive pairs at a time (a row-major layout
+// would put them 64 bytes apart: a 16-way bank conflict).
+// fp32 dot of one 16-byte weight chunk with 16 activations.  Each weight is
+// widened exactly without an int->float conversion: after flipping its sign
+// bit the byte is u = w + 128, one byte permute places it under the exponent
+// of 2^23 (the float 2^23 + u), and one packed subtract of 2^23 + 128 leaves
+// w; the products then go through packed FMAs, two per instruction.
+// xs: this lane's first activation pair of the chunk; pair j is at xs[32 * j]
+// (the staging layout [pass][pair][lane] keeps a warp's loads conflict-free).
+__device__ __forceinline__ float chunk_dot_f32(const uint4& wv, const uint64_t* xs) {
+    constexpr float kOff = 8388608.0f + 128.0f;                          // 2^23 + 128
+    const uint64_t neg_off = pack_f32x2(-kOff, -kOff);
+    const uint32_t wd[4] = {wv.x ^ 0x80808080u, wv.y ^ 0x80808080u, wv.z ^ 0x80808080u, wv.w ^ 0x80808080u};
+    uint64_t acc = 0;  // two fp32 partial sums
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t v = wd[i];
+        const uint64_t w01 = f32x2_add(
+            (static_cast<uint64_t>(__byte_perm(v, 0x4B000000u, 0x7651)) << 32) | __byte_perm(v, 0x4B000000u, 0x7650),
+            neg_off);
+        const uint64_t w23 = f32x2_add(
+            (static_cast<uint64_t>(__byte_perm(v, 0x4B000000u, 0x7653)) << 32) | __byte_perm(v, 0x4B000000u, 0x7652),
+            neg_off);
+        acc = f32x2_fma(w01, xs[32 * (2 * i)], acc);
+        acc = f32x2_fma(w23, xs[32 * (2 * i + 1)], acc);
+    }
+    return lo_f32(acc) + hi_f32(acc);
+}
+
+template <typename TX, int MAXM, int PPW>
+__global__ void __launch_bounds__(kSmallThreads, 2) k_mv_w8a16(const TX* __restrict__ x, int M, int K,
+                                                               const int8_t* __restrict__ w,
+                                                               const float* __restrict__ sw, int N,
+                                                               void* __restrict__ y, int ydt, SmallGeom geo) {
+    extern __shared__ __align__(16) uint64_t s_x[];  // [M][pass][8 pairs][32 lanes] fp32 pairs
+    __shared__ float s_part[kSmallWarps][MAXM];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nch = K / 16;
+    const int npass = (nch + 31) / 32;
+    const int r_in_blk = warp / geo.S, slice = warp % geo.S;
+    const int pass0 = slice * geo.ppw;
+    pdl_wait();
+    pdl_trigger();
+
+    constexpr int kRing = RingDepth<PPW>::value;
+    uint4 ring[kRing][PPW];
+    float ring_s[kRing];
+    auto load = [&](uint4 (&dst)[PPW], float& ds, int blk) {
+        const int n = blk * geo.R + r_in_blk;
+        const bool row_ok = blk < geo.nblocks && n < N;
+        const uint4* wr = reinterpret_cast<const uint4*>(w + static_cast<int64_t>(n) * K);
+#pragma unroll
+        for (int p = 0; p < PPW; ++p) {
+            const int c = (pass0 + p) * 32 + lane;
+            const bool ok = p < geo.ppw && row_ok && c < nch;
+            dst[p] = ok ? __ldcs(wr + c) : make_uint4(0, 0, 0, 0);
+        }
+        ds = row_ok ? __ldg(sw + n) : 0.0f;
+    };
+#pragma unroll
+    for (int i = 0; i < kRing - 1; ++i) load(ring[i], ring_s[i], blockIdx.x + i * gridDim.x);
+
+    // stage the activations as fp32 pairs (exact widening): the 8 values at
+    // k0 = 8t belong to chunk c = k0 / 16 (pass c / 32, lane c % 32), pairs
+    // (k0 % 16) / 2 .. + 3
+    const int nx = K / 8;
+    for (int m = 0; m < M; ++m) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K);
+        for (int t = threadIdx.x; t < nx; t += kSmallThreads) {
+            float f[8];
+            unpack8_f32<TX>(__ldg(xr + t), f);
+            const int c = t >> 1, q = c >> 5, l = c & 31, j0 = (t & 1) * 4;
+            uint64_t* dst = s_x + ((static_cast<int64_t>(m) * npass + q) * 8 + j0) * 32 + l;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[32 * j] = pack_f32x2(f[2 * j], f[2 * j + 1]);
+        }
+    }
+    __syncthreads();
+
+    auto step = [&](const uint4 (&cur)[PPW], float cs, int blk) {
+        const int n = blk * geo.R + r_in_blk;
+        float acc[MAXM];
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) acc[m] = 0.0f;
+        if (n < N) {
+#pragma unroll
+            for (int p = 0; p < PPW; ++p) {
+                if (p >= geo.ppw || (pass0 + p) * 32 >= nch) break;  // warp-uniform
+                const int c = (pass0 + p) * 32 + lane;
+                if (c < nch) {
+#pragma unroll
+                    for (int m = 0; m < MAXM; ++m)
+                        if (m < M)
+                            acc[m] += chunk_dot_f32(cur[p], s_x + ((static_cast<int64_t>(m) * npass + pass0 + p) * 8) * 32 + lane);
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) {
+            if (m < M) {
+                float a = acc[m];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+                if (geo.S == 1) {
+                    if (lane == 0 && n < N) {
+                        const float out = a * cs;
+                        if (ydt == 1)
+                            static_cast<__nv_bfloat16*>(y)[static_cast<int64_t>(m) * N + n] = __float2bfloat16_rn(out);
+                        else
+                            static_cast<__half*>(y)[static_cast<int64_t>(m) * N + n] = __float2half_rn(out);
+                    }
+                } else if (lane == 0) {
+                    s_part[warp][m] = a;
+                }
+            }
+        }
+        if (geo.S > 1) {
+            __syncthreads();
+            for (int t = threadIdx.x; t < geo.R * M; t += kSmallThreads) {
+                const int rr = t / M, m = t % M;
+                const int nn = blk * geo.R + rr;
+                if (nn < N) {
+                    float a = 0.0f;
+                    for (int sl = 0; sl < geo.S; ++sl) a += s_part[rr * geo.S + sl][m];
+                    const float out = a * __ldg(sw + nn);
+                    if (ydt == 1)
+                        static_cast<__nv_bfloat16*>(y)[static_cast<int64_t>(m) * N + nn] = __float2bfloat16_rn(out);
+                    else
+                        static_cast<__half*>(y)[static_cast<int64_t>(m) * N + nn] = __float2half_rn(out);
+                }
+            }
+            __syncthreads();
+        }
+    };
+    int blk = blockIdx.x;
+    while (blk < geo.nblocks) {
+#pragma unroll
+        for (int r = 0; r < kRing; ++r) {
+            if (blk < geo.nblocks) {
+                load(ring[(r + kRing - 1) % kRing], ring_s[(r + kRing - 1) % kRing], blk + (kRing - 1) * gridDim.x);
+                step(ring[r], ring_s[r], blk);
+            }
+            blk += gridDim.x;
+        }
+    }
+}
+
 // Slices per row: as many as keep at least 4 passes per warp (at most 8).
 static SmallGeom small_geom(int K, int N, bool w4) {
     SmallGeom g;
@@ -298,6 +454,40 @@ static cudaError_t launch_small_m_v(const void* x, int xdt, int M, int K, const 
                                     int gs, void* y, int ydt, int num_sms, cudaStream_t st) {
     if (xdt == 1) return launch_small_m_t<__nv_bfloat16, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
     return launch_small_m_t<__half, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
+}
+
+template <typename TX, int MAXM, int PPW>
+static cudaError_t launch_mv_t(const void* x, int M, int K, const int8_t* w, const float* sw, int N, void* y,
+                               int ydt, const SmallGeom& geo, int num_sms, cudaStream_t st) {
+    const size_t smem = static_cast<size_t>(M) * ((K / 16 + 31) / 32) * 2048;  // whole passes of pairs
+    auto kern = k_mv_w8a16<TX, MAXM, PPW>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+    }
+    const int grid = geo.nblocks < 2 * num_sms ? geo.nblocks : 2 * num_sms;
+    return launch_pdl(kern, grid, kSmallThreads, smem, st, static_cast<const TX*>(x), M, K, w, sw, N, y, ydt, geo);
+}
+
+template <typename TX, int MAXM>
+static cudaError_t launch_mv_ppw(const void* x, int M, int K, const int8_t* w, const float* sw, int N, void* y,
+                                 int ydt, int num_sms, cudaStream_t st) {
+    const SmallGeom geo = small_geom(K, N, false);
+    if (geo.ppw <= 2) return launch_mv_t<TX, MAXM, 2>(x, M, K, w, sw, N, y, ydt, geo, num_sms, st);
+    if (geo.ppw <= 4) return launch_mv_t<TX, MAXM, 4>(x, M, K, w, sw, N, y, ydt, geo, num_sms, st);
+    if (geo.ppw <= 5) return launch_mv_t<TX, MAXM, 5>(x, M, K, w, sw, N, y, ydt, geo, num_sms, st);
+    if (geo.ppw <= 8) return launch_mv_t<TX, MAXM, 8>(x, M, K, w, sw, N, y, ydt, geo, num_sms, st);
+    return cudaErrorInvalidValue;  // K beyond the kernel: rejected by the host checks first
+}
+
+cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* w, const float* sw, int N,
+                            void* y, int ydt, int num_sms, cudaStream_t st) {
+    if (xdt == 1) {
+        if (M <= 1) return launch_mv_ppw<__nv_bfloat16, 1>(x, M, K, w, sw, N, y, ydt, num_sms, st);
+        return launch_mv_ppw<__nv_bfloat16, 4>(x, M, K, w, sw, N, y, ydt, num_sms, st);
+    }
+    if (M <= 1) return launch_mv_ppw<__half, 1>(x, M, K, w, sw, N, y, ydt, num_sms, st);
+    return launch_mv_ppw<__half, 4>(x, M, K, w, sw, N, y, ydt, num_sms, st);
 }
 
 cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const void* w,
