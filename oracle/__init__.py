@@ -59,6 +59,9 @@ def _bind(path):
         "oracle_quantize_weight_pc": (None, [_ptr, _i64, _i64, _ptr, _ptr]),
         "oracle_quantize_weight_pg": (None, [_ptr, _i64, _i64, _i64, _ptr, _ptr]),
         "oracle_quantize_weight_int4_pg": (None, [_ptr, _i64, _i64, _i64, _ptr, _ptr]),
+        "oracle_quantize_weight_pc_clip": (None, [_ptr, _i64, _i64, ctypes.c_double, _ptr, _ptr]),
+        "oracle_quantize_weight_pg_clip": (None, [_ptr, _i64, _i64, _i64, ctypes.c_double, _ptr, _ptr]),
+        "oracle_percentile_position": (None, [ctypes.c_double, _i64, _ptr, _ptr]),
         "oracle_unpack_int4": (None, [_ptr, _i64, _i64, _ptr]),
         "oracle_gemm_i32": (_int, [_ptr, _ptr, _i64, _i64, _i64, _ptr]),
         "oracle_gemm_i32_grouped": (_int, [_ptr, _ptr, _i64, _i64, _i64, _i64, _ptr]),
@@ -166,6 +169,39 @@ def quantize_weight_pg(W, gs):
     qw = np.empty((N, K), np.int8)
     sw = np.empty((N, K // gs), np.float32)
     _load().oracle_quantize_weight_pg(_p(W), N, K, gs, _p(qw), _p(sw))
+    return qw, sw
+
+
+def percentile_position(p, n):
+    """-> (i, t): the p-th percentile of n ascending values lies a fraction t
+    of the way from the i-th to the (i+1)-th (t is fp32)."""
+    i = ctypes.c_int64()
+    t = ctypes.c_float()
+    _load().oracle_percentile_position(float(p), int(n), ctypes.byref(i), ctypes.byref(t))
+    return i.value, np.float32(t.value)
+
+
+def quantize_weight_pc_clip(W, p):
+    """Percentile-clipped per-channel weights (Cider README, section "说明",
+    clip_percentile): W f32 [N,K] -> (qw int8 [N,K] in [-127,127], sw f32 [N])."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    qw = np.empty((N, K), np.int8)
+    sw = np.empty((N,), np.float32)
+    _load().oracle_quantize_weight_pc_clip(_p(W), N, K, float(p), _p(qw), _p(sw))
+    return qw, sw
+
+
+def quantize_weight_pg_clip(W, gs, p):
+    """Percentile-clipped per-group weights: W f32 [N,K] -> (qw int8 [N,K],
+    sw f32 [N, K/gs])."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    if K % gs:
+        raise ValueError("gs must divide K")
+    qw = np.empty((N, K), np.int8)
+    sw = np.empty((N, K // gs), np.float32)
+    _load().oracle_quantize_weight_pg_clip(_p(W), N, K, gs, float(p), _p(qw), _p(sw))
     return qw, sw
 
 

@@ -31,6 +31,10 @@
  *  - scale_x, scale_w are fp32; t = x / scale_x is one correctly rounded fp32
  *    division by the stored scale (not a multiply by 127/amax);
  *  - an all-zero token has scale 0 and q = 0;
+ *  - clip_percentile: the percentile of the magnitudes |w| of a slab, by
+ *    linear interpolation at position p/100*(len-1) (the t of that position
+ *    rounded once to fp32, the interpolation in fp32), codes clipped to
+ *    [-127, 127]; a zero percentile falls back to max|w|;
  *  - INT4 weights: q in [-8,7] from scale = max|w_group|/7, stored as the
  *    offset-binary nibble q+8, two per byte, low nibble = even k;
  *  - the dequant is evaluated in fp64 here and rounded once to fp16/bf16
@@ -39,6 +43,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define ORACLE_F16 0
@@ -212,6 +217,95 @@ void oracle_quantize_weight_pg(const float* W, int64_t N, int64_t K, int64_t gs,
         for (int64_t g = 0; g < G; ++g)
             quantize_slab(W + n * K + g * gs, gs, 127.0f, -128, 127, qw + n * K + g * gs,
                           sw + n * G + g);
+}
+
+/* ---------------------------------------------------------------------- */
+/* Percentile-clipped weight scales  [README "说明": the conversion takes   */
+/* its scales by min-max by default and also supports a percentile method, */
+/* clip_percentile=99.9]                                                    */
+/* The clipping value c of a slab is the p-th percentile of its magnitudes */
+/* |w|, linearly interpolated between order statistics (the common         */
+/* definition: position p/100 * (len-1) in the ascending order); scale =   */
+/* c / 127 and codes clip symmetrically to [-127, 127].  A slab whose      */
+/* percentile is 0 (mostly zeros) takes c = max|w| instead.                */
+/* ---------------------------------------------------------------------- */
+
+/* Position of the p-th percentile among len ascending values: index i of
+ * the lower neighbour and the fraction t towards the next one.  Evaluated
+ * in double, t rounded once to float. */
+void oracle_percentile_position(double p, int64_t len, int64_t* i_out, float* t_out)
+{
+    double pos = p / 100.0 * (double)(len - 1);
+    int64_t i = (int64_t)floor(pos);
+    if (i > len - 1)
+        i = len - 1;
+    if (i < 0)
+        i = 0;
+    *i_out = i;
+    *t_out = (float)(pos - (double)i);
+}
+
+static int cmp_float_asc(const void* a, const void* b)
+{
+    float x = *(const float*)a, y = *(const float*)b;
+    return (x > y) - (x < y);
+}
+
+/* p-th percentile of |w[0..len)|: sort the magnitudes, then
+ * v = a[i] + t * (a[i+1] - a[i]) in three rounded fp32 operations. */
+static float abs_percentile(const float* w, int64_t len, int64_t i, float t)
+{
+    float* a = (float*)malloc((size_t)len * sizeof(float));
+    for (int64_t k = 0; k < len; ++k)
+        a[k] = fabsf(w[k]);
+    qsort(a, (size_t)len, sizeof(float), cmp_float_asc);
+    float v = a[i];
+    if (t != 0.0f && i + 1 < len) {
+        float d = a[i + 1] - a[i];
+        float td = t * d;
+        v = a[i] + td;
+    }
+    free(a);
+    return v;
+}
+
+static void quantize_slab_clip(const float* w, int64_t len, int64_t i, float t, int8_t* qw, float* s_out)
+{
+    float amax = 0.0f;
+    for (int64_t k = 0; k < len; ++k)
+        if (fabsf(w[k]) > amax)
+            amax = fabsf(w[k]);
+    float v = abs_percentile(w, len, i, t);
+    float c = (v == 0.0f) ? amax : v;
+    float s = c / 127.0f;
+    *s_out = s;
+    for (int64_t k = 0; k < len; ++k)
+        qw[k] = (c == 0.0f) ? 0 : (int8_t)clamp_int(oracle_round_half_away(w[k] / s), -127, 127);
+}
+
+/* per output channel, clipped: sw[n] = pct_p(|W[n,:]|) / 127 */
+void oracle_quantize_weight_pc_clip(const float* W, int64_t N, int64_t K, double p, int8_t* qw, float* sw)
+{
+    int64_t i;
+    float t;
+    oracle_percentile_position(p, K, &i, &t);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        quantize_slab_clip(W + n * K, K, i, t, qw + n * K, sw + n);
+}
+
+/* per group of gs, clipped: sw[n][g] = pct_p(|W[n, g*gs:(g+1)*gs]|) / 127 */
+void oracle_quantize_weight_pg_clip(const float* W, int64_t N, int64_t K, int64_t gs, double p,
+                                    int8_t* qw, float* sw)
+{
+    const int64_t G = K / gs;
+    int64_t i;
+    float t;
+    oracle_percentile_position(p, gs, &i, &t);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < G; ++g)
+            quantize_slab_clip(W + n * K + g * gs, gs, i, t, qw + n * K + g * gs, sw + n * G + g);
 }
 
 /* INT4, per group: q in [-8,7] from scale max|w|/7, packed as nibble q+8,

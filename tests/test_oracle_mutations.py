@@ -17,6 +17,7 @@ from oracle.build import CFLAGS, SRC
 from tests import test_oracle_golden as golden_tests
 from tests import test_oracle_invariants as inv_tests
 from tests import test_oracle_w8a16 as w8a16_tests
+from tests import test_oracle_clip as clip_tests
 
 MUTATIONS = {
     "round_half_to_even_codes": ("if (fabsf(d) >= 0.5f)", "if (fabsf(d) > 0.5f || (fabsf(d) == 0.5f && fmodf(r, 2.0f) != 0.0f))"),
@@ -33,6 +34,12 @@ MUTATIONS = {
     "w8a16_scale_dropped": ("y[m * N + n] = narrow(a * (double)sw[n], ydt);", "y[m * N + n] = narrow(a, ydt);"),
     "w8a16_weight_sign_dropped": ("(double)widen(x, m * K + k, xdt) * (double)w[n * K + k];",
                                   "(double)widen(x, m * K + k, xdt) * fabs((double)w[n * K + k]);"),
+    "clip_interpolation_sign": ("v = a[i] + td;", "v = a[i] - td;"),
+    "clip_position_uses_len": ("double pos = p / 100.0 * (double)(len - 1);", "double pos = p / 100.0 * (double)len;"),
+    "clip_asymmetric_128": ("clamp_int(oracle_round_half_away(w[k] / s), -127, 127)",
+                            "clamp_int(oracle_round_half_away(w[k] / s), -128, 127)"),
+    "clip_no_zero_fallback": ("float c = (v == 0.0f) ? amax : v;", "float c = v;"),
+    "clip_pg_group_offset_dropped": ("quantize_slab_clip(W + n * K + g * gs, gs,", "quantize_slab_clip(W + n * K, gs,"),
 }
 
 PINS = [
@@ -41,6 +48,10 @@ PINS = [
     golden_tests.test_w4a8_worked_example,
     lambda _golden: inv_tests.test_nibble_round_trip_all_bytes(),
     lambda _golden: w8a16_tests.test_w8a16_worked_example(),
+    lambda _golden: clip_tests.test_clip_pc_worked_example_p90(),
+    lambda _golden: clip_tests.test_clip_pc_worked_example_interpolated(),
+    lambda _golden: clip_tests.test_clip_pg_worked_example(),
+    lambda _golden: clip_tests.test_clip_zero_percentile_falls_back_to_max(),
 ]
 
 
