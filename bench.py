@@ -494,6 +494,19 @@ def bench_rows(device, pk, steps, warmup):
     sb = torch.empty((M,), dtype=torch.float32, device=device)
     ms = graph_time(lambda i: cider.cider_silu_mul_quantize(gts[i % 3], uts[i % 3], q=qb[i % 3], scale_x=sb), steps, warmup)
     record("silu_mul_quantize", ms, 0, M * F * 5 + M * 4, M=M, F=F)
+    del gts, uts, qb
+    # offline conversion with percentile-clipped scales (clip_percentile = 99.9)
+    for (N, K, gs) in ((10240, 2560, 0), (2560, 10240, 64)):
+        n = rotating(N * K * 5)
+        Ws = [torch.from_numpy(synth.weights(N, K, 4000 + i)).to(device) for i in range(n)]
+        if gs == 0:
+            ms = graph_time(lambda i: cider.cider_quantize_weight_pc_clip(Ws[i % n], 99.9), steps, warmup)
+            record("quantize_weight_pc_clip", ms, 0, N * K * 5 + N * 4, N=N, K=K, clip_percentile=99.9)
+        else:
+            ms = graph_time(lambda i: cider.cider_quantize_weight_pg_clip(Ws[i % n], gs, 99.9), steps, warmup)
+            record("quantize_weight_pg_clip", ms, 0, N * K * 5 + N * (K // gs) * 4, gs=gs, N=N, K=K,
+                   clip_percentile=99.9)
+        del Ws
     out.append(bench_stack(device, pk, steps=max(3, steps // 20), warmup=warmup))
     return out
 

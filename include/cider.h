@@ -223,6 +223,23 @@ CIDER_API cider_status_t cider_quantize_weight_pc(const float* W, int64_t N, int
 /* Per group of gs along K: scale_w[g][n] = max |W[n, g*gs:(g+1)*gs]| / 127 (group-major). */
 CIDER_API cider_status_t cider_quantize_weight_pg(const float* W, int64_t N, int64_t K, int64_t gs,
                                         int8_t* w, float* scale_w, void* stream);
+/* Percentile-clipped scales (Cider README, section "说明": the conversion's
+ * scales come from min-max by default or from a percentile,
+ * clip_percentile = 99.9).  Per slab -- an output row (_pc) or one group of
+ * gs = 64 or 128 along K (_pg) -- c = the clip_percentile-th percentile of
+ * |W| over the slab, linearly interpolated at position p/100 * (len - 1) of
+ * the ascending order (the position in double; its fraction rounded once to
+ * float; the interpolation in fp32); c = max|W| when that percentile is 0.
+ * scale_w = c / 127 and w = clamp(round(W / scale_w), -127, 127): values
+ * beyond the percentile saturate symmetrically.  clip_percentile = 100
+ * gives exactly the min-max result above.  Same layouts as the min-max
+ * versions (scale_w [N] or group-major [K/gs][N]); W, w and scale_w are
+ * device pointers owned by the caller.  Errors: CIDER_ERR_INVALID_ARG for
+ * clip_percentile outside [0, 100] (or NaN), bad sizes, gs, or NULL. */
+CIDER_API cider_status_t cider_quantize_weight_pc_clip(const float* W, int64_t N, int64_t K, double clip_percentile,
+                                             int8_t* w, float* scale_w, void* stream);
+CIDER_API cider_status_t cider_quantize_weight_pg_clip(const float* W, int64_t N, int64_t K, int64_t gs,
+                                             double clip_percentile, int8_t* w, float* scale_w, void* stream);
 /* INT4 per group: scale_w[g][n] = max|W_group| / 7, q = clamp(round(W/scale), -8, 7),
  * packed as described above. */
 CIDER_API cider_status_t cider_pack_weight_int4_pg(const float* W, int64_t N, int64_t K, int64_t gs,

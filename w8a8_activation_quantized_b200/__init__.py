@@ -54,6 +54,8 @@ _SIGNATURES = {
     "cider_silu_mul_quantize": (_INT, [_P, _P, _INT, _I64, _I64, _P, _P, _P, _P]),
     "cider_quantize_weight_pc": (_INT, [_P, _I64, _I64, _P, _P, _P]),
     "cider_quantize_weight_pg": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "cider_quantize_weight_pc_clip": (_INT, [_P, _I64, _I64, ctypes.c_double, _P, _P, _P]),
+    "cider_quantize_weight_pg_clip": (_INT, [_P, _I64, _I64, _I64, ctypes.c_double, _P, _P, _P]),
     "cider_pack_weight_int4_pg": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "cider_test_gemm_i32": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P]),
     "cider_test_gemm_i32_grouped": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _P, _P]),
@@ -281,6 +283,28 @@ def cider_quantize_weight_pg(W, gs, stream=None):
     s = torch.empty((K // gs, N), dtype=torch.float32, device=W.device)
     _check("cider_quantize_weight_pg", lib().cider_quantize_weight_pg(
         _ptr(_contig(W, "W")), N, K, gs, _ptr(w), _ptr(s), _stream(stream, W.device)))
+    return w, s
+
+
+def cider_quantize_weight_pc_clip(W, clip_percentile, stream=None):
+    """Percentile-clipped per channel: W fp32 [N, K] -> (w int8 [N, K] in
+    [-127, 127], scale_w fp32 [N])."""
+    N, K = W.shape
+    w = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    s = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _check("cider_quantize_weight_pc_clip", lib().cider_quantize_weight_pc_clip(
+        _ptr(_contig(W, "W")), N, K, float(clip_percentile), _ptr(w), _ptr(s), _stream(stream, W.device)))
+    return w, s
+
+
+def cider_quantize_weight_pg_clip(W, gs, clip_percentile, stream=None):
+    """Percentile-clipped per group: W fp32 [N, K] -> (w int8 [N, K],
+    scale_w fp32 [K/gs, N])."""
+    N, K = W.shape
+    w = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    s = torch.empty((K // gs, N), dtype=torch.float32, device=W.device)
+    _check("cider_quantize_weight_pg_clip", lib().cider_quantize_weight_pg_clip(
+        _ptr(_contig(W, "W")), N, K, gs, float(clip_percentile), _ptr(w), _ptr(s), _stream(stream, W.device)))
     return w, s
 
 

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -511,6 +512,45 @@ static cider_status_t quantize_weight(int mode, const float* W, int64_t N, int64
     cudaError_t e = launch_quantize_weight(mode, W, N, static_cast<int>(K), static_cast<int>(gs), out, sw,
                                            static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "weight quantize launch");
+}
+
+// Percentile-clipped scales.  The position of the percentile within a slab of
+// len values is p/100 * (len - 1) in double, split into the order statistic
+// k0 = floor and the fraction t (rounded once to float); the kernels
+// interpolate in fp32.
+static cider_status_t quantize_weight_clip(const float* W, int64_t N, int64_t K, int64_t gs, double p,
+                                           int8_t* out, float* sw, void* stream) {
+    t_last_error[0] = '\0';
+    if (!(p >= 0.0 && p <= 100.0))
+        return fail(CIDER_ERR_INVALID_ARG, "clip_percentile = %g must lie in [0, 100]", p);
+    if (N < 1 || K < 1) return fail(CIDER_ERR_INVALID_ARG, "N, K >= 1 required");
+    if (N > INT32_MAX || K > kMaxK) return fail(CIDER_ERR_INVALID_ARG, "size out of range");
+    if (gs != 0) {
+        cider_status_t s = check_gs(K, gs, false);
+        if (s != CIDER_OK) return s;
+    }
+    if (!W || !out || !sw) return fail(CIDER_ERR_INVALID_ARG, "NULL pointer");
+    DeviceInfo* d = nullptr;
+    cider_status_t s = device_info(&d);
+    if (s != CIDER_OK) return s;
+    const int64_t len = gs != 0 ? gs : K;
+    const double pos = p / 100.0 * static_cast<double>(len - 1);
+    int64_t k0 = static_cast<int64_t>(std::floor(pos));
+    k0 = std::min<int64_t>(std::max<int64_t>(k0, 0), len - 1);
+    const float t = static_cast<float>(pos - static_cast<double>(k0));
+    cudaError_t e = launch_quantize_weight_clip(W, N, static_cast<int>(K), static_cast<int>(gs), static_cast<int>(k0),
+                                                t, out, sw, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "clipped weight quantize launch");
+}
+
+cider_status_t cider_quantize_weight_pc_clip(const float* W, int64_t N, int64_t K, double clip_percentile, int8_t* w,
+                                             float* scale_w, void* stream) {
+    return quantize_weight_clip(W, N, K, 0, clip_percentile, w, scale_w, stream);
+}
+
+cider_status_t cider_quantize_weight_pg_clip(const float* W, int64_t N, int64_t K, int64_t gs, double clip_percentile,
+                                             int8_t* w, float* scale_w, void* stream) {
+    return quantize_weight_clip(W, N, K, gs, clip_percentile, w, scale_w, stream);
 }
 
 cider_status_t cider_quantize_weight_pc(const float* W, int64_t N, int64_t K, int8_t* w, float* scale_w,

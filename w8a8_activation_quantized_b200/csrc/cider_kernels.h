@@ -76,6 +76,10 @@ cudaError_t launch_silu_mul_quantize(const void* g, const void* u, int dt, int64
 // mode 0: per channel (out = int8 [N][K]); 1: per group int8; 2: per group int4 packed
 cudaError_t launch_quantize_weight(int mode, const float* W, int64_t N, int K, int gs, void* out,
                                    float* sw, cudaStream_t st);
+// percentile-clipped weights: gs = 0 per channel, else per group of gs (64 or 128);
+// k0, t: the percentile's position within a slab (order statistic k0, fraction t)
+cudaError_t launch_quantize_weight_clip(const float* W, int64_t N, int K, int gs, int k0, float t, int8_t* out,
+                                        float* sw, cudaStream_t st);
 cudaError_t launch_wait_selftest(unsigned* status, unsigned long long limit_ns, cudaStream_t st);
 cudaError_t launch_unpack_int4(const uint8_t* packed, int64_t N, int K, int8_t* w, cudaStream_t st);
 cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const void* w,

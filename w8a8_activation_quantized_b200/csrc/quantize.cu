@@ -342,6 +342,139 @@ cudaError_t launch_quantize_weight(int mode, const float* W, int64_t N, int K, i
     return launch_pdl(k_quantize_weight_group<true>, grid, 256, 0, st, W, N, K, gs, out, sw);
 }
 
+// ---- percentile-clipped weight scales (clip_percentile) ----------------------
+// Cider README, section "说明": besides min-max, the conversion can take its
+// scales from a percentile of the weights (clip_percentile = 99.9).  Per slab
+// (an output row, or one group of gs along K): c = the p-th percentile of
+// |w|, linearly interpolated between the order statistics k0 and k0 + 1 with
+// weight t (k0 and t come from the host); scale = c / 127; codes
+// clamp(round(w / scale), -127, 127).  A zero percentile takes c = max|w|.
+//
+// The order statistics are found bit by bit from the top: the k-th smallest
+// magnitude is the largest pattern r with at most k magnitudes below it
+// (|x| as an unsigned bit pattern orders like |x|).  Each of the 31 counting
+// passes (bit 31 of |x| is 0) counts for both statistics at once.  Exact for
+// any slab length; the conversion runs once per model, so the passes read
+// the row through L1 rather than holding it on chip.
+
+__device__ __forceinline__ float clip_value(uint32_t r0, uint32_t r1, bool two, float t, float amax) {
+    const float a = __uint_as_float(r0);
+    const float v = two ? __fadd_rn(a, __fmul_rn(t, __fsub_rn(__uint_as_float(r1), a))) : a;
+    return v == 0.0f ? amax : v;
+}
+__device__ __forceinline__ int8_t clip_code(float x, float s) {
+    return static_cast<int8_t>(max(quant_code(x, s), -127));
+}
+
+// Per channel: one CTA of 256 threads per output row.
+__global__ void __launch_bounds__(256) k_quantize_weight_pc_clip(const float* __restrict__ W, int K, int k0,
+                                                                 float t, int8_t* __restrict__ w,
+                                                                 float* __restrict__ sw) {
+    __shared__ int red[2][8][2];
+    __shared__ float redm[8];
+    pdl_wait();
+    pdl_trigger();
+    const int64_t n = blockIdx.x;
+    const float* wr = W + n * K;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    float amax = 0.0f;
+    for (int k = tid; k < K; k += 256) amax = fmaxf(amax, fabsf(wr[k]));
+    amax = warp_max(amax);
+    if (lane == 0) redm[wp] = amax;
+    __syncthreads();
+    amax = redm[0];
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, redm[i]);
+    uint32_t r0 = 0, r1 = 0;
+    for (int b = 30; b >= 0; --b) {
+        const uint32_t t0 = r0 | (1u << b), t1 = r1 | (1u << b);
+        int c0 = 0, c1 = 0;
+        for (int k = tid; k < K; k += 256) {
+            const uint32_t u = __float_as_uint(fabsf(__ldg(wr + k)));
+            c0 += u < t0;
+            c1 += u < t1;
+        }
+        c0 = __reduce_add_sync(0xffffffffu, c0);
+        c1 = __reduce_add_sync(0xffffffffu, c1);
+        // two buffers: a pass's writes never meet the previous pass's reads
+        int(*rb)[2] = red[b & 1];
+        if (lane == 0) {
+            rb[wp][0] = c0;
+            rb[wp][1] = c1;
+        }
+        __syncthreads();
+        c0 = c1 = 0;
+        for (int i = 0; i < 8; ++i) {
+            c0 += rb[i][0];
+            c1 += rb[i][1];
+        }
+        if (c0 <= k0) r0 = t0;
+        if (c1 <= k0 + 1) r1 = t1;
+    }
+    const float c = clip_value(r0, r1, t != 0.0f && k0 + 1 < K, t, amax);
+    const float s = act_scale(c);
+    if (tid == 0) sw[n] = s;
+    for (int k = tid; k < K; k += 256) w[n * K + k] = clip_code(wr[k], s);
+}
+
+// Per group: one warp per (row n, group g), the group's gs = 32 * VPL
+// magnitudes held in registers; scales group-major [G][N].
+template <int VPL>
+__global__ void __launch_bounds__(256) k_quantize_weight_pg_clip(const float* __restrict__ W, int64_t N, int K,
+                                                                 int k0, float t, int8_t* __restrict__ out,
+                                                                 float* __restrict__ sw) {
+    pdl_wait();
+    pdl_trigger();
+    constexpr int GS = 32 * VPL;
+    const int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = K / GS;
+    if (item >= N * G) return;  // whole warps
+    const int64_t n = item / G;
+    const int g = static_cast<int>(item % G);
+    const float* wg = W + n * K + static_cast<int64_t>(g) * GS;
+    float x[VPL];
+    uint32_t u[VPL];
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        x[j] = wg[lane + 32 * j];
+        u[j] = __float_as_uint(fabsf(x[j]));
+        amax = fmaxf(amax, fabsf(x[j]));
+    }
+    amax = warp_max(amax);
+    uint32_t r0 = 0, r1 = 0;
+    for (int b = 30; b >= 0; --b) {
+        const uint32_t t0 = r0 | (1u << b), t1 = r1 | (1u << b);
+        int c0 = 0, c1 = 0;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            c0 += u[j] < t0;
+            c1 += u[j] < t1;
+        }
+        c0 = __reduce_add_sync(0xffffffffu, c0);
+        c1 = __reduce_add_sync(0xffffffffu, c1);
+        if (c0 <= k0) r0 = t0;
+        if (c1 <= k0 + 1) r1 = t1;
+    }
+    const float c = clip_value(r0, r1, t != 0.0f && k0 + 1 < GS, t, amax);
+    const float s = act_scale(c);
+    if (lane == 0) sw[static_cast<int64_t>(g) * N + n] = s;
+    int8_t* w = out + n * K + static_cast<int64_t>(g) * GS;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) w[lane + 32 * j] = clip_code(x[j], s);
+}
+
+cudaError_t launch_quantize_weight_clip(const float* W, int64_t N, int K, int gs, int k0, float t, int8_t* out,
+                                        float* sw, cudaStream_t st) {
+    if (gs == 0)
+        return launch_pdl(k_quantize_weight_pc_clip, static_cast<unsigned>(N), 256, 0, st, W, K, k0, t, out, sw);
+    const int64_t items = N * (K / gs);
+    const unsigned grid = static_cast<unsigned>((items + 7) / 8);
+    if (gs == 64) return launch_pdl(k_quantize_weight_pg_clip<2>, grid, 256, 0, st, W, N, K, k0, t, out, sw);
+    if (gs == 128) return launch_pdl(k_quantize_weight_pg_clip<4>, grid, 256, 0, st, W, N, K, k0, t, out, sw);
+    return cudaErrorInvalidValue;  // rejected by the host checks first
+}
+
 // ---- INT4 unpack (the W4A8 load path's conversion), standalone ---------------
 __global__ void k_unpack_int4(const uint32_t* __restrict__ packed, int64_t words, uint2* __restrict__ w) {
     pdl_wait();
