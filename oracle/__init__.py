@@ -217,6 +217,16 @@ def quantize_weight_int4_pg(W, gs):
     return packed, sw
 
 
+def quantize_weight_int4_pc(W):
+    """INT4 weights with one scale per output channel (Cider README, table
+    "量化": W4A8 weights symmetric INT4, zp = 8, per column) -- the per-group
+    definition with a single group spanning K.  W f32 [N,K] -> (packed uint8
+    [N, K/2], sw f32 [N])."""
+    W = _c(W, np.float32)
+    packed, sw = quantize_weight_int4_pg(W, W.shape[1])
+    return packed, np.ascontiguousarray(sw[:, 0])
+
+
 def unpack_int4(packed, K):
     packed = _c(packed, np.uint8)
     N = packed.shape[0]
@@ -315,6 +325,13 @@ def w4a8_linear_pg(x, packed, sw, gs, xdt=F16, ydt=F16):
                                      _p(y), _p(scratch)) != 0:
         raise OverflowError("INT32 accumulator overflow")
     return y
+
+
+def w4a8_linear_pc(x, packed, sw, xdt=F16, ydt=F16):
+    """W4A8 linear with per-output-channel scales (sw [N]): the per-group
+    linear with one group spanning K, y = round(acc * scale_x * sw[n])."""
+    K = _bits(x, xdt).shape[1]
+    return w4a8_linear_pg(x, packed, _c(sw, np.float32).reshape(-1, 1), K, xdt, ydt)
 
 
 def silu_mul(g, u, dt=F16):

@@ -18,6 +18,7 @@ from tests import test_oracle_golden as golden_tests
 from tests import test_oracle_invariants as inv_tests
 from tests import test_oracle_w8a16 as w8a16_tests
 from tests import test_oracle_clip as clip_tests
+from tests import test_oracle_w4pc as w4pc_tests
 
 MUTATIONS = {
     "round_half_to_even_codes": ("if (fabsf(d) >= 0.5f)", "if (fabsf(d) > 0.5f || (fabsf(d) == 0.5f && fmodf(r, 2.0f) != 0.0f))"),
@@ -52,6 +53,7 @@ PINS = [
     lambda _golden: clip_tests.test_clip_pc_worked_example_interpolated(),
     lambda _golden: clip_tests.test_clip_pg_worked_example(),
     lambda _golden: clip_tests.test_clip_zero_percentile_falls_back_to_max(),
+    lambda _golden: w4pc_tests.test_w4pc_worked_example(),
 ]
 
 
