@@ -478,6 +478,12 @@ def bench_rows(device, pk, steps, warmup):
     wsp = torch.empty((cider.cider_workspace_bytes_mnk(M, N, K),), dtype=torch.uint8, device=device)
     ms = graph_time(lambda i: cider.cider_w4a8_linear_pg(x, p4s[i % n], s4, gs, y=ys[i % n], workspace=wsp), steps, warmup)
     record("w4a8_linear_pg", ms, 2.0 * M * N * K, N * K // 2 + s4.numel() * 4 + M * K * 2 + M * N * 2, gs=gs, M=M, N=N, K=K)
+    del p4s
+    # W4A8 with one scale per output channel, same shape
+    p4, s4 = cider.cider_pack_weight_int4_pc(torch.from_numpy(synth.weights(N, K, 3001)).to(device))
+    p4s = [p4] + [p4.roll(i, 0).contiguous() for i in range(1, n)]
+    ms = graph_time(lambda i: cider.cider_w4a8_linear_pc(x, p4s[i % n], s4, y=ys[i % n], workspace=wsp), steps, warmup)
+    record("w4a8_linear_pc", ms, 2.0 * M * N * K, N * K // 2 + N * 4 + M * K * 2 + M * N * 2, M=M, N=N, K=K)
     del p4s, ys
     # memory-bound producers
     for (M, K) in ((4096, 2560), (8192, 10240)):
@@ -539,7 +545,7 @@ ROW_CASES = {
     "pg64_m1": ("pg", 1, 2560, 10240, 64), "pg64_m4096": ("pg", 4096, 2560, 10240, 64),
     "pg128_m128": ("pg", 128, 2560, 10240, 128), "pg64_m128": ("pg", 128, 2560, 10240, 64),
     "pg64_m1024": ("pg", 1024, 2560, 10240, 64), 
-    "w4a8_m2048": ("w4", 2048, 12288, 4096, 64),
+    "w4a8_m2048": ("w4", 2048, 12288, 4096, 64), "w4a8pc_m2048": ("w4pc", 2048, 12288, 4096, 0),
     "stack_8b": ("stack", 2048, 0, 0, 0),
 }
 
@@ -566,6 +572,9 @@ def run_row(args):
     elif kind == "pg":
         w, s = cider.cider_quantize_weight_pg(W, gs)
         call = lambda y, ws_: cider.cider_w8a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)
+    elif kind == "w4pc":
+        w, s = cider.cider_pack_weight_int4_pc(W)
+        call = lambda y, ws_: cider.cider_w4a8_linear_pc(x, w, s, y=y, workspace=ws_)
     else:
         w, s = cider.cider_pack_weight_int4_pg(W, gs)
         call = lambda y, ws_: cider.cider_w4a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)

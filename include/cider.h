@@ -104,6 +104,12 @@ CIDER_API size_t cider_workspace_bytes(int64_t M, int64_t K);
  * least cider_workspace_bytes(M, K)) runs without splitting K. */
 CIDER_API size_t cider_workspace_bytes_mnk(int64_t M, int64_t N, int64_t K);
 
+/* Workspace of cider_w4a8_linear_pc, which runs on the tensor cores at every
+ * M: q [M][K] int8 and scale_x [M] fp32 (256-byte aligned) for any M >= 1,
+ * plus room for its split-K partial sums as in cider_workspace_bytes_mnk.
+ * Given only the first part, it runs without splitting K. */
+CIDER_API size_t cider_workspace_bytes_w4a8_pc(int64_t M, int64_t N, int64_t K);
+
 /* Calls with 1 <= M <= threshold use the fused small-M (decode-shaped) kernel;
  * larger M use quantize + the tcgen05 GEMM.  The threshold is process-wide;
  * 0 sends every call to the GEMM path.  Values above 16 are rejected.  The
@@ -164,6 +170,22 @@ CIDER_API cider_status_t cider_w4a8_linear_pg(const void* x, cider_dtype_t xdt, 
                                     int64_t gs, void* y, cider_dtype_t ydt,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* W4A8 linear, one scale per output channel (Cider README, table "量化",
+ * W4A8 weights symmetric INT4, zero point 8, "per-column"; table "模式" and
+ * section "Metal Kernel 流水线" for the on-chip INT4 -> INT8 unpack).
+ * y[m,n] = round(acc[m,n] * scale_x[m] * scale_w[n]) with acc the INT32 sum
+ * over all of K of the activation codes times the unpacked weights (nibble
+ * - 8).  w_packed: [N][K/2] bytes as described above (from
+ * cider_pack_weight_int4_pc); scale_w: [N] fp32.  Requires K % 32 == 0.
+ * Every M runs on the tensor cores (there is no separate decode kernel for
+ * this form), so the workspace is cider_workspace_bytes_w4a8_pc(M, N, K)
+ * (at least its q and scale_x part, even for small M).  Errors as
+ * cider_w4a8_linear_pg. */
+CIDER_API cider_status_t cider_w4a8_linear_pc(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
+                                    const uint8_t* w_packed, const float* scale_w, int64_t N,
+                                    void* y, cider_dtype_t ydt,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* W8A8 per-channel linear for callers that cannot allocate device memory.
  * The pages have no counterpart: this is an addition of this library.
  *
@@ -203,6 +225,9 @@ CIDER_API cider_status_t cider_w8a8_gemm_pg_q(const int8_t* q, const float* scal
 CIDER_API cider_status_t cider_w4a8_gemm_pg_q(const int8_t* q, const float* scale_x, int64_t M, int64_t K,
                                     const uint8_t* w_packed, const float* scale_w, int64_t N,
                                     int64_t gs, void* y, cider_dtype_t ydt, void* stream);
+CIDER_API cider_status_t cider_w4a8_gemm_pc_q(const int8_t* q, const float* scale_x, int64_t M, int64_t K,
+                                    const uint8_t* w_packed, const float* scale_w, int64_t N,
+                                    void* y, cider_dtype_t ydt, void* stream);
 
 /* ---- decoder-MLP producer ------------------------------------------------ */
 /* a = round_dt(silu(gate) * up) evaluated in fp32, then per-token quantized as
@@ -243,6 +268,10 @@ CIDER_API cider_status_t cider_quantize_weight_pg_clip(const float* W, int64_t N
 /* INT4 per group: scale_w[g][n] = max|W_group| / 7, q = clamp(round(W/scale), -8, 7),
  * packed as described above. */
 CIDER_API cider_status_t cider_pack_weight_int4_pg(const float* W, int64_t N, int64_t K, int64_t gs,
+                                         uint8_t* w_packed, float* scale_w, void* stream);
+/* INT4 per output channel: scale_w[n] = max_k |W[n,k]| / 7, q = clamp(round(W/scale), -8, 7),
+ * packed as described above; scale_w: [N].  Requires an even K. */
+CIDER_API cider_status_t cider_pack_weight_int4_pc(const float* W, int64_t N, int64_t K,
                                          uint8_t* w_packed, float* scale_w, void* stream);
 
 /* ---- test exports (stable, but not part of the operation's interface) ---- */

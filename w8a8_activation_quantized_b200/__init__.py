@@ -47,16 +47,20 @@ _SIGNATURES = {
     "cider_w8a16_mv_pc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_w8a8_linear_pg": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P, _SZ, _P]),
     "cider_w4a8_linear_pg": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P, _SZ, _P]),
+    "cider_w4a8_linear_pc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P, _SZ, _P]),
+    "cider_workspace_bytes_w4a8_pc": (_SZ, [_I64, _I64, _I64]),
     "cider_w8a8_linear_pc_noalloc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_w8a8_gemm_pc_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_w8a8_gemm_pg_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P]),
     "cider_w4a8_gemm_pg_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P]),
+    "cider_w4a8_gemm_pc_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_silu_mul_quantize": (_INT, [_P, _P, _INT, _I64, _I64, _P, _P, _P, _P]),
     "cider_quantize_weight_pc": (_INT, [_P, _I64, _I64, _P, _P, _P]),
     "cider_quantize_weight_pg": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "cider_quantize_weight_pc_clip": (_INT, [_P, _I64, _I64, ctypes.c_double, _P, _P, _P]),
     "cider_quantize_weight_pg_clip": (_INT, [_P, _I64, _I64, _I64, ctypes.c_double, _P, _P, _P]),
     "cider_pack_weight_int4_pg": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "cider_pack_weight_int4_pc": (_INT, [_P, _I64, _I64, _P, _P, _P]),
     "cider_test_gemm_i32": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P]),
     "cider_test_gemm_i32_grouped": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _P, _P]),
     "cider_test_unpack_int4": (_INT, [_P, _I64, _I64, _P, _P]),
@@ -123,6 +127,10 @@ def cider_workspace_bytes(M: int, K: int) -> int:
 
 def cider_workspace_bytes_mnk(M: int, N: int, K: int) -> int:
     return int(lib().cider_workspace_bytes_mnk(M, N, K))
+
+
+def cider_workspace_bytes_w4a8_pc(M: int, N: int, K: int) -> int:
+    return int(lib().cider_workspace_bytes_w4a8_pc(M, N, K))
 
 
 def cider_set_small_m_threshold(threshold: int):
@@ -208,6 +216,23 @@ def cider_w4a8_linear_pg(x, w_packed, scale_w, gs, y=None, out_dtype=None, works
     return y
 
 
+def cider_w4a8_linear_pc(x, w_packed, scale_w, y=None, out_dtype=None, workspace=None, stream=None):
+    """W4A8 linear with one scale per output channel: w_packed uint8 [N, K/2],
+    scale_w fp32 [N]."""
+    _contig(x, "x"), _contig(w_packed, "w_packed")
+    M, K = x.shape
+    N = w_packed.shape[0]
+    y = _out(y, M, N, out_dtype or x.dtype, x.device)
+    if workspace is None:
+        need = cider_workspace_bytes_w4a8_pc(M, N, K)
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=x.device)
+    ws, ws_bytes = workspace, workspace.numel() * workspace.element_size()
+    _check("cider_w4a8_linear_pc", lib().cider_w4a8_linear_pc(
+        _ptr(x), _DT[x.dtype], M, K, _ptr(w_packed), _ptr(scale_w), N, _ptr(y), _DT[y.dtype],
+        _ptr(ws), ws_bytes, _stream(stream, x.device)))
+    return y
+
+
 def cider_w8a8_linear_pc_noalloc(x, w, scale_w, y=None, out_dtype=None, stream=None):
     """The per-channel linear without a workspace, for callers that cannot
     allocate device memory: its scratch is a fixed 32 MiB array inside the
@@ -249,6 +274,16 @@ def cider_w4a8_gemm_pg_q(q, scale_x, w_packed, scale_w, gs, y=None, out_dtype=to
     y = _out(y, M, N, out_dtype, q.device)
     _check("cider_w4a8_gemm_pg_q", lib().cider_w4a8_gemm_pg_q(
         _ptr(q), _ptr(scale_x), M, K, _ptr(w_packed), _ptr(scale_w), N, gs, _ptr(y), _DT[y.dtype],
+        _stream(stream, q.device)))
+    return y
+
+
+def cider_w4a8_gemm_pc_q(q, scale_x, w_packed, scale_w, y=None, out_dtype=torch.float16, stream=None):
+    M, K = q.shape
+    N = w_packed.shape[0]
+    y = _out(y, M, N, out_dtype, q.device)
+    _check("cider_w4a8_gemm_pc_q", lib().cider_w4a8_gemm_pc_q(
+        _ptr(q), _ptr(scale_x), M, K, _ptr(w_packed), _ptr(scale_w), N, _ptr(y), _DT[y.dtype],
         _stream(stream, q.device)))
     return y
 
@@ -315,6 +350,16 @@ def cider_pack_weight_int4_pg(W, gs, stream=None):
     s = torch.empty((K // gs, N), dtype=torch.float32, device=W.device)
     _check("cider_pack_weight_int4_pg", lib().cider_pack_weight_int4_pg(
         _ptr(_contig(W, "W")), N, K, gs, _ptr(p), _ptr(s), _stream(stream, W.device)))
+    return p, s
+
+
+def cider_pack_weight_int4_pc(W, stream=None):
+    """W fp32 [N, K] -> (packed uint8 [N, K/2], scale_w fp32 [N])."""
+    N, K = W.shape
+    p = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    s = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _check("cider_pack_weight_int4_pc", lib().cider_pack_weight_int4_pc(
+        _ptr(_contig(W, "W")), N, K, _ptr(p), _ptr(s), _stream(stream, W.device)))
     return p, s
 
 

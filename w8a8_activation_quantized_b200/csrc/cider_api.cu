@@ -102,6 +102,12 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // The fused small-M kernel keeps the M code rows in shared memory and at most
 // 8 passes of 512 weights per warp in registers (K <= 32768).
+// q [M][K] int8 and scale_x [M] fp32 of the quantize + tensor-core path
+size_t tensor_path_bytes(int64_t M, int64_t K) {
+    if (M <= 0 || K <= 0) return 0;
+    return align256(static_cast<size_t>(M) * K) + align256(static_cast<size_t>(M) * 4);
+}
+
 bool small_m_path(int64_t M, int64_t K) {
     return M >= 1 && M <= g_small_m_threshold.load() && M * K <= kSmallSmemLimit && K <= kSmallMaxK;
 }
@@ -128,6 +134,14 @@ cider_status_t check_gs(int64_t K, int64_t gs, bool w4) {
     if (gs != 64 && gs != 128) return fail(CIDER_ERR_INVALID_ARG, "gs = %lld must be 64 or 128", (long long)gs);
     if (K % gs) return fail(CIDER_ERR_INVALID_ARG, "gs = %lld must divide K = %lld", (long long)gs, (long long)K);
     if (w4 && K % 32) return fail(CIDER_ERR_INVALID_ARG, "W4A8 needs K %% 32 == 0 (K = %lld)", (long long)K);
+    return CIDER_OK;
+}
+
+// gs and K rules of a linear mode: per group needs gs in {64, 128} dividing K;
+// packed INT4 weights need K % 32 == 0 (16-byte rows of K/2 bytes).
+cider_status_t check_mode_k(int mode, int64_t K, int64_t gs) {
+    if (mode == kModePG || mode == kModeW4) return check_gs(K, gs, mode == kModeW4);
+    if (mode == kModeW4PC && K % 32) return fail(CIDER_ERR_INVALID_ARG, "W4A8 needs K %% 32 == 0 (K = %lld)", (long long)K);
     return CIDER_OK;
 }
 
@@ -224,11 +238,12 @@ cider_status_t linear(int mode, const void* x, int xdt, int64_t M, int64_t K, co
     t_last_error[0] = '\0';
     cider_status_t s = check_common(x, M, K, w, sw, N, y, xdt, ydt);
     if (s != CIDER_OK) return s;
-    if (mode != kModePC && (s = check_gs(K, gs, mode == kModeW4)) != CIDER_OK) return s;
+    if ((s = check_mode_k(mode, K, gs)) != CIDER_OK) return s;
     if (M == 0) return CIDER_OK;
     const size_t ysz = static_cast<size_t>(M) * N * 2;
-    const size_t wbytes = mode == kModeW4 ? static_cast<size_t>(N) * K / 2 : static_cast<size_t>(N) * K;
-    const size_t swbytes = mode == kModePC ? N * 4 : static_cast<size_t>(K / gs) * N * 4;
+    const bool packed = mode == kModeW4 || mode == kModeW4PC;
+    const size_t wbytes = packed ? static_cast<size_t>(N) * K / 2 : static_cast<size_t>(N) * K;
+    const size_t swbytes = (mode == kModePC || mode == kModeW4PC) ? N * 4 : static_cast<size_t>(K / gs) * N * 4;
     const Range ry = rng(y, ysz);
     if (overlap(ry, rng(x, static_cast<size_t>(M) * K * 2)) || overlap(ry, rng(w, wbytes)) ||
         overlap(ry, rng(sw, swbytes)))
@@ -236,13 +251,13 @@ cider_status_t linear(int mode, const void* x, int xdt, int64_t M, int64_t K, co
     DeviceInfo* d = nullptr;
     if ((s = device_info(&d)) != CIDER_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (small_m_path(M, K)) {
+    if (mode != kModeW4PC && small_m_path(M, K)) {  // per-channel INT4: tensor-core path at every M
         cudaError_t e = launch_small_m(mode, x, xdt, static_cast<int>(M), static_cast<int>(K), w, sw,
                                        static_cast<int>(N), static_cast<int>(gs), y, ydt, d->num_sms, st);
         if (e != cudaSuccess) return cuda_fail(e, "small-M kernel launch");
         return CIDER_OK;
     }
-    const size_t need = cider_workspace_bytes(M, K);
+    const size_t need = mode == kModeW4PC ? tensor_path_bytes(M, K) : cider_workspace_bytes(M, K);
     if (!ws || ws_bytes < need)
         return fail(CIDER_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, ws ? ws_bytes : 0);
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(CIDER_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
@@ -273,7 +288,7 @@ cider_status_t gemm_q(int mode, const int8_t* q, const float* sx, int64_t M, int
     t_last_error[0] = '\0';
     cider_status_t s = check_common(q, M, K, w, sw, N, y, CIDER_F16, ydt);
     if (s != CIDER_OK) return s;
-    if (mode != kModePC && (s = check_gs(K, gs, mode == kModeW4)) != CIDER_OK) return s;
+    if ((s = check_mode_k(mode, K, gs)) != CIDER_OK) return s;
     if (M == 0) return CIDER_OK;
     if (!sx || (reinterpret_cast<uintptr_t>(sx) & 3u)) return fail(CIDER_ERR_INVALID_ARG, "scale_x must be non-NULL and 4-byte aligned");
     const Range ry = rng(y, static_cast<size_t>(M) * N * 2);
@@ -366,7 +381,15 @@ cider_status_t cider_device_status(void* stream) {
 
 size_t cider_workspace_bytes(int64_t M, int64_t K) {
     if (M <= 0 || K <= 0 || small_m_path(M, K)) return 0;
-    return align256(static_cast<size_t>(M) * K) + align256(static_cast<size_t>(M) * 4);
+    return tensor_path_bytes(M, K);
+}
+
+size_t cider_workspace_bytes_w4a8_pc(int64_t M, int64_t N, int64_t K) {
+    const size_t need = tensor_path_bytes(M, K);
+    if (need == 0 || N <= 0) return need;
+    DeviceInfo* d = nullptr;
+    if (device_info(&d) != CIDER_OK) return need;
+    return need + part_bytes(grouped_split_plan(M, N, K, d->num_sms));
 }
 
 size_t cider_workspace_bytes_mnk(int64_t M, int64_t N, int64_t K) {
@@ -459,6 +482,12 @@ cider_status_t cider_w4a8_linear_pg(const void* x, cider_dtype_t xdt, int64_t M,
     return linear(kModeW4, x, xdt, M, K, w_packed, scale_w, N, gs, y, ydt, workspace, workspace_bytes, stream);
 }
 
+cider_status_t cider_w4a8_linear_pc(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, const uint8_t* w_packed,
+                                    const float* scale_w, int64_t N, void* y, cider_dtype_t ydt, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+    return linear(kModeW4PC, x, xdt, M, K, w_packed, scale_w, N, 0, y, ydt, workspace, workspace_bytes, stream);
+}
+
 cider_status_t cider_w8a8_gemm_pc_q(const int8_t* q, const float* scale_x, int64_t M, int64_t K, const int8_t* w,
                                     const float* scale_w, int64_t N, void* y, cider_dtype_t ydt, void* stream) {
     return gemm_q(kModePC, q, scale_x, M, K, w, scale_w, N, 0, y, ydt, stream);
@@ -474,6 +503,11 @@ cider_status_t cider_w4a8_gemm_pg_q(const int8_t* q, const float* scale_x, int64
                                     const uint8_t* w_packed, const float* scale_w, int64_t N, int64_t gs,
                                     void* y, cider_dtype_t ydt, void* stream) {
     return gemm_q(kModeW4, q, scale_x, M, K, w_packed, scale_w, N, gs, y, ydt, stream);
+}
+
+cider_status_t cider_w4a8_gemm_pc_q(const int8_t* q, const float* scale_x, int64_t M, int64_t K, const uint8_t* w_packed,
+                                    const float* scale_w, int64_t N, void* y, cider_dtype_t ydt, void* stream) {
+    return gemm_q(kModeW4PC, q, scale_x, M, K, w_packed, scale_w, N, 0, y, ydt, stream);
 }
 
 cider_status_t cider_silu_mul_quantize(const void* gate, const void* up, cider_dtype_t dt, int64_t M, int64_t F,
@@ -501,10 +535,11 @@ static cider_status_t quantize_weight(int mode, const float* W, int64_t N, int64
     t_last_error[0] = '\0';
     if (N < 1 || K < 1) return fail(CIDER_ERR_INVALID_ARG, "N, K >= 1 required");
     if (N > INT32_MAX || K > kMaxK) return fail(CIDER_ERR_INVALID_ARG, "size out of range");
-    if (mode != 0) {
+    if (mode == 1 || mode == 2) {
         cider_status_t s = check_gs(K, gs, mode == 2);
         if (s != CIDER_OK) return s;
     }
+    if (mode == 3 && K % 2) return fail(CIDER_ERR_INVALID_ARG, "INT4 packing needs an even K (K = %lld)", (long long)K);
     if (!W || !out || !sw) return fail(CIDER_ERR_INVALID_ARG, "NULL pointer");
     DeviceInfo* d = nullptr;
     cider_status_t s = device_info(&d);
@@ -566,6 +601,11 @@ cider_status_t cider_quantize_weight_pg(const float* W, int64_t N, int64_t K, in
 cider_status_t cider_pack_weight_int4_pg(const float* W, int64_t N, int64_t K, int64_t gs, uint8_t* w_packed,
                                          float* scale_w, void* stream) {
     return quantize_weight(2, W, N, K, gs, w_packed, scale_w, stream);
+}
+
+cider_status_t cider_pack_weight_int4_pc(const float* W, int64_t N, int64_t K, uint8_t* w_packed, float* scale_w,
+                                         void* stream) {
+    return quantize_weight(3, W, N, K, 0, w_packed, scale_w, stream);
 }
 
 cider_status_t cider_test_gemm_i32(const int8_t* q, const int8_t* w, int64_t M, int64_t N, int64_t K,

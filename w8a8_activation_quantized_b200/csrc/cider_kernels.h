@@ -19,6 +19,7 @@ enum : int {
     kModeW4 = 2,    // per-group epilogue, INT4 packed weights unpacked on chip
     kModeI32 = 3,   // test: store the INT32 accumulator
     kModeI32G = 4,  // test: store every per-group INT32 partial
+    kModeW4PC = 5,  // per-channel epilogue, INT4 packed weights unpacked on chip
 };
 
 // Kernel variants of the per-channel GEMM (the grouped modes always use the
@@ -73,7 +74,8 @@ cudaError_t launch_quantize_act(const void* x, int xdt, int64_t M, int K, int8_t
                                 cudaStream_t st);
 cudaError_t launch_silu_mul_quantize(const void* g, const void* u, int dt, int64_t M, int F,
                                      int8_t* q, float* sx, void* a_out, cudaStream_t st);
-// mode 0: per channel (out = int8 [N][K]); 1: per group int8; 2: per group int4 packed
+// mode 0: per channel (out = int8 [N][K]); 1: per group int8; 2: per group int4 packed;
+// 3: per channel int4 packed
 cudaError_t launch_quantize_weight(int mode, const float* W, int64_t N, int K, int gs, void* out,
                                    float* sw, cudaStream_t st);
 // percentile-clipped weights: gs = 0 per channel, else per group of gs (64 or 128);

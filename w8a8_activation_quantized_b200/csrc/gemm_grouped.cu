@@ -39,6 +39,12 @@
 // per partial; these do not overlap, which puts the floor near 384 cycles
 // per group per SM sub-partition -- the epilogue, not the tensor core, bounds
 // this kernel at gs = 64 and gs = 128.
+// W4A8 with per-output-channel scales (mode kModeW4PC; Cider README, table
+// "量化": symmetric INT4, zero point 8, per column) runs the same producer and
+// converter warps, but the MMA warp accumulates a whole work unit into one
+// TMEM buffer (no bias, one hand-off per tile) and the epilogue applies
+// acc * scale_w[n] once; scale_x is applied by the same store (or split-K
+// reduce) as the per-group modes.
 // Every mbarrier wait is bounded.
 #include <algorithm>
 
@@ -48,7 +54,8 @@ namespace cider {
 
 template <int MODE>
 struct GroupedCfg {
-    static constexpr bool W4 = (MODE == kModeW4);
+    static constexpr bool W4 = (MODE == kModeW4 || MODE == kModeW4PC);
+    static constexpr bool PC = (MODE == kModeW4PC);  // one scale per output channel
     static constexpr int BM = 128;
     static constexpr int BN = 128;
     static constexpr int EPI_WARPS = 8;
@@ -115,8 +122,9 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nunits = num_units(p);
-    const int G = p.K / p.gs;
-    const int gpk = kBK / p.gs;  // groups per k-block: 1 or 2
+    // per-channel mode: the unit's "groups" are its k-blocks
+    const int G = C::PC ? p.num_k_blocks : p.K / p.gs;
+    const int gpk = C::PC ? 1 : kBK / p.gs;  // groups per k-block: 1 or 2
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -188,9 +196,33 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
             uint32_t phase = 0;
             uint32_t acc_i = 0;  // partial-buffer uses so far
             bool ok = true;
-            const int steps = p.gs / kUmmaK;
+            const int steps = C::PC ? 0 : p.gs / kUmmaK;
             for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
                 const GroupUnit w = group_unit(p, u, G, gpk);
+                if constexpr (C::PC) {
+                    // the unit's k-blocks accumulate into one buffer: one hand-off per unit
+                    const uint32_t b = acc_i % NB;
+                    if (!mbar_wait(&acce[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d = tmem_base + b * BN;
+                    for (int kb = w.kb0; kb < w.kb1 && ok; ++kb) {
+                        if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
+                        if (!mbar_wait(&conv[stage], phase, p.status, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
+                        const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
+#pragma unroll
+                        for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+                            umma_i8(d, adesc + (kk * kUmmaK >> 4), bdesc + (kk * kUmmaK >> 4), idesc,
+                                    (kb > w.kb0 || kk > 0) ? 1u : 0u);
+                        umma_commit(&empty[stage]);
+                        if (++stage == S) { stage = 0; phase ^= 1u; }
+                    }
+                    if (!ok) break;
+                    umma_commit(&accf[b]);
+                    ++acc_i;
+                    continue;
+                }
                 int g = w.g0;
                 for (int kb = w.kb0; kb < w.kb1 && ok; ++kb) {
                     if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
@@ -255,7 +287,8 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
                 pf_unit();
             }
         };
-        for (int i = 0; i < kScaleSlots - 1; ++i) prefetch();
+        if (!C::PC)
+            for (int i = 0; i < kScaleSlots - 1; ++i) prefetch();
 
         const uint64_t neg_bias2 = pack_u32x2(__float_as_uint(-12582912.0f), __float_as_uint(-12582912.0f));
         uint32_t acc_i = 0, nstore = 0;
@@ -273,6 +306,40 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
             // the next step (crossing into the next group) is in flight while the
             // current step is rescaled, and the preset restore completes behind the
             // last step.
+            if constexpr (C::PC) {
+                // sum2 = acc * scale_w[n] for this warp's 64 columns, read once per unit
+                const uint32_t b = acc_i % NB;
+                if (!mbar_wait(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + lane_addr + b * BN + half * C::EPI_COLS;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(taddr + 16 * c, r);
+                    tmem_ld_wait();
+                    const int n0 = nw + 16 * c;
+                    float ws[16];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        // N % 8 == 0: a group of four columns is either all inside or all outside
+                        const float4 v4 = n0 + 4 * q4 < p.N ? __ldg(reinterpret_cast<const float4*>(p.sw + n0 + 4 * q4))
+                                                            : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        ws[4 * q4] = v4.x;
+                        ws[4 * q4 + 1] = v4.y;
+                        ws[4 * q4 + 2] = v4.z;
+                        ws[4 * q4 + 3] = v4.w;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        sum2[8 * c + j] = pack_u32x2(
+                            __float_as_uint(__int2float_rn(static_cast<int32_t>(r[2 * j])) * ws[2 * j]),
+                            __float_as_uint(__int2float_rn(static_cast<int32_t>(r[2 * j + 1])) * ws[2 * j + 1]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_relaxed(&acce[b]);  // buffer b read out
+                ++acc_i;
+            } else {
             uint32_t rr[2][16];
             {
                 const uint32_t b0 = acc_i % NB;
@@ -314,6 +381,7 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
                 __syncwarp();  // every lane has read the scale slot before it is refilled
                 ++acc_i;
             }
+            }  // per-group modes
             if (!ok) break;
             if (MODE != kModeI32G && w.slot >= 0) {
                 // this piece's fp32 sums: four 32 x 16 boxes into its tile-local slot
@@ -513,6 +581,7 @@ cudaError_t launch_gemm_grouped(const GemmLaunch& L, cudaStream_t st) {
         case kModePG: return bf ? launch_grouped_t<kModePG, __nv_bfloat16>(L, st) : launch_grouped_t<kModePG, __half>(L, st);
         case kModeW4: return bf ? launch_grouped_t<kModeW4, __nv_bfloat16>(L, st) : launch_grouped_t<kModeW4, __half>(L, st);
         case kModeI32G: return launch_grouped_t<kModeI32G, __half>(L, st);
+        case kModeW4PC: return bf ? launch_grouped_t<kModeW4PC, __nv_bfloat16>(L, st) : launch_grouped_t<kModeW4PC, __half>(L, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -624,7 +624,8 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t st) {
         case kModeI32: return launch_gemm_mode<kModeI32, __half>(L, st);
         case kModePG:
         case kModeW4:
-        case kModeI32G: return launch_gemm_grouped(L, st);
+        case kModeI32G:
+        case kModeW4PC: return launch_gemm_grouped(L, st);
         default: return cudaErrorInvalidValue;
     }
 }

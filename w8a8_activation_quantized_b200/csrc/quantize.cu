@@ -296,6 +296,35 @@ __global__ void __launch_bounds__(256) k_quantize_weight_pc(const float* __restr
     for (int k = threadIdx.x; k < K; k += 256) w[n * K + k] = static_cast<int8_t>(quant_code(wr[k], s));
 }
 
+// INT4 per output channel: one CTA per row; scale = max|W[n,:]| / 7, codes
+// clamp(round(W / scale), -8, 7) stored as q + 8, even k in the low nibble.
+__global__ void __launch_bounds__(256) k_pack_weight_int4_pc(const float* __restrict__ W, int K,
+                                                             uint8_t* __restrict__ out, float* __restrict__ sw) {
+    __shared__ float red[8];
+    pdl_wait();
+    pdl_trigger();
+    const int64_t n = blockIdx.x;
+    const float* wr = W + n * K;
+    float amax = 0.0f;
+    for (int k = threadIdx.x; k < K; k += 256) amax = fmaxf(amax, fabsf(wr[k]));
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+    const float s = __fdiv_rn(amax, 7.0f);
+    if (threadIdx.x == 0) sw[n] = s;
+    uint8_t* p = out + n * (K / 2);
+    for (int j = threadIdx.x; j < K / 2; j += 256) {
+        int c0 = 0, c1 = 0;
+        if (s != 0.0f) {
+            c0 = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(wr[2 * j], s)), -8.0f), 7.0f));
+            c1 = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(wr[2 * j + 1], s)), -8.0f), 7.0f));
+        }
+        p[j] = static_cast<uint8_t>((c0 + 8) | ((c1 + 8) << 4));
+    }
+}
+
 // Per group (INT8 or INT4): one warp per (row n, group g); scales group-major [G][N].
 template <bool INT4>
 __global__ void __launch_bounds__(256) k_quantize_weight_group(const float* __restrict__ W,
@@ -336,6 +365,8 @@ cudaError_t launch_quantize_weight(int mode, const float* W, int64_t N, int K, i
                                    float* sw, cudaStream_t st) {
     if (mode == 0)
         return launch_pdl(k_quantize_weight_pc, static_cast<unsigned>(N), 256, 0, st, W, K, static_cast<int8_t*>(out), sw);
+    if (mode == 3)
+        return launch_pdl(k_pack_weight_int4_pc, static_cast<unsigned>(N), 256, 0, st, W, K, static_cast<uint8_t*>(out), sw);
     const int64_t items = N * (K / gs);
     const unsigned grid = static_cast<unsigned>((items + 7) / 8);
     if (mode == 1) return launch_pdl(k_quantize_weight_group<false>, grid, 256, 0, st, W, N, K, gs, out, sw);
