@@ -513,6 +513,23 @@ def bench_rows(device, pk, steps, warmup):
             record("quantize_weight_pg_clip", ms, 0, N * K * 5 + N * (K // gs) * 4, gs=gs, N=N, K=K,
                    clip_percentile=99.9)
         del Ws
+    # decode attention, the pages' SDPA table configurations (D = 128, fp16)
+    for (H_kv, N) in ((32, 4096), (8, 4096), (4, 4096), (32, 32768), (8, 32768), (4, 32768)):
+        H_q, D = 32, 128
+        kv_bytes = 2 * H_kv * N * D * 2
+        n = rotating(kv_bytes)
+        g = torch.Generator(device=device)
+        g.manual_seed(5000 + H_kv + N)
+        qs = torch.randn((H_q, D), generator=g, device=device).half()
+        ks = [torch.randn((H_kv, N, D), generator=g, device=device).half() for _ in range(n)]
+        vs = [torch.randn((H_kv, N, D), generator=g, device=device).half() for _ in range(n)]
+        os_ = torch.empty((H_q, D), dtype=torch.float16, device=device)
+        wsd = torch.empty((max(16, cider.cider_sdpa_decode_workspace_bytes(H_q, H_kv, N, D)),), dtype=torch.uint8,
+                          device=device)
+        ms = graph_time(lambda i: cider.cider_sdpa_decode(qs, ks[i % n], vs[i % n], out=os_, workspace=wsd),
+                        steps, warmup)
+        record("sdpa_decode", ms, 0, kv_bytes + 2 * H_q * D * 2, H_q=H_q, H_kv=H_kv, N=N, D=D)
+        del ks, vs
     out.append(bench_stack(device, pk, steps=max(3, steps // 20), warmup=warmup))
     return out
 

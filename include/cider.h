@@ -274,6 +274,22 @@ CIDER_API cider_status_t cider_pack_weight_int4_pg(const float* W, int64_t N, in
 CIDER_API cider_status_t cider_pack_weight_int4_pc(const float* W, int64_t N, int64_t K,
                                          uint8_t* w_packed, float* scale_w, void* stream);
 
+/* ---- decode attention (Cider README, section "优化 SDPA（解码注意力）") --------
+ * Scaled dot-product attention for one query token per head with no mask:
+ * for query head h and its KV head g = h / (H_q / H_kv),
+ *   out[h] = sum_j softmax_j(q[h] . K[g][j] / sqrt(D)) V[g][j].
+ * q [H_q][D], K and V [H_kv][N][D] (head-major cache), out [H_q][D]; all in
+ * dt (fp16 or bf16), device memory owned by the caller, 16-byte aligned.
+ * D must be 128; H_kv must divide H_q; 1 <= N < 2^31.  The sequence is cut
+ * into chunks whose fp32 partial results go to the workspace
+ * (cider_sdpa_decode_workspace_bytes; it depends on the device's SM count);
+ * a second kernel merges them.  Errors: CIDER_ERR_INVALID_ARG for the shape
+ * rules, a short workspace, misalignment or out overlapping an input. */
+CIDER_API size_t cider_sdpa_decode_workspace_bytes(int64_t H_q, int64_t H_kv, int64_t N, int64_t D);
+CIDER_API cider_status_t cider_sdpa_decode(const void* q, const void* k, const void* v, cider_dtype_t dt,
+                                 int64_t H_q, int64_t H_kv, int64_t N, int64_t D, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- test exports (stable, but not part of the operation's interface) ---- */
 /* The tcgen05 GEMM with an INT32 store epilogue: acc[m][n] = sum_k q[m,k]*w[n,k]. */
 CIDER_API cider_status_t cider_test_gemm_i32(const int8_t* q, const int8_t* w, int64_t M, int64_t N,

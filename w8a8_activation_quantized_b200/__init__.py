@@ -49,6 +49,8 @@ _SIGNATURES = {
     "cider_w4a8_linear_pg": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P, _SZ, _P]),
     "cider_w4a8_linear_pc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P, _SZ, _P]),
     "cider_workspace_bytes_w4a8_pc": (_SZ, [_I64, _I64, _I64]),
+    "cider_sdpa_decode_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64]),
+    "cider_sdpa_decode": (_INT, [_P, _P, _P, _INT, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "cider_w8a8_linear_pc_noalloc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_w8a8_gemm_pc_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_w8a8_gemm_pg_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P]),
@@ -361,6 +363,27 @@ def cider_pack_weight_int4_pc(W, stream=None):
     _check("cider_pack_weight_int4_pc", lib().cider_pack_weight_int4_pc(
         _ptr(_contig(W, "W")), N, K, _ptr(p), _ptr(s), _stream(stream, W.device)))
     return p, s
+
+
+def cider_sdpa_decode_workspace_bytes(H_q: int, H_kv: int, N: int, D: int = 128) -> int:
+    return int(lib().cider_sdpa_decode_workspace_bytes(H_q, H_kv, N, D))
+
+
+def cider_sdpa_decode(q, k, v, out=None, workspace=None, stream=None):
+    """Decode attention: q [H_q, D], k and v [H_kv, N, D] (fp16 or bf16, D = 128)
+    -> out [H_q, D]: softmax(q . k / sqrt(D)) v per head, H_q / H_kv query
+    heads per KV head."""
+    _contig(q, "q"), _contig(k, "k"), _contig(v, "v")
+    H_q, D = q.shape
+    H_kv, N, _ = k.shape
+    out = torch.empty((H_q, D), dtype=q.dtype, device=q.device) if out is None else out
+    if workspace is None:
+        need = int(lib().cider_sdpa_decode_workspace_bytes(H_q, H_kv, N, D))
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=q.device)
+    _check("cider_sdpa_decode", lib().cider_sdpa_decode(
+        _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], H_q, H_kv, N, D, _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream, q.device)))
+    return out
 
 
 # ---- test exports ---------------------------------------------------------------

@@ -13,6 +13,7 @@
 
 #include "../../include/cider.h"
 #include "cider_kernels.h"
+#include "sdpa_decode.h"
 
 namespace cider {
 
@@ -606,6 +607,50 @@ cider_status_t cider_pack_weight_int4_pg(const float* W, int64_t N, int64_t K, i
 cider_status_t cider_pack_weight_int4_pc(const float* W, int64_t N, int64_t K, uint8_t* w_packed, float* scale_w,
                                          void* stream) {
     return quantize_weight(3, W, N, K, 0, w_packed, scale_w, stream);
+}
+
+// ---- decode attention ---------------------------------------------------------
+static cider_status_t sdpa_check(int64_t H_q, int64_t H_kv, int64_t N, int64_t D) {
+    if (D != kSdpaD) return fail(CIDER_ERR_INVALID_ARG, "D = %lld: the decode-attention kernels take D = 128", (long long)D);
+    if (H_q < 1 || H_kv < 1 || H_q % H_kv)
+        return fail(CIDER_ERR_INVALID_ARG, "H_q = %lld must be a positive multiple of H_kv = %lld", (long long)H_q, (long long)H_kv);
+    if (H_q > 65535) return fail(CIDER_ERR_INVALID_ARG, "H_q = %lld exceeds 65535", (long long)H_q);
+    if (N < 1 || N > INT32_MAX) return fail(CIDER_ERR_INVALID_ARG, "N = %lld must lie in [1, 2^31)", (long long)N);
+    return CIDER_OK;
+}
+
+size_t cider_sdpa_decode_workspace_bytes(int64_t H_q, int64_t H_kv, int64_t N, int64_t D) {
+    if (sdpa_check(H_q, H_kv, N, D) != CIDER_OK) return 0;
+    DeviceInfo* d = nullptr;
+    if (device_info(&d) != CIDER_OK) return 0;
+    return sdpa_part_bytes(H_q, sdpa_plan(H_q, H_kv, N, d->num_sms));
+}
+
+cider_status_t cider_sdpa_decode(const void* q, const void* k, const void* v, cider_dtype_t dt, int64_t H_q,
+                                 int64_t H_kv, int64_t N, int64_t D, void* out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    t_last_error[0] = '\0';
+    cider_status_t s = sdpa_check(H_q, H_kv, N, D);
+    if (s != CIDER_OK) return s;
+    if (dt != CIDER_F16 && dt != CIDER_BF16) return fail(CIDER_ERR_INVALID_ARG, "dtype %d unknown", (int)dt);
+    if (!q || !k || !v || !out || !workspace) return fail(CIDER_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+        return fail(CIDER_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    DeviceInfo* d = nullptr;
+    if ((s = device_info(&d)) != CIDER_OK) return s;
+    const SdpaPlan plan = sdpa_plan(H_q, H_kv, N, d->num_sms);
+    const size_t need = sdpa_part_bytes(H_q, plan);
+    if (workspace_bytes < need)
+        return fail(CIDER_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes);
+    const size_t kv = static_cast<size_t>(H_kv) * N * D * 2;
+    const Range ro = rng(out, static_cast<size_t>(H_q) * D * 2);
+    if (overlap(ro, rng(q, static_cast<size_t>(H_q) * D * 2)) || overlap(ro, rng(k, kv)) || overlap(ro, rng(v, kv)) ||
+        overlap(ro, rng(workspace, need)))
+        return fail(CIDER_ERR_INVALID_ARG, "out overlaps an input or the workspace");
+    cudaError_t e = launch_sdpa_decode(q, k, v, dt == CIDER_BF16 ? 1 : 0, static_cast<int>(H_q), static_cast<int>(H_kv),
+                                       static_cast<int>(N), plan, static_cast<float*>(workspace), out,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "decode-attention launch");
 }
 
 cider_status_t cider_test_gemm_i32(const int8_t* q, const int8_t* w, int64_t M, int64_t N, int64_t K,

@@ -1,0 +1,260 @@
+// sdpa_decode.cu -- decode attention: scaled dot-product attention for one
+// query token per head, no mask, several query heads per KV head.
+//
+// What it computes (Cider README, section "优化 SDPA（解码注意力）"): for query
+// head h and its KV head g = h / (H_q / H_kv),
+//   out_h = sum_j softmax_j(q_h . k_{g,j} / sqrt(D)) v_{g,j},   D = 128,
+// with q [H_q][D], K and V [H_kv][N][D] (head-major cache) in fp16 or bf16,
+// out [H_q][D] in the same format.
+//
+// The pages' three techniques, B200 form:
+//  * one CTA serves a tile of up to four query heads of one KV group, so the
+//    group's K and V stream from HBM once per tile (the pages' contiguous-chunk
+//    GQA scheduling; four heads per thread is their register tiling);
+//  * the sequence is cut into chunks, one CTA per (chunk, KV head, head tile),
+//    about four CTAs per SM, and a second kernel merges the chunks (their
+//    two-pass split of the KV sequence);
+//  * inside a CTA, each half-warp streams every 16th key of the chunk: lane l
+//    holds dims 8l .. 8l+7 of the row (one 16-byte load of K and of V), the
+//    score is a 4-step shuffle reduction within the half-warp, and the
+//    softmax runs online in the log2 domain (q pre-scaled by log2(e)/sqrt(D)).
+// Partial results are fp32: the unnormalised output, the running maximum and
+// the running sum of exponentials, per (head, chunk).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cmath>
+#include <type_traits>
+
+#include "cider_device.cuh"
+#include "cider_kernels.h"
+#include "sdpa_decode.h"
+
+namespace cider {
+namespace {
+
+constexpr int kSdpaThreads = 256;  // 8 warps = 16 half-warp key streams
+constexpr int kStreams = kSdpaThreads / 16;
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&f)[8]) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 t;
+        if constexpr (sizeof(T) == 2 && std::is_same<T, __half>::value)
+            t = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+        else
+            t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+// Merge online-softmax state (m2, l2, a2) into (m, l, a); m = -inf means empty.
+template <int ND>
+__device__ __forceinline__ void merge_state(float& m, float& l, float (&a)[ND], float m2, float l2, const float (&a2)[ND]) {
+    const float M = fmaxf(m, m2);
+    if (M == -INFINITY) return;  // both empty
+    const float s1 = exp2f(m - M), s2 = exp2f(m2 - M);
+    l = l * s1 + l2 * s2;
+#pragma unroll
+    for (int d = 0; d < ND; ++d) a[d] = a[d] * s1 + a2[d] * s2;
+    m = M;
+}
+
+// One CTA: KV head hk, head tile `tile` (query heads h0 .. h0+TH-1), chunk c.
+template <int TH, typename T>
+__global__ void __launch_bounds__(kSdpaThreads) k_sdpa_decode_split(const T* __restrict__ q, const T* __restrict__ k,
+                                                                     const T* __restrict__ v, int G, int tiles, int N,
+                                                                     int chunk, int chunks, float qscale,
+                                                                     float* __restrict__ part) {
+    constexpr int D = kSdpaD;
+    __shared__ float s_m[kSdpaThreads / 32][TH], s_l[kSdpaThreads / 32][TH];
+    __shared__ float s_o[kSdpaThreads / 32][TH][D];
+    pdl_wait();
+    pdl_trigger();
+    const int c = blockIdx.x;
+    const int hk = blockIdx.y / tiles;
+    const int h0 = hk * G + (blockIdx.y % tiles) * TH;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hl = lane & 15;                       // dims 8 hl .. 8 hl + 7
+    const int stream = warp * 2 + (lane >> 4);      // 0 .. 15
+    float qr[TH][8];
+#pragma unroll
+    for (int i = 0; i < TH; ++i) {
+        load8(q + static_cast<int64_t>(h0 + i) * D + 8 * hl, qr[i]);
+#pragma unroll
+        for (int d = 0; d < 8; ++d) qr[i][d] *= qscale;
+    }
+    float m[TH], l[TH], acc[TH][8];
+#pragma unroll
+    for (int i = 0; i < TH; ++i) {
+        m[i] = -INFINITY;
+        l[i] = 0.0f;
+#pragma unroll
+        for (int d = 0; d < 8; ++d) acc[i][d] = 0.0f;
+    }
+    const int j0 = c * chunk, j1 = min(N, j0 + chunk);
+    const T* kb = k + static_cast<int64_t>(hk) * N * D + 8 * hl;
+    const T* vb = v + static_cast<int64_t>(hk) * N * D + 8 * hl;
+    // the trip count is the same for every lane of the CTA: the shuffles below
+    // always run with the whole warp; keys past the chunk only skip the update
+    for (int base = j0; base < j1; base += kStreams) {
+        const int j = base + stream;
+        const bool valid = j < j1;
+        float kf[8], vf[8];
+        if (valid) {
+            load8(kb + static_cast<int64_t>(j) * D, kf);
+            load8(vb + static_cast<int64_t>(j) * D, vf);
+        } else {
+#pragma unroll
+            for (int d = 0; d < 8; ++d) kf[d] = vf[d] = 0.0f;
+        }
+        float s[TH];
+#pragma unroll
+        for (int i = 0; i < TH; ++i) {
+            float t = 0.0f;
+#pragma unroll
+            for (int d = 0; d < 8; ++d) t = fmaf(qr[i][d], kf[d], t);
+            s[i] = t;
+        }
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+            for (int i = 0; i < TH; ++i) s[i] += __shfl_xor_sync(0xffffffffu, s[i], off);
+        if (valid) {
+#pragma unroll
+            for (int i = 0; i < TH; ++i) {
+                const float mn = fmaxf(m[i], s[i]);
+                const float corr = exp2f(m[i] - mn);  // 0 for the first key (m = -inf)
+                const float p = exp2f(s[i] - mn);
+                l[i] = fmaf(l[i], corr, p);
+#pragma unroll
+                for (int d = 0; d < 8; ++d) acc[i][d] = fmaf(p, vf[d], acc[i][d] * corr);
+                m[i] = mn;
+            }
+        }
+    }
+    // the two half-warps of a warp hold the same dims: merge them
+#pragma unroll
+    for (int i = 0; i < TH; ++i) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m[i], 16);
+        const float l2 = __shfl_xor_sync(0xffffffffu, l[i], 16);
+        float a2[8];
+#pragma unroll
+        for (int d = 0; d < 8; ++d) a2[d] = __shfl_xor_sync(0xffffffffu, acc[i][d], 16);
+        merge_state<8>(m[i], l[i], acc[i], m2, l2, a2);
+    }
+    if (lane < 16) {
+#pragma unroll
+        for (int i = 0; i < TH; ++i) {
+            if (lane == 0) {
+                s_m[warp][i] = m[i];
+                s_l[warp][i] = l[i];
+            }
+#pragma unroll
+            for (int d = 0; d < 8; ++d) s_o[warp][i][8 * hl + d] = acc[i][d];
+        }
+    }
+    __syncthreads();
+    // merge the 8 warps: thread t owns (head t / D, dim t % D)
+    for (int t = threadIdx.x; t < TH * D; t += kSdpaThreads) {
+        const int i = t / D, d = t % D;
+        float M = -INFINITY;
+        for (int w = 0; w < kSdpaThreads / 32; ++w) M = fmaxf(M, s_m[w][i]);
+        float L = 0.0f, O = 0.0f;
+        for (int w = 0; w < kSdpaThreads / 32; ++w) {
+            const float sc = s_m[w][i] == -INFINITY ? 0.0f : exp2f(s_m[w][i] - M);
+            L = fmaf(s_l[w][i], sc, L);
+            O = fmaf(s_o[w][i][d], sc, O);
+        }
+        float* pp = part + (static_cast<int64_t>(h0 + i) * chunks + c) * (D + 2);
+        pp[d] = O;
+        if (d == 0) {
+            pp[D] = M;
+            pp[D + 1] = L;
+        }
+    }
+}
+
+// out[h][d] = sum_c o_c[d] 2^(m_c - M) / sum_c l_c 2^(m_c - M): one CTA per query head.
+template <typename T>
+__global__ void __launch_bounds__(kSdpaD) k_sdpa_decode_merge(const float* __restrict__ part, int chunks,
+                                                             T* __restrict__ out) {
+    constexpr int D = kSdpaD;
+    pdl_wait();
+    pdl_trigger();
+    const int h = blockIdx.x, d = threadIdx.x;
+    const float* ph = part + static_cast<int64_t>(h) * chunks * (D + 2);
+    float M = -INFINITY;
+    for (int c = 0; c < chunks; ++c) M = fmaxf(M, ph[c * (D + 2) + D]);
+    float L = 0.0f, O = 0.0f;
+    for (int c = 0; c < chunks; ++c) {
+        const float* pc = ph + c * (D + 2);
+        const float sc = exp2f(pc[D] - M);
+        L = fmaf(pc[D + 1], sc, L);
+        O = fmaf(pc[d], sc, O);
+    }
+    const float y = O / L;
+    if constexpr (std::is_same<T, __half>::value)
+        out[static_cast<int64_t>(h) * D + d] = __float2half_rn(y);
+    else
+        out[static_cast<int64_t>(h) * D + d] = __float2bfloat16_rn(y);
+}
+
+template <int TH, typename T>
+cudaError_t launch_t(const void* q, const void* k, const void* v, int H_q, int H_kv, int N, const SdpaPlan& p,
+                     float* part, void* out, cudaStream_t st) {
+    const int G = H_q / H_kv;
+    const float qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kSdpaD)));
+    const dim3 grid(static_cast<unsigned>(p.chunks), static_cast<unsigned>(H_kv * p.tiles));
+    cudaError_t e = launch_pdl(k_sdpa_decode_split<TH, T>, grid, kSdpaThreads, 0, st, static_cast<const T*>(q),
+                               static_cast<const T*>(k), static_cast<const T*>(v), G, p.tiles, N, p.chunk, p.chunks,
+                               qscale, part);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_sdpa_decode_merge<T>, static_cast<unsigned>(H_q), kSdpaD, 0, st,
+                      static_cast<const float*>(part), p.chunks, static_cast<T*>(out));
+}
+
+template <typename T>
+cudaError_t launch_dt(const void* q, const void* k, const void* v, int H_q, int H_kv, int N, const SdpaPlan& p,
+                      float* part, void* out, cudaStream_t st) {
+    switch (p.th) {
+        case 4: return launch_t<4, T>(q, k, v, H_q, H_kv, N, p, part, out, st);
+        case 2: return launch_t<2, T>(q, k, v, H_q, H_kv, N, p, part, out, st);
+        default: return launch_t<1, T>(q, k, v, H_q, H_kv, N, p, part, out, st);
+    }
+}
+
+}  // namespace
+
+SdpaPlan sdpa_plan(int64_t H_q, int64_t H_kv, int64_t N, int num_sms) {
+    SdpaPlan p{};
+    const int64_t G = H_q / H_kv;
+    p.th = G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1);
+    p.tiles = static_cast<int>(G / p.th);
+    const int64_t rows = H_kv * p.tiles;                  // CTAs per chunk index
+    const int64_t target = 4 * static_cast<int64_t>(num_sms);
+    int64_t chunks = std::max<int64_t>(1, (target + rows - 1) / rows);
+    chunks = std::min<int64_t>(chunks, (N + kStreams - 1) / kStreams);  // at least 16 keys per chunk
+    int64_t chunk = (N + chunks - 1) / chunks;
+    chunk = (chunk + kStreams - 1) / kStreams * kStreams;
+    p.chunk = static_cast<int>(chunk);
+    p.chunks = static_cast<int>((N + chunk - 1) / chunk);
+    return p;
+}
+
+size_t sdpa_part_bytes(int64_t H_q, const SdpaPlan& p) {
+    return static_cast<size_t>(H_q) * p.chunks * (kSdpaD + 2) * sizeof(float);
+}
+
+cudaError_t launch_sdpa_decode(const void* q, const void* k, const void* v, int dt, int H_q, int H_kv, int N,
+                               const SdpaPlan& plan, float* part, void* out, cudaStream_t st) {
+    return dt == 1 ? launch_dt<__nv_bfloat16>(q, k, v, H_q, H_kv, N, plan, part, out, st)
+                   : launch_dt<__half>(q, k, v, H_q, H_kv, N, plan, part, out, st);
+}
+
+}  // namespace cider
