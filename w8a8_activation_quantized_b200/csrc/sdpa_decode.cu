@@ -36,6 +36,25 @@ namespace {
 
 constexpr int kSdpaThreads = 256;  // 8 warps = 16 half-warp key streams
 constexpr int kStreams = kSdpaThreads / 16;
+constexpr int kMaxChunks = 1024;   // chunk scales of one head fit in shared memory
+
+// 2^x by the hardware approximation (PTX ex2.approx: relative error near
+// 2^-22, 2^-inf = +0); the softmax weights need no more.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float warp_reduce_max(float v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_reduce_sum(float v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
 
 template <typename T>
 __device__ __forceinline__ void load8(const T* p, float (&f)[8]) {
@@ -58,7 +77,7 @@ template <int ND>
 __device__ __forceinline__ void merge_state(float& m, float& l, float (&a)[ND], float m2, float l2, const float (&a2)[ND]) {
     const float M = fmaxf(m, m2);
     if (M == -INFINITY) return;  // both empty
-    const float s1 = exp2f(m - M), s2 = exp2f(m2 - M);
+    const float s1 = ex2(m - M), s2 = ex2(m2 - M);
     l = l * s1 + l2 * s2;
 #pragma unroll
     for (int d = 0; d < ND; ++d) a[d] = a[d] * s1 + a2[d] * s2;
@@ -128,13 +147,19 @@ __global__ void __launch_bounds__(kSdpaThreads) k_sdpa_decode_split(const T* __r
         if (valid) {
 #pragma unroll
             for (int i = 0; i < TH; ++i) {
-                const float mn = fmaxf(m[i], s[i]);
-                const float corr = exp2f(m[i] - mn);  // 0 for the first key (m = -inf)
-                const float p = exp2f(s[i] - mn);
-                l[i] = fmaf(l[i], corr, p);
+                // rescale only when the key raises the running maximum (the same
+                // decision in the whole half-warp; rare after the first keys)
+                if (s[i] > m[i]) {
+                    const float corr = ex2(m[i] - s[i]);  // 0 for the first key (m = -inf)
+                    l[i] *= corr;
 #pragma unroll
-                for (int d = 0; d < 8; ++d) acc[i][d] = fmaf(p, vf[d], acc[i][d] * corr);
-                m[i] = mn;
+                    for (int d = 0; d < 8; ++d) acc[i][d] *= corr;
+                    m[i] = s[i];
+                }
+                const float p = ex2(s[i] - m[i]);
+                l[i] += p;
+#pragma unroll
+                for (int d = 0; d < 8; ++d) acc[i][d] = fmaf(p, vf[d], acc[i][d]);
             }
         }
     }
@@ -167,7 +192,7 @@ __global__ void __launch_bounds__(kSdpaThreads) k_sdpa_decode_split(const T* __r
         for (int w = 0; w < kSdpaThreads / 32; ++w) M = fmaxf(M, s_m[w][i]);
         float L = 0.0f, O = 0.0f;
         for (int w = 0; w < kSdpaThreads / 32; ++w) {
-            const float sc = s_m[w][i] == -INFINITY ? 0.0f : exp2f(s_m[w][i] - M);
+            const float sc = s_m[w][i] == -INFINITY ? 0.0f : ex2(s_m[w][i] - M);
             L = fmaf(s_l[w][i], sc, L);
             O = fmaf(s_o[w][i][d], sc, O);
         }
@@ -180,24 +205,43 @@ __global__ void __launch_bounds__(kSdpaThreads) k_sdpa_decode_split(const T* __r
     }
 }
 
-// out[h][d] = sum_c o_c[d] 2^(m_c - M) / sum_c l_c 2^(m_c - M): one CTA per query head.
+// out[h][d] = sum_c o_c[d] 2^(m_c - M) / sum_c l_c 2^(m_c - M): one CTA per
+// query head.  The maximum and the sum run across the block's threads; the
+// chunk scales wait in shared memory and the output loop keeps eight
+// independent loads in flight.
 template <typename T>
 __global__ void __launch_bounds__(kSdpaD) k_sdpa_decode_merge(const float* __restrict__ part, int chunks,
                                                              T* __restrict__ out) {
     constexpr int D = kSdpaD;
+    __shared__ float s_sc[kMaxChunks];
+    __shared__ float s_red[2][D / 32];
     pdl_wait();
     pdl_trigger();
-    const int h = blockIdx.x, d = threadIdx.x;
+    const int h = blockIdx.x, d = threadIdx.x, lane = d & 31, w = d >> 5;
     const float* ph = part + static_cast<int64_t>(h) * chunks * (D + 2);
     float M = -INFINITY;
-    for (int c = 0; c < chunks; ++c) M = fmaxf(M, ph[c * (D + 2) + D]);
-    float L = 0.0f, O = 0.0f;
-    for (int c = 0; c < chunks; ++c) {
-        const float* pc = ph + c * (D + 2);
-        const float sc = exp2f(pc[D] - M);
-        L = fmaf(pc[D + 1], sc, L);
-        O = fmaf(pc[d], sc, O);
+    for (int c = d; c < chunks; c += D) M = fmaxf(M, ph[c * (D + 2) + D]);
+    M = warp_reduce_max(M);
+    if (lane == 0) s_red[0][w] = M;
+    __syncthreads();
+    M = s_red[0][0];
+#pragma unroll
+    for (int i = 1; i < D / 32; ++i) M = fmaxf(M, s_red[0][i]);
+    float L = 0.0f;
+    for (int c = d; c < chunks; c += D) {
+        const float sc = ex2(ph[c * (D + 2) + D] - M);
+        s_sc[c] = sc;
+        L = fmaf(ph[c * (D + 2) + D + 1], sc, L);
     }
+    L = warp_reduce_sum(L);
+    if (lane == 0) s_red[1][w] = L;
+    __syncthreads();
+    L = 0.0f;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) L += s_red[1][i];
+    float O = 0.0f;
+#pragma unroll 8
+    for (int c = 0; c < chunks; ++c) O = fmaf(ph[c * (D + 2) + d], s_sc[c], O);
     const float y = O / L;
     if constexpr (std::is_same<T, __half>::value)
         out[static_cast<int64_t>(h) * D + d] = __float2half_rn(y);
@@ -240,6 +284,7 @@ SdpaPlan sdpa_plan(int64_t H_q, int64_t H_kv, int64_t N, int num_sms) {
     const int64_t target = 4 * static_cast<int64_t>(num_sms);
     int64_t chunks = std::max<int64_t>(1, (target + rows - 1) / rows);
     chunks = std::min<int64_t>(chunks, (N + kStreams - 1) / kStreams);  // at least 16 keys per chunk
+    chunks = std::min<int64_t>(chunks, kMaxChunks);                      // the merge keeps one scale per chunk
     int64_t chunk = (N + chunks - 1) / chunks;
     chunk = (chunk + kStreams - 1) / kStreams * kStreams;
     p.chunk = static_cast<int>(chunk);
