@@ -57,8 +57,7 @@ __device__ __forceinline__ float warp_reduce_sum(float v) {
 }
 
 template <typename T>
-__device__ __forceinline__ void load8(const T* p, float (&f)[8]) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
+__device__ __forceinline__ void cvt8(const uint4& raw, float (&f)[8]) {
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -70,6 +69,10 @@ __device__ __forceinline__ void load8(const T* p, float (&f)[8]) {
         f[2 * i] = t.x;
         f[2 * i + 1] = t.y;
     }
+}
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&f)[8]) {
+    cvt8<T>(__ldg(reinterpret_cast<const uint4*>(p)), f);
 }
 
 // Merge online-softmax state (m2, l2, a2) into (m, l, a); m = -inf means empty.
@@ -119,13 +122,34 @@ __global__ void __launch_bounds__(kSdpaThreads) k_sdpa_decode_split(const T* __r
     const int j0 = c * chunk, j1 = min(N, j0 + chunk);
     const T* kb = k + static_cast<int64_t>(hk) * N * D + 8 * hl;
     const T* vb = v + static_cast<int64_t>(hk) * N * D + 8 * hl;
-    // the trip count is the same for every lane of the CTA: the shuffles below
-    // always run with the whole warp; keys past the chunk only skip the update
+    // The trip count is the same for every lane of the CTA: the shuffles below
+    // always run with the whole warp; keys past the chunk only skip the update.
+    // With two or four heads per thread the next key's K and V rows are loaded
+    // while the current key is used (measured: GQA4 / GQA8 at N = 32K 65.0 /
+    // 59.7 -> 50.6 / 46.6 us); with one head the direct loads measured faster
+    // (MHA at N = 32K: 102.6 us against 152.6 us with the prefetch).
+    constexpr bool kPrefetch = TH > 1;
+    const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+    uint4 knext = zero4, vnext = zero4;
+    if (kPrefetch && j0 + stream < j1) {
+        knext = __ldg(reinterpret_cast<const uint4*>(kb + static_cast<int64_t>(j0 + stream) * D));
+        vnext = __ldg(reinterpret_cast<const uint4*>(vb + static_cast<int64_t>(j0 + stream) * D));
+    }
     for (int base = j0; base < j1; base += kStreams) {
         const int j = base + stream;
         const bool valid = j < j1;
         float kf[8], vf[8];
-        if (valid) {
+        if constexpr (kPrefetch) {
+            const uint4 kraw = knext, vraw = vnext;
+            const int jn = j + kStreams;
+            knext = vnext = zero4;
+            if (jn < j1) {
+                knext = __ldg(reinterpret_cast<const uint4*>(kb + static_cast<int64_t>(jn) * D));
+                vnext = __ldg(reinterpret_cast<const uint4*>(vb + static_cast<int64_t>(jn) * D));
+            }
+            cvt8<T>(kraw, kf);  // zeros past the chunk
+            cvt8<T>(vraw, vf);
+        } else if (valid) {
             load8(kb + static_cast<int64_t>(j) * D, kf);
             load8(vb + static_cast<int64_t>(j) * D, vf);
         } else {
