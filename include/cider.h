@@ -280,7 +280,7 @@ CIDER_API cider_status_t cider_pack_weight_int4_pc(const float* W, int64_t N, in
  *   out[h] = sum_j softmax_j(q[h] . K[g][j] / sqrt(D)) V[g][j].
  * q [H_q][D], K and V [H_kv][N][D] (head-major cache), out [H_q][D]; all in
  * dt (fp16 or bf16), device memory owned by the caller, 16-byte aligned.
- * D must be 128; H_kv must divide H_q; 1 <= N < 2^31.  The sequence is cut
+ * D must be 128; H_kv must divide H_q; 1 <= N <= 2^30.  The sequence is cut
  * into chunks whose fp32 partial results go to the workspace
  * (cider_sdpa_decode_workspace_bytes; it depends on the device's SM count);
  * a second kernel merges them.  Errors: CIDER_ERR_INVALID_ARG for the shape

@@ -615,7 +615,8 @@ static cider_status_t sdpa_check(int64_t H_q, int64_t H_kv, int64_t N, int64_t D
     if (H_q < 1 || H_kv < 1 || H_q % H_kv)
         return fail(CIDER_ERR_INVALID_ARG, "H_q = %lld must be a positive multiple of H_kv = %lld", (long long)H_q, (long long)H_kv);
     if (H_q > 65535) return fail(CIDER_ERR_INVALID_ARG, "H_q = %lld exceeds 65535", (long long)H_q);
-    if (N < 1 || N > INT32_MAX) return fail(CIDER_ERR_INVALID_ARG, "N = %lld must lie in [1, 2^31)", (long long)N);
+    // the kernels index keys with 32-bit ints (chunk ends up to N + chunk)
+    if (N < 1 || N > (int64_t(1) << 30)) return fail(CIDER_ERR_INVALID_ARG, "N = %lld must lie in [1, 2^30]", (long long)N);
     return CIDER_OK;
 }
 

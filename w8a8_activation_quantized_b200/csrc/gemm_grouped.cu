@@ -36,9 +36,13 @@
 // M) every tile is a tail tile.
 // Cost model (measured on B200): per group and 128 x 128 tile the epilogue
 // moves every partial TMEM -> registers once and issues two fp32 operations
-// per partial; these do not overlap, which puts the floor near 384 cycles
-// per group per SM sub-partition -- the epilogue, not the tensor core, bounds
-// this kernel at gs = 64 and gs = 128.
+// per partial; these do not overlap, which puts its floor near 384 cycles per
+// group per SM sub-partition.  The kernel runs at about 1000 cycles per
+// group: with the epilogue's fp32 work, its TMEM reads, the TMA loads or the
+// i8 MMAs switched off in experiments the time barely moves, so the per-group
+// hand-off between the MMA warp and the epilogue (commit, wait, release)
+// sets the pace; the tensor time of a group adds to it rather than
+// overlapping it.
 // W4A8 with per-output-channel scales (mode kModeW4PC; Cider README, table
 // "量化": symmetric INT4, zero point 8, per column) runs the same producer and
 // converter warps, but the MMA warp accumulates a whole work unit into one
