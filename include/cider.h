@@ -315,6 +315,10 @@ CIDER_API cider_status_t cider_test_set_split_k(int splits);
  * and clears the status word. */
 CIDER_API cider_status_t cider_test_bounded_wait(int64_t limit_ns, void* stream);
 /* The W4A8 load path's unpack: w[n][k] = nibble(n, k) - 8. */
+/* The decode-attention cut for a device with num_sms SMs, without a device:
+ * out4 = {query heads per CTA, head tiles per KV group, keys per chunk,
+ * chunks}.  Same shape rules as cider_sdpa_decode. */
+CIDER_API cider_status_t cider_test_sdpa_plan(int64_t H_q, int64_t H_kv, int64_t N, int64_t num_sms, int32_t* out4);
 CIDER_API cider_status_t cider_test_unpack_int4(const uint8_t* w_packed, int64_t N, int64_t K, int8_t* w,
                                       void* stream);
 

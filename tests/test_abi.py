@@ -104,3 +104,74 @@ def test_no_device_means_unsupported_or_cuda_error(lib):
     # valid arguments, no device: the call must fail loudly, never compute on the CPU
     st = _lin_pc(lib)
     assert st in (2, 3)
+
+
+# ---- the entry points added for the pages' other forms: host-side checks ----
+
+def _sdpa(lib, **kw):
+    a = dict(q=P, k=ctypes.c_void_p(4096), v=ctypes.c_void_p(1 << 16), dt=0, H_q=32, H_kv=8, N=64, D=128,
+             out=ctypes.c_void_p(1 << 20), ws=ctypes.c_void_p(1 << 22), wsb=1 << 20, st=None)
+    a.update(kw)
+    return lib.cider_sdpa_decode(a["q"], a["k"], a["v"], a["dt"], a["H_q"], a["H_kv"], a["N"], a["D"], a["out"],
+                                 a["ws"], a["wsb"], a["st"])
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(D=64), "D must be 128"),
+    (dict(H_q=30), "H_kv must divide H_q"),
+    (dict(H_kv=0), "H_kv >= 1"),
+    (dict(N=0), "N >= 1"),
+    (dict(N=(1 << 30) + 1), "N <= 2^30"),
+    (dict(dt=7), "dtype"),
+    (dict(v=None), "NULL"),
+    (dict(k=ctypes.c_void_p(4100)), "misaligned"),
+])
+def test_sdpa_arguments_rejected_on_host(lib, kw, why):
+    assert _sdpa(lib, **kw) == 1, why
+    assert lib.cider_last_error()
+
+
+def test_sdpa_without_a_device_fails_loudly(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _sdpa(lib) in (2, 3)
+
+
+@pytest.mark.parametrize("H_q,H_kv", [(32, 32), (32, 8), (32, 4), (8, 1), (6, 3), (3, 1), (64, 2)])
+@pytest.mark.parametrize("N", [1, 15, 16, 17, 1000, 1024, 4096, 32768, 1 << 20])
+@pytest.mark.parametrize("sms", [148, 132, 1])
+def test_sdpa_plan_covers_every_key(H_q, H_kv, N, sms):
+    th, tiles, chunk, chunks = cider.cider_test_sdpa_plan(H_q, H_kv, N, sms)
+    G = H_q // H_kv
+    assert th in (1, 2, 4) and th * tiles == G
+    assert th == (4 if G % 4 == 0 else 2 if G % 2 == 0 else 1)
+    assert chunk % 16 == 0 and chunk >= 16
+    assert 1 <= chunks <= 1024
+    assert (chunks - 1) * chunk < N <= chunks * chunk  # every chunk has a key; every key has a chunk
+    # enough CTAs to fill the device, unless the keys or the merge's chunk limit run out first
+    assert H_kv * tiles * chunks >= min(4 * sms, H_kv * tiles * -(-N // 16)) or chunks >= 1024 or \
+        chunks == -(-N // chunk)
+
+
+def test_sdpa_plan_rejects_bad_shapes(lib):
+    with pytest.raises(cider.CiderError):
+        cider.cider_test_sdpa_plan(30, 8, 64, 148)
+    with pytest.raises(cider.CiderError):
+        cider.cider_test_sdpa_plan(32, 8, 64, 0)
+
+
+def test_clip_and_w4pc_arguments_rejected_on_host(lib):
+    W, out, sw = P, ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 21)
+    for p in (-0.5, 100.5, float("nan")):
+        assert lib.cider_quantize_weight_pc_clip(W, 8, 64, p, out, sw, None) == 1
+    assert lib.cider_quantize_weight_pg_clip(W, 8, 256, 32, 99.9, out, sw, None) == 1      # gs not 64/128
+    assert lib.cider_pack_weight_int4_pc(W, 8, 63, out, sw, None) == 1                      # odd K
+    assert lib.cider_w4a8_linear_pc(P, 0, 4, 48, ctypes.c_void_p(4096), ctypes.c_void_p(8192), 16,
+                                    ctypes.c_void_p(1 << 20), 0, None, 0, None) == 1          # K % 32
+
+
+def test_w4pc_workspace_covers_small_m(lib):
+    # the per-column W4A8 form has no decode kernel: even M = 1 needs q and scale_x
+    assert lib.cider_workspace_bytes_w4a8_pc(1, 256, 1024) >= 1024 + 256
+    assert lib.cider_workspace_bytes_w4a8_pc(0, 256, 1024) == 0

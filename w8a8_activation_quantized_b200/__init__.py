@@ -51,6 +51,7 @@ _SIGNATURES = {
     "cider_workspace_bytes_w4a8_pc": (_SZ, [_I64, _I64, _I64]),
     "cider_sdpa_decode_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64]),
     "cider_sdpa_decode": (_INT, [_P, _P, _P, _INT, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "cider_test_sdpa_plan": (_INT, [_I64, _I64, _I64, _I64, _P]),
     "cider_w8a8_linear_pc_noalloc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_w8a8_gemm_pc_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
     "cider_w8a8_gemm_pg_q": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P]),
@@ -367,6 +368,13 @@ def cider_pack_weight_int4_pc(W, stream=None):
 
 def cider_sdpa_decode_workspace_bytes(H_q: int, H_kv: int, N: int, D: int = 128) -> int:
     return int(lib().cider_sdpa_decode_workspace_bytes(H_q, H_kv, N, D))
+
+
+def cider_test_sdpa_plan(H_q, H_kv, N, num_sms):
+    """-> (query heads per CTA, head tiles per KV group, keys per chunk, chunks)."""
+    out = (ctypes.c_int32 * 4)()
+    _check("cider_test_sdpa_plan", lib().cider_test_sdpa_plan(H_q, H_kv, N, num_sms, out))
+    return tuple(out)
 
 
 def cider_sdpa_decode(q, k, v, out=None, workspace=None, stream=None):

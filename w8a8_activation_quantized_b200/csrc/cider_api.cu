@@ -627,6 +627,19 @@ size_t cider_sdpa_decode_workspace_bytes(int64_t H_q, int64_t H_kv, int64_t N, i
     return sdpa_part_bytes(H_q, sdpa_plan(H_q, H_kv, N, d->num_sms));
 }
 
+cider_status_t cider_test_sdpa_plan(int64_t H_q, int64_t H_kv, int64_t N, int64_t num_sms, int32_t* out4) {
+    t_last_error[0] = '\0';
+    cider_status_t s = sdpa_check(H_q, H_kv, N, kSdpaD);
+    if (s != CIDER_OK) return s;
+    if (num_sms < 1 || num_sms > 4096 || !out4) return fail(CIDER_ERR_INVALID_ARG, "num_sms in [1, 4096] and out4 required");
+    const SdpaPlan p = sdpa_plan(H_q, H_kv, N, static_cast<int>(num_sms));
+    out4[0] = p.th;
+    out4[1] = p.tiles;
+    out4[2] = p.chunk;
+    out4[3] = p.chunks;
+    return CIDER_OK;
+}
+
 cider_status_t cider_sdpa_decode(const void* q, const void* k, const void* v, cider_dtype_t dt, int64_t H_q,
                                  int64_t H_kv, int64_t N, int64_t D, void* out, void* workspace,
                                  size_t workspace_bytes, void* stream) {
