@@ -194,15 +194,20 @@ CIDER_API cider_status_t cider_w4a8_linear_pc(const void* x, cider_dtype_t xdt, 
  * pool and forbids outside allocations, or code that must stay inside a
  * memory budget fixed at start-up.  This entry point computes exactly what
  * cider_w8a8_linear_pc computes, but keeps the quantized activations and
- * their scales in a scratch array built into the library: 32 MiB of device
- * memory, which every GPU that loads the library holds until the process
- * exits.  It allocates nothing and calls no allocating routine.
+ * their scales -- and, for shapes whose last round of output tiles is cut
+ * along K, the fp32 partial sums of those tiles when they fit after them --
+ * in a scratch array built into the library: 32 MiB of device memory, which
+ * every GPU that loads the library holds until the process exits.  It
+ * allocates nothing and calls no allocating routine.
  *  - Limit: cider_workspace_bytes(M, K) must not exceed 32 MiB (roughly
  *    M * K + 4 * M <= 32 MiB); larger calls return CIDER_ERR_INVALID_ARG with
  *    a message and launch nothing.  Calls that take the fused small-M kernel
  *    do not touch the scratch.
  *  - The first call on each device looks up the scratch's device address,
- *    with that device current; make that first call before any stream capture.
+ *    with that device current; make that first call before any stream
+ *    capture.  The address is kept for the life of the process: after a
+ *    cudaDeviceReset() the array is reloaded elsewhere, so a process that
+ *    resets a device must not call this entry point again on it.
  *  - All calls on a device share the one scratch array and it keeps the last
  *    call's contents.  Calls whose kernels overlap on the GPU (on different
  *    streams, or from different host threads) race on it and give wrong
@@ -314,11 +319,11 @@ CIDER_API cider_status_t cider_test_set_split_k(int splits);
  * (1 .. 1e8).  The next cider_device_status() then returns CIDER_ERR_TIMEOUT
  * and clears the status word. */
 CIDER_API cider_status_t cider_test_bounded_wait(int64_t limit_ns, void* stream);
-/* The W4A8 load path's unpack: w[n][k] = nibble(n, k) - 8. */
 /* The decode-attention cut for a device with num_sms SMs, without a device:
  * out4 = {query heads per CTA, head tiles per KV group, keys per chunk,
  * chunks}.  Same shape rules as cider_sdpa_decode. */
 CIDER_API cider_status_t cider_test_sdpa_plan(int64_t H_q, int64_t H_kv, int64_t N, int64_t num_sms, int32_t* out4);
+/* The W4A8 load path's unpack: w[n][k] = nibble(n, k) - 8. */
 CIDER_API cider_status_t cider_test_unpack_int4(const uint8_t* w_packed, int64_t N, int64_t K, int8_t* w,
                                       void* stream);
 

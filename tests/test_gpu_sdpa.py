@@ -1,13 +1,18 @@
 """Decode attention on the GPU (Cider README, section "优化 SDPA（解码注意
 力）") against the float64 oracle: the pages' configurations (MHA, GQA4, GQA8
 at D = 128) up to N = 32K, ragged sequence lengths (one key, fewer keys than
-a chunk's streams, chunk tails), other group sizes, bf16, and the argument
-checks.
+a chunk's streams, chunk tails), other group sizes, bf16, peaked weights
+(queries scaled by 8, outputs of order one), a maximum that arrives in the
+last chunk, and the argument checks.
 
-Tolerance: every output is a convex combination of its KV head's value rows,
-so |out| <= max|V|; its final rounding costs at most one unit of the format
-at that size and the fp32 chunked softmax adds far less.  The bound is four
-units at max|V|: 2^-9 * max|V| for fp16, 2^-6 * max|V| for bf16."""
+Tolerance (tests/sdpa_tolerance.py): element by element, one unit of the
+output format at the output itself plus a bound on the kernels' fp32 error
+that scales with sum_j p_j |v_j| and with the depth of the kernels'
+summation, derived from the arithmetic they do.  tests/test_sdpa_tolerance.py
+shows on the host that this bound rejects a dropped chunk, an unrescaled
+chunk partial and a dropped key stream.  The pages report a maximum
+difference of 1.22e-4 (fp16) against their reference; the largest
+difference seen here is printed by test_sdpa_max_difference_report."""
 import numpy as np
 import pytest
 import torch
@@ -16,10 +21,11 @@ import oracle
 from oracle import sdpa
 import w8a8_activation_quantized_b200 as cider
 from tests.parity import dev_bits, host_bits
+from tests import sdpa_tolerance as tl
 
 pytestmark = pytest.mark.gpu
 D = 128
-TOL = {oracle.F16: 2.0 ** -9, oracle.BF16: 2.0 ** -6}
+MAX_DIFF = {}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -30,23 +36,19 @@ def _device():
     cider.cider_device_status()
 
 
-def _inputs(H_q, H_kv, N, seed, dt=oracle.F16):
-    rng = np.random.default_rng(seed)
-    q = oracle.narrow(rng.normal(0, 1, size=(H_q, D)), dt)
-    k = oracle.narrow(rng.normal(0, 1, size=(H_kv, N, D)), dt)
-    v = oracle.narrow(rng.normal(0, 1, size=(H_kv, N, D)), dt)
-    return q, k, v
+def _num_sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
 
 
-def _check(H_q, H_kv, N, seed, dt=oracle.F16):
-    q, k, v = _inputs(H_q, H_kv, N, seed, dt)
+def _check(H_q, H_kv, N, seed, dt=oracle.F16, kind="diffuse"):
+    q, k, v = tl.make_inputs(kind, H_q, H_kv, N, seed, dt)
     out = cider.cider_sdpa_decode(dev_bits(q, dt), dev_bits(k, dt), dev_bits(v, dt))
-    got = oracle.as_float(host_bits(out), dt).astype(np.float64)
-    ref = oracle.as_float(sdpa.sdpa_decode(q, k, v, dt), dt).astype(np.float64)
-    vmax = np.abs(oracle.widen(v, dt)).max(axis=(1, 2)).repeat(H_q // H_kv)[:, None]
-    err = np.abs(got - ref)
-    assert np.all(np.isfinite(got))
-    assert np.all(err <= TOL[dt] * vmax), f"max err / max|V| = {np.max(err / vmax):.3g}"
+    got = host_bits(out)
+    ref = sdpa.sdpa_decode(q, k, v, dt)
+    assert np.all(np.isfinite(oracle.as_float(got, dt)))
+    n_bad, max_diff = tl.violations(ref, got, q, k, v, dt, _num_sms())
+    MAX_DIFF[(kind, H_q, H_kv, N, dt)] = max_diff
+    assert n_bad == 0, f"{n_bad} outputs out of tolerance; max |diff| = {max_diff:.3g}"
     return out
 
 
@@ -62,23 +64,49 @@ def test_sdpa_ragged(H_q, H_kv, N):
     _check(H_q, H_kv, N, seed=N * 7 + H_q + H_kv)
 
 
+@pytest.mark.parametrize("kind", ["peaked", "last_max"])
+@pytest.mark.parametrize("H_kv", [32, 8, 4])
+@pytest.mark.parametrize("N", [1024, 4096, 32768])
+def test_sdpa_concentrated(H_kv, N, kind):
+    _check(32, H_kv, N, seed=3 * N + H_kv, kind=kind)
+
+
+@pytest.mark.parametrize("kind", ["diffuse", "last_max"])
+@pytest.mark.parametrize("H_kv", [32, 4])
+def test_sdpa_bf16_kinds(H_kv, kind):
+    _check(32, H_kv, 2049, seed=H_kv + 1, dt=oracle.BF16, kind=kind)
+
+
 @pytest.mark.parametrize("H_kv", [32, 4])
 def test_sdpa_bf16(H_kv):
     _check(32, H_kv, 2049, seed=H_kv, dt=oracle.BF16)
 
 
 def test_sdpa_single_key_is_its_value_exactly():
-    q, k, v = _inputs(32, 8, 1, seed=5)
+    q, k, v = tl.make_inputs("diffuse", 32, 8, 1, seed=5)
     out = cider.cider_sdpa_decode(dev_bits(q, oracle.F16), dev_bits(k, oracle.F16), dev_bits(v, oracle.F16))
     np.testing.assert_array_equal(host_bits(out), np.repeat(v[:, 0, :], 4, axis=0))
 
 
 def test_sdpa_argument_checks():
-    q, k, v = _inputs(32, 8, 64, seed=6)
+    q, k, v = tl.make_inputs("diffuse", 32, 8, 64, seed=6)
     qd, kd, vd = (dev_bits(a, oracle.F16) for a in (q, k, v))
     with pytest.raises(cider.CiderError):  # H_kv must divide H_q
-        cider.cider_sdpa_decode(dev_bits(_inputs(30, 8, 64, 1)[0], oracle.F16), kd, vd)
+        cider.cider_sdpa_decode(dev_bits(tl.make_inputs("diffuse", 30, 8, 64, 1)[0], oracle.F16), kd, vd)
     with pytest.raises(cider.CiderError):  # D = 128 only
         cider.cider_sdpa_decode(qd[:, :64].contiguous(), kd[:, :, :64].contiguous(), vd[:, :, :64].contiguous())
     with pytest.raises(cider.CiderError):  # workspace too small
         cider.cider_sdpa_decode(qd, kd, vd, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+
+
+def test_sdpa_max_difference_report():
+    """The largest |GPU - oracle| over the fp16 cases of this module, beside the
+    pages' 1.22e-4 (fp16, against their reference implementation)."""
+    f16 = {key: d for key, d in MAX_DIFF.items() if key[-1] == oracle.F16}
+    if not f16:
+        pytest.skip("no fp16 case ran in this session")
+    worst = max(f16, key=f16.get)
+    print(f"\nsdpa fp16 max |diff| over {len(f16)} cases: {f16[worst]:.3g} at {worst[:4]} (pages: 1.22e-4)")
+    pages = [d for key, d in f16.items() if key[0] == "diffuse" and key[1] == 32 and key[3] in (1024, 4096, 32768)]
+    if pages:
+        print(f"sdpa fp16 max |diff| over the pages' nine configurations: {max(pages):.3g}")

@@ -5,9 +5,12 @@ owns all of the GPU's memory through its own pool, or code held to a memory
 budget fixed at start-up.  They cannot pass the workspace that
 cider_w8a8_linear_pc needs, so this entry point keeps its scratch in a fixed
 array built into the library.  These tests call it through the C ABI and
-check it against the entry point that takes a workspace, on two calls in a
-row with different inputs and shapes, so that a call reading what the
-previous call left in the shared scratch would be caught.
+check it against the entry point that takes a workspace and against the
+oracle (sampled token rows, which are independent), on calls in a row with
+different inputs and shapes, so that a call reading what the previous call
+left in the shared scratch would be caught.  The last of them is large
+enough for the per-channel GEMM to split K, so its partial sums also live in
+the scratch.
 
 This file is named to be collected last, and it passes both on its own in a
 fresh process and after the rest of the suite.
@@ -21,7 +24,7 @@ import torch
 import oracle
 import w8a8_activation_quantized_b200 as cider
 from w8a8_activation_quantized_b200 import synth
-from tests.parity import TOL, dev, host_bits
+from tests.parity import TOL, check_y, dev, host_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -54,9 +57,11 @@ def _device():
 def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
     old = cider.cider_get_small_m_threshold()
     try:
-        cider.cider_set_small_m_threshold(0)  # both calls take the tensor-core path, which uses the scratch
-        for (M, N, K, seed) in [(300, 1032, 4096, 1), (129, 264, 2560, 2)]:
-            x = torch.from_numpy(synth.activations(M, K, seed)).cuda()
+        cider.cider_set_small_m_threshold(0)  # every call takes the tensor-core path, which uses the scratch
+        # the third shape's CTA-pair tiles leave a partial last round, cut along K
+        for (M, N, K, seed) in [(300, 1032, 4096, 1), (129, 264, 2560, 2), (1024, 5120, 8192, 3)]:
+            xh = synth.activations(M, K, seed)
+            x = torch.from_numpy(xh).cuda()
             qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed))
             w, s = dev(qw), dev(sw)
             y_ref = cider.cider_w8a8_linear_pc(x, w, s)
@@ -64,6 +69,9 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
             assert _call_noalloc(x, w, s, y) == 0, cider.lib().cider_last_error()
             torch.cuda.synchronize()
             _close(y, y_ref)
+            rows = np.unique(np.concatenate([[0, 127, 128, 255, 256, M - 1],
+                                             np.random.default_rng(seed).choice(M, 10, replace=False)]))
+            check_y(y[torch.from_numpy(rows).cuda()], oracle.linear_pc(xh[rows], qw, sw), oracle.F16)
     finally:
         cider.cider_set_small_m_threshold(old)
     cider.cider_device_status()
@@ -77,6 +85,7 @@ def test_noalloc_small_m_and_too_large():
     y = torch.empty((M, N), dtype=torch.float16, device="cuda")
     assert _call_noalloc(x, w, s, y) == 0
     _close(y, cider.cider_w8a8_linear_pc(x, w, s))
+    check_y(y, oracle.linear_pc(synth.activations(M, K, 3), qw, sw), oracle.F16)
     # beyond the built-in scratch: rejected with a message, nothing launched
     big = torch.empty((8192, 8192), dtype=torch.float16, device="cuda")
     wb = torch.empty((16, 8192), dtype=torch.int8, device="cuda")

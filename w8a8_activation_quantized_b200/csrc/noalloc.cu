@@ -15,13 +15,15 @@
 namespace cider {
 namespace {
 
-// Room for q [M][K] int8 plus scale_x [M] fp32, each 256-byte aligned.
+// Room for q [M][K] int8 plus scale_x [M] fp32, each 256-byte aligned, and,
+// when they fit after those, the fp32 partial sums of tiles cut along K.
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 
 // Shared by every call on a device: it keeps whatever the last call wrote.
 // Nothing in it needs to start at zero: each call writes the M rows of codes
 // and the M scales it reads, and the GEMM never reads rows beyond M (its tile
-// loads fill those with zeros).
+// loads fill those with zeros); every K piece of a split tile stores its whole
+// partial-sum slot before the reduce kernel reads it.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
