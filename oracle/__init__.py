@@ -69,6 +69,7 @@ def _bind(path):
         "oracle_dequant_pg": (None, [_ptr, _ptr, _ptr, _i64, _i64, _i64, _int, _ptr]),
         "oracle_linear_pc": (_int, [_ptr, _int, _i64, _i64, _ptr, _ptr, _i64, _int, _ptr]),
         "oracle_w8a16_linear_pc": (_int, [_ptr, _int, _i64, _i64, _ptr, _ptr, _i64, _int, _ptr]),
+        "oracle_w8a16_linear_pg": (_int, [_ptr, _int, _i64, _i64, _ptr, _ptr, _i64, _i64, _int, _ptr]),
         "oracle_linear_pg": (_int, [_ptr, _int, _i64, _i64, _ptr, _ptr, _i64, _i64, _int, _ptr]),
         "oracle_w4a8_linear_pg": (_int, [_ptr, _int, _i64, _i64, _ptr, _ptr, _i64, _i64, _int,
                                          _ptr, _ptr]),
@@ -298,6 +299,21 @@ def w8a16_linear_pc(x, w, sw, xdt=F16, ydt=F16):
     N = w.shape[0]
     y = np.empty((M, N), np.uint16)
     _load().oracle_w8a16_linear_pc(_p(b), xdt, M, K, _p(w), _p(sw), N, ydt, _p(y))
+    return y
+
+
+def w8a16_linear_pg(x, w, sw, gs, xdt=F16, ydt=F16):
+    """W8A16 decode product with per-group weight scales (sw [N, K/gs]), no
+    activation quantization: y = round(sum_g sw[n,g] * sum_{k in g} x[m,k] *
+    w[n,k]) in fp64.  Returns fp16/bf16 bit patterns [M,N]."""
+    b = _bits(x, xdt)
+    w, sw = _c(w, np.int8), _c(sw, np.float32)
+    M, K = b.shape
+    N = w.shape[0]
+    if gs < 1 or K % gs or sw.shape != (N, K // gs):
+        raise ValueError("gs must divide K and sw must be [N, K/gs]")
+    y = np.empty((M, N), np.uint16)
+    _load().oracle_w8a16_linear_pg(_p(b), xdt, M, K, _p(w), _p(sw), N, gs, ydt, _p(y))
     return y
 
 

@@ -463,6 +463,33 @@ int oracle_w8a16_linear_pc(const uint16_t* x, int xdt, int64_t M, int64_t K, con
     return 0;
 }
 
+/* W8A16 decode product, per-group weight scales sw[n][K/gs] ([README]
+ * section "Metal Kernel 流水线", Decode, and the per-group INT8 MV kernel of the
+ * project's kernel list): the weights of group g of row n are dequantized by
+ * sw[n][g] on the fly, the activations are used as they are:
+ * y[m,n] = round(sum_g sw[n][g] * sum_{k in g} x[m,k] * w[n,k]), x widened
+ * exactly, each group's sum and the sum over groups (ascending g) in fp64,
+ * one rounding to the output type. */
+int oracle_w8a16_linear_pg(const uint16_t* x, int xdt, int64_t M, int64_t K, const int8_t* w,
+                           const float* sw, int64_t N, int64_t gs, int ydt, uint16_t* y)
+{
+    const int64_t G = K / gs;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double sum = 0.0;
+            for (int64_t g = 0; g < G; ++g) {
+                double part = 0.0;
+                for (int64_t k = g * gs; k < (g + 1) * gs; ++k)
+                    part += (double)widen(x, m * K + k, xdt) * (double)w[n * K + k];
+                sum += (double)sw[n * G + g] * part;
+            }
+            y[m * N + n] = narrow(sum, ydt);
+        }
+    }
+    return 0;
+}
+
 /* W8A8, per-group weight scales sw[n][K/gs]. */
 int oracle_linear_pg(const uint16_t* x, int xdt, int64_t M, int64_t K, const int8_t* w,
                      const float* sw, int64_t N, int64_t gs, int ydt, uint16_t* y)

@@ -33,8 +33,11 @@ MUTATIONS = {
     "weight_scale_divisor_128": ("quantize_slab(W + n * K, K, 127.0f,", "quantize_slab(W + n * K, K, 128.0f,"),
     "pg_group_offset_dropped": ("quantize_slab(W + n * K + g * gs, gs,", "quantize_slab(W + n * K, gs,"),
     "w8a16_scale_dropped": ("y[m * N + n] = narrow(a * (double)sw[n], ydt);", "y[m * N + n] = narrow(a, ydt);"),
-    "w8a16_weight_sign_dropped": ("(double)widen(x, m * K + k, xdt) * (double)w[n * K + k];",
-                                  "(double)widen(x, m * K + k, xdt) * fabs((double)w[n * K + k]);"),
+    "w8a16_weight_sign_dropped": ("a += (double)widen(x, m * K + k, xdt) * (double)w[n * K + k];",
+                                  "a += (double)widen(x, m * K + k, xdt) * fabs((double)w[n * K + k]);"),
+    "w8a16_pg_first_group_scale_only": ("sum += (double)sw[n * G + g] * part;", "sum += (double)sw[n * G] * part;"),
+    "w8a16_pg_group_offset_dropped": ("for (int64_t k = g * gs; k < (g + 1) * gs; ++k)\n                    part +=",
+                                      "for (int64_t k = 0; k < gs; ++k)\n                    part +="),
     "clip_interpolation_sign": ("v = a[i] + td;", "v = a[i] - td;"),
     "clip_position_uses_len": ("double pos = p / 100.0 * (double)(len - 1);", "double pos = p / 100.0 * (double)len;"),
     "clip_asymmetric_128": ("clamp_int(oracle_round_half_away(w[k] / s), -127, 127)",
@@ -49,6 +52,7 @@ PINS = [
     golden_tests.test_w4a8_worked_example,
     lambda _golden: inv_tests.test_nibble_round_trip_all_bytes(),
     lambda _golden: w8a16_tests.test_w8a16_worked_example(),
+    lambda _golden: w8a16_tests.test_w8a16_pg_worked_example(),
     lambda _golden: clip_tests.test_clip_pc_worked_example_p90(),
     lambda _golden: clip_tests.test_clip_pc_worked_example_interpolated(),
     lambda _golden: clip_tests.test_clip_pg_worked_example(),
