@@ -378,37 +378,69 @@ def run_cider(args):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": f"w8a8_linear_pc M={M} N={N} K={K} fp16 in/out (quantize + tcgen05 GEMM + dequant)",
-                   "x": "fp16 N(0,1), 1% of input channels x50", "w": "N(0,0.02) -> int8 per output channel",
+                   "inputs": "x fp16 N(0,1) with 1% of channels x50; w N(0,0.02) -> int8 per channel",
                    "parallelism": f"{ws} independent replicas" if ws > 1 else "single GPU",
-                   "l2": f"inputs larger than L2: {n_sets} rotating input sets, {n_sets * set_bytes / 2**20:.0f} MiB",
-                   "launch": "K steps captured in one CUDA graph, replayed once in the timed region"},
-        "tops_per_gpu": value / ws, "pct_int8_peak": 100.0 * (value / ws) / int8_peak,
+                   "l2": f"inputs larger than L2: {n_sets} rotating sets, {n_sets * set_bytes / 2**20:.0f} MiB",
+                   "launch": "K steps in one CUDA graph, replayed once in the timed region"},
+        "pct_int8_peak": 100.0 * (value / ws) / int8_peak,
         "breakdown_ms": {"quantize_act": ms_quant, "gemm_pc": ms_gemm},
-        "roofline": {"bound": "tensor", "kernel": "k_gemm_pair per-channel (tcgen05.mma.cta_group::2 kind::i8)",
+        "roofline": {"bound": "tensor", "kernel": "k_gemm_pair (tcgen05.mma.cta_group::2 kind::i8)",
                      "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
-                     "traffic": gemm_traffic(), "traffic_unit": "bytes per launch (ncu dram read+write)",
-                     "algorithmic_bytes": M * K + N * K + M * N * 2 + 4 * (M + N),
-                     "peak_note": f"dense INT8 = {INT8_PER_BF16:g} x {pk['src']} bf16 cuBLAS burst {pk['bf16']:.1f} TFLOP/s"},
+                     "traffic": gemm_traffic(), "algorithmic_bytes": M * K + N * K + M * N * 2 + 4 * (M + N),
+                     "peak_note": f"INT8 = {INT8_PER_BF16:g} x {pk['src']} bf16 burst {pk['bf16']:.1f} TFLOP/s"},
         "e2e": {"value": e2e_tops, "unit": UNIT, "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": x0.numel() * 2, "d2h_bytes_per_step": M * N * 2,
-                "pipeline": f"{n_chunks} row chunks over copy-in / compute / copy-out streams"},
+                "pipeline": f"{n_chunks} row chunks, copy-in / compute / copy-out streams"},
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
+    rows = []
     if not args.no_rows:
         try:
-            line["rows"] = bench_rows(device, pk, steps=min(args.steps, 100), warmup=args.warmup)
+            rows = bench_rows(device, pk, steps=min(args.steps, 100), warmup=args.warmup)
         except Exception as e:  # a failing extra row must not cost the headline line
             line["rows_error"] = f"{type(e).__name__}: {e}"
     cider.cider_device_status()
     if rank == 0 and ws == 1:
         line["cpu_baseline"] = None if args.no_cpu_baseline else cpu_baseline(M, N, K, SEED0)
     if rank == 0:
+        # every row in full, then a compact summary, then the headline last
+        for r in rows:
+            print(json.dumps({"bench_row": r}), flush=True)
+        if rows:
+            print(json.dumps({"rows_summary_us_frac": rows_summary(rows)}), flush=True)
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def row_key(r):
+    """Short name of a bench row: kind, parameters and shape."""
+    n = r["row"]
+    if n == "w8a8_linear_pc":
+        return f"pc M{r['M']}"
+    if n == "w8a8_linear_pg":
+        return f"pg{r['gs']} M{r['M']}"
+    if n == "w4a8_linear_pg":
+        return f"w4pg{r['gs']} M{r['M']}"
+    if n == "w4a8_linear_pc":
+        return f"w4pc M{r['M']}"
+    if n in ("w8a16_mv_pc", "w8a16_mv_pg"):
+        return n.replace("w8a16_", "") + (f"{r['gs']}" if r.get("gs") else "") + f" M{r['M']}"
+    if n == "quantize_act":
+        return f"quant {r['M']}x{r['K']}"
+    if n == "sdpa_decode":
+        return f"sdpa {r['H_q']}/{r['H_kv']} N{r['N']}"
+    if n == "decoder_linear_stack":
+        return "stack8b"
+    return n + (f" M{r['M']}" if "M" in r else "")
+
+
+def rows_summary(rows):
+    """{short name: [microseconds per call, fraction of the row's roofline]}."""
+    return {row_key(r): [round(r["ms"] * 1e3, 2), round(r["frac"], 3)] for r in rows}
 
 
 def bench_rows(device, pk, steps, warmup):
@@ -466,7 +498,15 @@ def bench_rows(device, pk, steps, warmup):
             record("w8a8_linear_pg", ms, 2.0 * M * N * K, N * K + sg.numel() * 4 + M * K * 2 + M * N * 2,
                    gs=gs, M=M, N=N, K=K)
             del wgs, ys
-        del wg, sg
+        # W8A16 decode product with per-group scales (no activation quantization), M=1
+        x1 = torch.from_numpy(synth.activations(1, K, 2001)).to(device)
+        n = rotating(N * K)
+        wgs = [wg] + [wg.roll(i, 0).contiguous() for i in range(1, n)]
+        y1 = torch.empty((1, N), dtype=torch.float16, device=device)
+        ms = graph_time(lambda i: cider.cider_w8a16_mv_pg(x1, wgs[i % n], sg, gs, y=y1), steps, warmup)
+        record("w8a16_mv_pg", ms, 2.0 * N * K, N * K + sg.numel() * 4 + K * 2 + N * 2, gs=gs, M=1, N=N, K=K,
+               path="W8A16 per-group decode kernel (no activation quantization)")
+        del wgs, wg, sg
     del W
     # W4A8, N=12288 K=4096 M=2048 gs=64
     M, N, K, gs = 2048, 12288, 4096, 64
@@ -558,12 +598,17 @@ ROW_CASES = {
     "pc_m1024": ("pc", 1024, 10240, 2560, 0), "pc_m4096": ("pc", 4096, 10240, 2560, 0),
     "pc_m8192": ("pc", 8192, 10240, 2560, 0),
     "pg128_m1": ("pg", 1, 2560, 10240, 128), "pg128_m4096": ("pg", 4096, 2560, 10240, 128),
-    "mv_m1": ("mv", 1, 10240, 2560, 0),
+    "mv_m1": ("mv", 1, 10240, 2560, 0), "mvpg64_m1": ("mvpg", 1, 2560, 10240, 64),
+    "mvpg128_m1": ("mvpg", 1, 2560, 10240, 128),
     "pg64_m1": ("pg", 1, 2560, 10240, 64), "pg64_m4096": ("pg", 4096, 2560, 10240, 64),
     "pg128_m128": ("pg", 128, 2560, 10240, 128), "pg64_m128": ("pg", 128, 2560, 10240, 64),
     "pg64_m1024": ("pg", 1024, 2560, 10240, 64), 
     "w4a8_m2048": ("w4", 2048, 12288, 4096, 64), "w4a8pc_m2048": ("w4pc", 2048, 12288, 4096, 0),
     "stack_8b": ("stack", 2048, 0, 0, 0),
+    "quant_m4096_k2560": ("quant", 4096, 0, 2560, 0), "quant_m8192_k10240": ("quant", 8192, 0, 10240, 0),
+    # decode attention: (kind, H_kv, N keys, 0, 0) with H_q = 32, D = 128
+    "sdpa_mha_n32k": ("sdpa", 32, 32768, 0, 0), "sdpa_gqa4_n32k": ("sdpa", 8, 32768, 0, 0),
+    "sdpa_gqa8_n32k": ("sdpa", 4, 32768, 0, 0), "sdpa_gqa8_n4k": ("sdpa", 4, 4096, 0, 0),
 }
 
 
@@ -578,6 +623,36 @@ def run_row(args):
     kind, M, N, K, gs = ROW_CASES[args.row]
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
+    cider.cider_test_set_fused_quantize({"auto": 0, "off": 1, "on": 2}[args.fused])
+    if kind == "sdpa":  # decode attention alone, K/V rotated beyond L2
+        H_q, H_kv, Nk, D = 32, M, N, 128
+        kv_bytes = 2 * H_kv * Nk * D * 2
+        n = rotating(kv_bytes)
+        g = torch.Generator(device=device)
+        g.manual_seed(5000 + H_kv + Nk)
+        q = torch.randn((H_q, D), generator=g, device=device).half()
+        ks = [torch.randn((H_kv, Nk, D), generator=g, device=device).half() for _ in range(n)]
+        vs = [torch.randn((H_kv, Nk, D), generator=g, device=device).half() for _ in range(n)]
+        out = torch.empty((H_q, D), dtype=torch.float16, device=device)
+        wsd = torch.empty((max(16, cider.cider_sdpa_decode_workspace_bytes(H_q, H_kv, Nk, D)),), dtype=torch.uint8,
+                          device=device)
+        ms = graph_time(lambda i: cider.cider_sdpa_decode(q, ks[i % n], vs[i % n], out=out, workspace=wsd),
+                        args.steps, args.warmup)
+        cider.cider_device_status()
+        print(json.dumps({"row": args.row, "kind": kind, "H_q": H_q, "H_kv": H_kv, "N": Nk, "ms": ms,
+                          "GB/s": (kv_bytes + 2 * H_q * D * 2) / (ms * 1e-3) / 1e9}), flush=True)
+        return 0
+    if kind == "quant":  # activation quantization alone, inputs rotated beyond L2
+        n = rotating(M * K * 3)
+        xs = [torch.from_numpy(synth.activations(M, K, 7 + i)).to(device) for i in range(min(n, 4))]
+        qb = [torch.empty((M, K), dtype=torch.int8, device=device) for _ in range(len(xs))]
+        sb = torch.empty((M,), dtype=torch.float32, device=device)
+        ms = graph_time(lambda i: cider.cider_quantize_act(xs[i % len(xs)], q=qb[i % len(xs)], scale_x=sb),
+                        args.steps, args.warmup)
+        cider.cider_device_status()
+        print(json.dumps({"row": args.row, "kind": kind, "M": M, "K": K, "ms": ms,
+                          "GB/s": (M * K * 3 + M * 4) / (ms * 1e-3) / 1e9}), flush=True)
+        return 0
     x = torch.from_numpy(synth.activations(M, K, 1000 + M)).to(device)
     W = torch.from_numpy(synth.weights(N, K, 1001)).to(device)
     if kind == "pc":
@@ -589,6 +664,9 @@ def run_row(args):
     elif kind == "pg":
         w, s = cider.cider_quantize_weight_pg(W, gs)
         call = lambda y, ws_: cider.cider_w8a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)
+    elif kind == "mvpg":
+        w, s = cider.cider_quantize_weight_pg(W, gs)
+        call = lambda y, ws_: cider.cider_w8a16_mv_pg(x, w, s, gs, y=y)
     elif kind == "w4pc":
         w, s = cider.cider_pack_weight_int4_pc(W)
         call = lambda y, ws_: cider.cider_w4a8_linear_pc(x, w, s, y=y, workspace=ws_)
@@ -614,6 +692,8 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--row", choices=sorted(ROW_CASES), help="time one hot-path row alone (for profiling)")
+    ap.add_argument("--fused", choices=["auto", "off", "on"], default="auto",
+                    help="with --row: where the per-channel linear quantizes (inside the GEMM launch or not)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

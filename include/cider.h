@@ -22,7 +22,9 @@
  *    enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream)
  *    and returns as soon as its kernels are launched.
  *  - Layouts are dense row-major: x [M][K], w [N][K] (nn.Linear convention:
- *    output channel n, input channel k), y [M][N], q [M][K].  Per-group weight
+ *    output channel n, input channel k), y [M][N], q [M][K]; only
+ *    cider_quantize_act takes row strides.  A strided input goes through
+ *    cider_quantize_act into a dense q and then a *_gemm_*_q entry point.  Per-group weight
  *    scales are GROUP-MAJOR, scale_w[K/gs][N], so that one group's scales for
  *    consecutive output channels are contiguous.  Packed INT4 weights are
  *    [N][K/2] bytes; byte j of row n holds k = 2j in its low nibble and
@@ -123,9 +125,14 @@ CIDER_API int64_t cider_get_small_m_threshold(void);
 /* Online per-token activation quantization (Cider README, section
  * "Metal Kernel 流水线", step quantize_per_token; juejin post, section
  * "W8A8 对称量化：Cider 的选择").
- * x: [M][K] fp16/bf16 (xdt); q: [M][K] int8 out; scale_x: [M] fp32 out. */
-CIDER_API cider_status_t cider_quantize_act(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
-                                  int8_t* q, float* scale_x, void* stream);
+ * x: M rows of K fp16/bf16 values (xdt), row m at x + m * ldx elements;
+ * q: M rows of K int8 codes out, row m at q + m * ldq bytes; scale_x: [M]
+ * fp32 out.  The row strides let a caller quantize a strided view, such as
+ * a slice of a fused buffer: ldx >= K, a multiple of 8 (16-byte rows);
+ * ldq >= K, a multiple of 16.  The bytes between K and the stride are neither
+ * read (x) nor written (q).  x, q and scale_x must not overlap. */
+CIDER_API cider_status_t cider_quantize_act(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, int64_t ldx,
+                                  int8_t* q, int64_t ldq, float* scale_x, void* stream);
 
 /* W8A8 linear, per-output-channel weight scales (Cider README, section
  * "底层 API" perchannel_linear; table "W8A8 量化粒度", Per-channel).
@@ -148,6 +155,23 @@ CIDER_API cider_status_t cider_w8a8_linear_pc(const void* x, cider_dtype_t xdt, 
  * scale_w: [N] fp32; y: [M][N] (ydt).  No workspace. */
 CIDER_API cider_status_t cider_w8a16_mv_pc(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
                                  const int8_t* w, const float* scale_w, int64_t N,
+                                 void* y, cider_dtype_t ydt, void* stream);
+
+/* W8A16 decode matrix-vector product, per-group weight scales along K (gs =
+ * 64 or 128): the pages' per-group INT8 MV decode kernel (Cider README,
+ * section "Metal Kernel 流水线", Decode, and the per-group MV kernel of its
+ * kernel list).  y[m,n] = round_ydt(sum_g scale_w[g][n] * sum_{k in g}
+ * x[m,k] * w[n,k]) with x widened to fp32, each chunk of 16 products summed
+ * in fp32, scaled by its group's scale and accumulated in fp32; the
+ * activations are NOT quantized.  x: [M][K] (xdt), 1 <= M <= 4, K <= 32768;
+ * w: [N][K] int8; scale_w: [K/gs][N] fp32 (group-major, as for the per-group
+ * linears); y: [M][N] (ydt).  No workspace.  Besides the common checks,
+ * CIDER_ERR_INVALID_ARG when gs is not 64 or 128 or does not divide K, or
+ * when the shape's staged activations (M * K * 4 bytes), the group scales of
+ * one SM's share of the rows and three weight stages exceed the shared
+ * memory of an SM. */
+CIDER_API cider_status_t cider_w8a16_mv_pg(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
+                                 const int8_t* w, const float* scale_w, int64_t N, int64_t gs,
                                  void* y, cider_dtype_t ydt, void* stream);
 
 /* W8A8 linear, per-group weight scales along K (gs = 64 or 128; Cider README,
@@ -304,9 +328,21 @@ CIDER_API cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8
                                            int64_t K, int64_t gs, int32_t* acc_g, void* stream);
 /* Forces the kernel variant of the per-channel and INT32 GEMM for later calls
  * (process-wide): 0 = automatic (default), 1 = single-CTA 128x128 tiles,
- * 2 = single-CTA 128x256 tiles, 3 = CTA-pair 256x256 tiles.  Lets tests cover
- * every variant on small shapes. */
+ * 2 = single-CTA 128x256 tiles, 3 = CTA-pair 256x256 tiles, 4 = single-CTA
+ * 128x80 tiles.  Lets tests cover every variant on small shapes. */
 CIDER_API cider_status_t cider_test_set_gemm_variant(int variant);
+/* Selects, for later calls (process-wide), how the per-channel linear
+ * (cider_w8a8_linear_pc and the workspace-free form) quantizes its
+ * activations on the tensor-core path: 0 = automatic (default: inside the
+ * GEMM launch for M <= 1024, by the separate quantize kernel above), 1 =
+ * always the separate kernel, 2 = always inside the GEMM launch.  Either way
+ * the call leaves the codes q [M][K] at the start of the workspace and
+ * scale_x [M] at byte offset align256(M * K), which lets tests check the
+ * fused quantization bit for bit.  The fused launch synchronises its grid
+ * once (one CTA per SM, all resident); it needs the GPU's SMs to itself for
+ * that moment, and a barrier that cannot complete within 2 s records
+ * CIDER_ERR_TIMEOUT for cider_device_status(). */
+CIDER_API cider_status_t cider_test_set_fused_quantize(int mode);
 /* Forces the split-K piece count of the per-group GEMM for later calls
  * (process-wide): 0 = automatic (default), 1 = never split, 2 .. 16 = that
  * many K pieces per tile (fewer when K has fewer 128-wide blocks).  The INT32

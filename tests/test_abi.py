@@ -175,3 +175,29 @@ def test_w4pc_workspace_covers_small_m(lib):
     # the per-column W4A8 form has no decode kernel: even M = 1 needs q and scale_x
     assert lib.cider_workspace_bytes_w4a8_pc(1, 256, 1024) >= 1024 + 256
     assert lib.cider_workspace_bytes_w4a8_pc(0, 256, 1024) == 0
+
+
+def _quant(lib, **kw):
+    a = dict(x=P, xdt=0, M=4, K=64, ldx=64, q=ctypes.c_void_p(1 << 20), ldq=64, sx=ctypes.c_void_p(1 << 21), st=None)
+    a.update(kw)
+    return lib.cider_quantize_act(a["x"], a["xdt"], a["M"], a["K"], a["ldx"], a["q"], a["ldq"], a["sx"], a["st"])
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(ldx=48), "ldx < K"),
+    (dict(ldq=32), "ldq < K"),
+    (dict(ldx=68), "ldx not a multiple of 8"),
+    (dict(ldq=72), "ldq not a multiple of 16"),
+    (dict(K=40, ldx=40, ldq=48), "K % 16"),
+    (dict(ldx=128, q=ctypes.c_void_p(256 + 3 * 128 * 2)), "q inside the strided span of x"),
+])
+def test_quantize_act_stride_checks(lib, kw, why):
+    assert _quant(lib, **kw) == 1, why
+    assert lib.cider_last_error()
+
+
+def test_quantize_act_strided_span_allows_q_past_it(lib):
+    # x rows 0..3 at stride 128 span (3 * 128 + 64) * 2 bytes from 256; q right after is legal,
+    # and the call then fails only for want of a device (not an argument error)
+    q = ctypes.c_void_p(256 + (3 * 128 + 64) * 2 + 16 * 40)
+    assert _quant(lib, ldx=128, q=q) in (2, 3)

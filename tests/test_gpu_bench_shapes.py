@@ -108,3 +108,13 @@ def test_w8a16_mv_pc_bench_shape(pc_weights):
     y = cider.cider_w8a16_mv_pc(dev(x), dev(qw), dev(sw))
     torch.cuda.synchronize()
     check_y(y, oracle.w8a16_linear_pc(x, qw, sw), F16)
+
+
+@pytest.mark.parametrize("gs", [128, 64])
+def test_w8a16_mv_pg_bench_shape(gs, pg_weights):
+    N, K = 2560, 10240
+    qw, sw = pg_weights[gs]
+    x = synth.activations(1, K, 2001)
+    y = cider.cider_w8a16_mv_pg(dev(x), dev(qw), dev(np.ascontiguousarray(sw.T)), gs)
+    torch.cuda.synchronize()
+    check_y(y, oracle.w8a16_linear_pg(x, qw, sw, gs), F16)

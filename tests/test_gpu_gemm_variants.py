@@ -1,5 +1,5 @@
 """Every kernel variant of the per-channel GEMM against the oracle on small and
-ragged shapes: single-CTA 128x128 and 128x256 tiles, and the CTA-pair
+ragged shapes: single-CTA 128x80, 128x128 and 128x256 tiles, and the CTA-pair
 256x256 tile (tcgen05.mma.cta_group::2).  Bit-exact INT32 accumulators, and
 the fused dequant within the row-relative tolerance."""
 import numpy as np
@@ -13,7 +13,7 @@ from tests.parity import act, check_y, dev, dev_bits
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = {"single128": 1, "single256": 2, "pair256": 3}
+VARIANTS = {"single128": 1, "single256": 2, "pair256": 3, "single80": 4}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -121,3 +121,25 @@ def test_linear_pc_tail_split_automatic(dt):
     assert torch.equal(y_auto, y_plain)
     rows = np.arange(0, M, 37)
     check_y(y_auto, oracle.linear_pc(x[rows], qw, sw, xdt=dt, ydt=dt), dt, rows=rows)
+
+
+def test_mid_m_variants_agree_bit_for_bit():
+    """M = 128, N = 10240 (the pages' table shape) takes the 128 x 80 tile by
+    default (128 tiles in one round on 148 SMs); the INT32 sums are exact and
+    the dequant expression is the same in every variant, so the 128 x 80,
+    128 x 128 and 128 x 256 results are equal bit for bit."""
+    M, N, K = 128, 10240, 2560
+    cider.cider_set_small_m_threshold(4)
+    x = act(M, K, seed=128)
+    qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed=129))
+    xd, wd, sd = dev_bits(x, oracle.F16), dev(qw), dev(sw)
+    outs = {}
+    for name, v in (("auto", 0), ("single80", 4), ("single128", 1), ("single256", 2)):
+        cider.cider_test_set_gemm_variant(v)
+        outs[name] = cider.cider_w8a8_linear_pc(xd, wd, sd)
+    cider.cider_test_set_gemm_variant(0)
+    torch.cuda.synchronize()
+    for name in ("single80", "single128", "single256"):
+        assert torch.equal(outs[name], outs["auto"]), name
+    rows = np.arange(0, M, 9)
+    check_y(outs["auto"], oracle.linear_pc(x[rows], qw, sw), oracle.F16, rows=rows)

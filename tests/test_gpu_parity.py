@@ -54,6 +54,24 @@ def test_quantize_act_bitexact(M, K, dt):
     np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
 
 
+@pytest.mark.parametrize("dt", [F16, BF16])
+def test_quantize_act_row_strides(dt):
+    """A strided view (a slice of a wider buffer) quantizes to the same codes and
+    scales as the oracle on those rows, into a strided q; the bytes between K
+    and the stride of q are left untouched."""
+    M, K, LDX, LDQ = 37, 1024, 1536, 1040
+    wide = act(M, LDX, seed=41, dt=dt)
+    xs = wide[:, 256:256 + K]
+    qbuf = torch.full((M, LDQ), 77, dtype=torch.int8, device="cuda")
+    xd = dev_bits(wide, dt)[:, 256:256 + K]
+    q, s = cider.cider_quantize_act(xd, q=qbuf[:, :K])
+    torch.cuda.synchronize()
+    qo, so = oracle.quantize_act(np.ascontiguousarray(xs), dt)
+    np.testing.assert_array_equal(qbuf[:, :K].cpu().numpy(), qo)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    assert bool((qbuf[:, K:] == 77).all())
+
+
 def test_quantize_act_ties_and_extremes():
     K = 64
     rows = np.zeros((4, K), np.float32)
@@ -67,6 +85,25 @@ def test_quantize_act_ties_and_extremes():
     np.testing.assert_array_equal(s.cpu().numpy(), s_ref)
     np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
     assert list(q_ref[0, :8]) == [127, 3, -3, 1, -1, 127, -127, 2]
+
+
+def test_quantize_act_bf16_ties_and_extremes():
+    """bf16 tokens at the ends of the fp32 range, where the fast path's
+    reciprocal of the scale is huge or infinite: bit-exact codes and scales."""
+    K = 64
+    rows = np.zeros((5, K), np.float64)
+    rows[0, :8] = [127, 2.5, -2.5, 0.5, -0.5, 126.5, -126.5, 1.5]   # exact .5 ties, scale 1
+    rows[1, :4] = [1e-37, -3e-38, 5e-38, 7.1e-38]                    # amax ~1e-37: a subnormal scale, 1/scale = inf
+    rows[2, :4] = [2.0 ** -130, -(2.0 ** -131), 2.0 ** -133, 0.0]    # subnormal-only token
+    rows[3, :4] = [3.38e38, -3.38e38, 1.0, 2.0e38]                   # near the largest bf16
+    rows[4, :4] = [4e-36, -1.3e-36, 2.2e-36, 0.9e-36]                # scale ~3e-38: 1/scale finite and huge
+    x = oracle.narrow(rows, BF16)
+    q_ref, s_ref = oracle.quantize_act(x, BF16)
+    q, s = cider.cider_quantize_act(dev_bits(x, BF16))
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
+    assert list(q_ref[0, :8]) == [127, 3, -3, 1, -1, 127, -127, 2]
+    assert s_ref[1] > 0 and s_ref[1] < np.finfo(np.float32).tiny  # the subnormal-scale case is exercised
 
 
 # ---------------------------------------------------------------- offline weight quantization

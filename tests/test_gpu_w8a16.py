@@ -1,7 +1,9 @@
-"""The W8A16 decode kernel (no activation quantization; Cider README, section
-"Metal Kernel 流水线", Decode) against the oracle's W8A16 mode, within the
-row-relative tolerance, for 1 <= M <= 4, both input dtypes and both output
-dtypes, including shapes whose K is split across warps."""
+"""The W8A16 decode kernels (no activation quantization; Cider README, section
+"Metal Kernel 流水线", Decode: the per-channel and the per-group INT8 MV
+kernels) against the oracle's W8A16 modes, within the row-relative
+tolerance, for 1 <= M <= 4, both input dtypes and both output dtypes,
+including shapes whose K is split across warps, whose rows wrap the ring of
+shared-memory stages, and the argument checks."""
 import numpy as np
 import pytest
 import torch
@@ -55,3 +57,76 @@ def test_w8a16_mv_zero_token_and_argument_checks():
     with pytest.raises(cider.CiderError):  # activation rows must fit in shared memory
         cider.cider_w8a16_mv_pc(dev_bits(act(4, 16384, seed=1), oracle.F16),
                                 dev(np.zeros((8, 16384), np.int8)), dev(np.ones(8, np.float32)))
+
+
+# ---- per-group weight scales (cider_w8a16_mv_pg) ---------------------------------
+
+def _pg_plan_fits(M, N, K, gs, num_sms):
+    """The kernel's shared-memory plan: stages of R rows (R * K <= 24 KB), one
+    CTA per SM on min(num_sms, N / R) CTAs; fp32 activation pairs of whole
+    512-weight passes, the group scales of the CTA's rows and the slice
+    partials (each rounded up to 128 bytes), then at least three stages in
+    225 KB."""
+    al = lambda v: (v + 127) // 128 * 128
+    R = 8
+    while R > 1 and R * K > 24 * 1024:
+        R //= 2
+    S = 8 // R
+    grid = min(num_sms, max(1, N // R))
+    rows_max = -(-N // grid)
+    used = al(M * ((K // 16 + 31) // 32) * 2048) + al((K // gs) * rows_max * 4) + al(rows_max * S * M * 4)
+    return used < 225 * 1024 and (225 * 1024 - used) // (R * K) >= 3
+
+
+@pytest.mark.parametrize("M", [1, 2, 4])
+@pytest.mark.parametrize("N,K,gs", [(2560, 10240, 64), (2560, 10240, 128), (10240, 2560, 64), (264, 1088, 64),
+                                    (20480, 1024, 128), (8, 64, 64), (136, 32768, 128), (136, 16384, 128)])
+def test_w8a16_mv_pg(M, N, K, gs):
+    x = act(M, K, seed=M + N + K + gs)
+    qw, sw = oracle.quantize_weight_pg(synth.weights(N, K, seed=N + K + gs), gs)
+    args = (dev_bits(x, oracle.F16), dev(qw), dev(np.ascontiguousarray(sw.T)), gs)
+    if not _pg_plan_fits(M, N, K, gs, torch.cuda.get_device_properties(0).multi_processor_count):
+        with pytest.raises(cider.CiderError, match="shared memory"):
+            cider.cider_w8a16_mv_pg(*args)
+        return
+    y = cider.cider_w8a16_mv_pg(*args)
+    check_y(y, oracle.w8a16_linear_pg(x, qw, sw, gs), oracle.F16)
+
+
+@pytest.mark.parametrize("xdt,ydt", [(oracle.BF16, oracle.BF16), (oracle.F16, oracle.BF16)])
+def test_w8a16_mv_pg_dtypes_and_zero_token(xdt, ydt):
+    M, N, K, gs = 3, 1032, 4096, 64
+    x = act(M, K, seed=19, dt=xdt)
+    x[2] = 0
+    qw, sw = oracle.quantize_weight_pg(synth.weights(N, K, seed=20), gs)
+    out = torch.bfloat16 if ydt == oracle.BF16 else torch.float16
+    y = cider.cider_w8a16_mv_pg(dev_bits(x, xdt), dev(qw), dev(np.ascontiguousarray(sw.T)), gs, out_dtype=out)
+    check_y(y, oracle.w8a16_linear_pg(x, qw, sw, gs, xdt=xdt, ydt=ydt), ydt)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(y[2]).item() == 0
+
+
+def test_w8a16_mv_pg_one_group_equals_per_channel_kernel_shape():
+    """With gs = 128 = K the per-group product is the per-channel one; both
+    kernels must agree with the oracle on the same inputs."""
+    M, N, K = 2, 264, 128
+    x = act(M, K, seed=21)
+    qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed=22))
+    y_pg = cider.cider_w8a16_mv_pg(dev_bits(x, oracle.F16), dev(qw), dev(sw[None, :].copy()), 128)
+    y_pc = cider.cider_w8a16_mv_pc(dev_bits(x, oracle.F16), dev(qw), dev(sw))
+    ref = oracle.w8a16_linear_pc(x, qw, sw)
+    check_y(y_pg, ref, oracle.F16)
+    check_y(y_pc, ref, oracle.F16)
+
+
+def test_w8a16_mv_pg_argument_checks():
+    N, K = 264, 1024
+    x = dev_bits(act(1, K, seed=1), oracle.F16)
+    w = dev(np.zeros((N, K), np.int8))
+    with pytest.raises(cider.CiderError):  # gs must be 64 or 128
+        cider.cider_w8a16_mv_pg(x, w, dev(np.ones((K // 32, N), np.float32)), 32)
+    with pytest.raises(cider.CiderError):  # decode shapes only
+        cider.cider_w8a16_mv_pg(dev_bits(act(5, K, seed=1), oracle.F16), w, dev(np.ones((K // 64, N), np.float32)), 64)
+    with pytest.raises(cider.CiderError):  # staged rows + scales beyond shared memory
+        cider.cider_w8a16_mv_pg(dev_bits(act(4, 10240, seed=1), oracle.F16), dev(np.zeros((40960, 10240), np.int8)),
+                                dev(np.ones((160, 40960), np.float32)), 64)

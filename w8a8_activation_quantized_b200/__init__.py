@@ -42,9 +42,10 @@ _SIGNATURES = {
     "cider_workspace_bytes_mnk": (_SZ, [_I64, _I64, _I64]),
     "cider_set_small_m_threshold": (_INT, [_I64]),
     "cider_get_small_m_threshold": (_I64, []),
-    "cider_quantize_act": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P]),
+    "cider_quantize_act": (_INT, [_P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "cider_w8a8_linear_pc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P, _SZ, _P]),
     "cider_w8a16_mv_pc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P]),
+    "cider_w8a16_mv_pg": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P]),
     "cider_w8a8_linear_pg": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P, _SZ, _P]),
     "cider_w4a8_linear_pg": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _I64, _P, _INT, _P, _SZ, _P]),
     "cider_w4a8_linear_pc": (_INT, [_P, _INT, _I64, _I64, _P, _P, _I64, _P, _INT, _P, _SZ, _P]),
@@ -69,6 +70,7 @@ _SIGNATURES = {
     "cider_test_unpack_int4": (_INT, [_P, _I64, _I64, _P, _P]),
     "cider_test_set_gemm_variant": (_INT, [_INT]),
     "cider_test_set_split_k": (_INT, [_INT]),
+    "cider_test_set_fused_quantize": (_INT, [_INT]),
     "cider_test_bounded_wait": (_INT, [_I64, _P]),
 }
 EXPORTS = tuple(_SIGNATURES)
@@ -147,13 +149,16 @@ def cider_get_small_m_threshold() -> int:
 # ---- the operations -----------------------------------------------------------
 
 def cider_quantize_act(x, q=None, scale_x=None, stream=None):
-    """x [M, K] fp16/bf16 -> (q int8 [M, K], scale_x fp32 [M])."""
-    _contig(x, "x")
+    """x [M, K] fp16/bf16 -> (q int8 [M, K], scale_x fp32 [M]).  x and q may be
+    row-strided views (unit stride along K); their row strides are passed on."""
     M, K = x.shape
+    if x.stride(1) != 1 or (q is not None and q.stride(1) != 1):
+        raise ValueError("x and q need unit stride along K")
     q = torch.empty((M, K), dtype=torch.int8, device=x.device) if q is None else q
     scale_x = torch.empty((M,), dtype=torch.float32, device=x.device) if scale_x is None else scale_x
     _check("cider_quantize_act", lib().cider_quantize_act(
-        _ptr(x), _DT[x.dtype], M, K, _ptr(q), _ptr(scale_x), _stream(stream, x.device)))
+        _ptr(x), _DT[x.dtype], M, K, x.stride(0) if M > 1 else K, _ptr(q), q.stride(0) if M > 1 else K,
+        _ptr(scale_x), _stream(stream, x.device)))
     return q, scale_x
 
 
@@ -190,6 +195,20 @@ def cider_w8a16_mv_pc(x, w, scale_w, y=None, out_dtype=None, stream=None):
     y = _out(y, M, N, out_dtype or x.dtype, x.device)
     _check("cider_w8a16_mv_pc", lib().cider_w8a16_mv_pc(
         _ptr(x), _DT[x.dtype], M, K, _ptr(w), _ptr(scale_w), N, _ptr(y), _DT[y.dtype], _stream(stream, x.device)))
+    return y
+
+
+def cider_w8a16_mv_pg(x, w, scale_w, gs, y=None, out_dtype=None, stream=None):
+    """W8A16 decode product with per-group weight scales (1 <= M <= 4):
+    y = sum_g scale_w[g, n] * sum_{k in g} x[m,k] * w[n,k], fp16/bf16 x used
+    as is; scale_w fp32 [K/gs, N] (group-major)."""
+    _contig(x, "x"), _contig(w, "w")
+    M, K = x.shape
+    N = w.shape[0]
+    y = _out(y, M, N, out_dtype or x.dtype, x.device)
+    _check("cider_w8a16_mv_pg", lib().cider_w8a16_mv_pg(
+        _ptr(x), _DT[x.dtype], M, K, _ptr(w), _ptr(scale_w), N, gs, _ptr(y), _DT[y.dtype],
+        _stream(stream, x.device)))
     return y
 
 
@@ -415,8 +434,13 @@ def cider_test_gemm_i32_grouped(q, w, gs, acc_g=None, stream=None):
 
 
 def cider_test_set_gemm_variant(variant: int):
-    """0 automatic, 1 single-CTA 128x128, 2 single-CTA 128x256, 3 CTA-pair 256x256."""
+    """0 automatic, 1 single-CTA 128x128, 2 single-CTA 128x256, 3 CTA-pair 256x256, 4 single-CTA 128x80."""
     _check("cider_test_set_gemm_variant", lib().cider_test_set_gemm_variant(variant))
+
+
+def cider_test_set_fused_quantize(mode: int):
+    """0 automatic, 1 always the separate quantize kernel, 2 always inside the GEMM launch."""
+    _check("cider_test_set_fused_quantize", lib().cider_test_set_fused_quantize(mode))
 
 
 def cider_test_set_split_k(splits: int):

@@ -148,6 +148,21 @@ cider_status_t check_mode_k(int mode, int64_t K, int64_t gs) {
 
 std::atomic<int> g_gemm_variant{kGemmAuto};  // test override
 std::atomic<int> g_split_override{0};         // test override of the split-K piece count (0 = automatic)
+std::atomic<int> g_fuse_override{0};          // test override of the fused quantize: 0 auto, 1 never, 2 always
+std::atomic<unsigned> g_fuse_next{0};         // next grid-barrier slot of a fused launch
+constexpr int64_t kFuseMaxM = 1024;           // automatic fusion up to this many tokens
+
+// The per-channel linear quantizes its activations inside the GEMM launch
+// (one launch instead of two; the first weight tiles stream while the grid
+// quantizes) for mid-size M, where the separate quantize kernel is a large,
+// latency-bound share of the call; beyond that the separate, software-
+// pipelined quantize kernel is the cheaper producer.
+bool use_fused_quantize(int mode, int64_t M) {
+    if (mode != kModePC) return false;
+    const int f = g_fuse_override.load();
+    if (f != 0) return f == 2;
+    return M <= kFuseMaxM;
+}
 constexpr int kMaxSplits = 16;
 
 int pick_variant(int64_t M, int64_t N, int num_sms);
@@ -195,20 +210,31 @@ size_t part_bytes(const SplitPlan& sp) {
 }
 
 // Per-channel GEMM variant: the CTA-pair 256x256 tile when it still gives
-// every pair of SMs a tile, else single-CTA tiles of 128x256 or 128x128.
+// every pair of SMs a tile, else single-CTA tiles of 128x256, or -- when those
+// leave SMs idle -- 128x128 or 128x80, whichever gives the busiest SM fewer
+// weight rows to stream (rounds of the persistent grid x tile width; at
+// M <= 128, N = 10240 that is one round of 128 tiles of 80 rows instead of
+// 80 tiles of 128 rows on 80 SMs).
 int pick_variant(int64_t M, int64_t N, int num_sms) {
     const int forced = g_gemm_variant.load();
     if (forced != kGemmAuto) return forced;
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
     if (M > 128 && pair_tiles >= num_sms / 2) return kGemmPair;
-    const int64_t tiles256 = ((M + 127) / 128) * ((N + 255) / 256);
-    return tiles256 < num_sms ? kGemmSingle128 : kGemmSingle256;
+    const int64_t mb = (M + 127) / 128;
+    const int64_t tiles256 = mb * ((N + 255) / 256);
+    if (tiles256 >= num_sms) return kGemmSingle256;
+    auto rows_per_sm = [&](int64_t bn) { return (mb * ((N + bn - 1) / bn) + num_sms - 1) / num_sms * bn; };
+    return rows_per_sm(80) < rows_per_sm(128) ? kGemmSingle80 : kGemmSingle128;
 }
 
 cider_status_t run_gemm(int mode, const int8_t* q, const float* sx, int64_t M, int64_t K,
                         const void* w, const float* sw, int64_t N, int64_t gs, void* y, int ydt,
-                        const DeviceInfo* d, cudaStream_t st, SplitPlan sp = {0, 1, 0, 0}, float* part = nullptr) {
+                        const DeviceInfo* d, cudaStream_t st, SplitPlan sp = {0, 1, 0, 0}, float* part = nullptr,
+                        const void* x = nullptr, int xdt = 0) {
     GemmLaunch L;
+    L.x = x;
+    L.xdt = xdt;
+    L.fuse_slot = x ? static_cast<int>(g_fuse_next.fetch_add(1u) % kFuseSlots) : 0;
     L.mode = mode;
     L.q = q;
     L.w = w;
@@ -254,7 +280,7 @@ cider_status_t linear(int mode, const void* x, int xdt, int64_t M, int64_t K, co
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (mode != kModeW4PC && small_m_path(M, K)) {  // per-channel INT4: tensor-core path at every M
         cudaError_t e = launch_small_m(mode, x, xdt, static_cast<int>(M), static_cast<int>(K), w, sw,
-                                       static_cast<int>(N), static_cast<int>(gs), y, ydt, d->num_sms, st);
+                                       static_cast<int>(N), static_cast<int>(gs), y, ydt, d->num_sms, d->status, st);
         if (e != cudaSuccess) return cuda_fail(e, "small-M kernel launch");
         return CIDER_OK;
     }
@@ -279,7 +305,9 @@ cider_status_t linear(int mode, const void* x, int xdt, int64_t M, int64_t K, co
     if (overlap(ry, rng(ws, used))) return fail(CIDER_ERR_INVALID_ARG, "y overlaps the workspace");
     int8_t* q = static_cast<int8_t*>(ws);
     float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(static_cast<size_t>(M) * K));
-    cudaError_t e = launch_quantize_act(x, xdt, M, static_cast<int>(K), q, sx, st);
+    if (use_fused_quantize(mode, M))  // one launch: the GEMM quantizes x into q / sx itself
+        return run_gemm(mode, q, sx, M, K, w, sw, N, gs, y, ydt, d, st, plan, part, x, xdt);
+    cudaError_t e = launch_quantize_act(x, xdt, M, static_cast<int>(K), K, q, K, sx, d->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
     return run_gemm(mode, q, sx, M, K, w, sw, N, gs, y, ydt, d, st, plan, part);
 }
@@ -418,26 +446,32 @@ cider_status_t cider_set_small_m_threshold(int64_t threshold) {
 
 int64_t cider_get_small_m_threshold(void) { return g_small_m_threshold.load(); }
 
-cider_status_t cider_quantize_act(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, int8_t* q,
-                                  float* scale_x, void* stream) {
+cider_status_t cider_quantize_act(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, int64_t ldx, int8_t* q,
+                                  int64_t ldq, float* scale_x, void* stream) {
     t_last_error[0] = '\0';
     if (M < 0 || K < 1) return fail(CIDER_ERR_INVALID_ARG, "M >= 0 and K >= 1 required");
     if (K % 16) return fail(CIDER_ERR_INVALID_ARG, "K = %lld must be a multiple of 16", (long long)K);
     if (K > kMaxK) return fail(CIDER_ERR_INVALID_ARG, "K exceeds %lld", (long long)kMaxK);
+    if (ldx < K || ldq < K)
+        return fail(CIDER_ERR_INVALID_ARG, "row strides ldx = %lld and ldq = %lld must be >= K = %lld", (long long)ldx,
+                    (long long)ldq, (long long)K);
+    if (ldx % 8 || ldq % 16)
+        return fail(CIDER_ERR_INVALID_ARG, "ldx must be a multiple of 8 elements and ldq of 16 bytes (16-byte rows)");
     if (xdt != CIDER_F16 && xdt != CIDER_BF16) return fail(CIDER_ERR_INVALID_ARG, "dtype %d unknown", (int)xdt);
     if (M == 0) return CIDER_OK;
     if (M > INT32_MAX) return fail(CIDER_ERR_INVALID_ARG, "M must be < 2^31");
     if (!x || !q || !scale_x) return fail(CIDER_ERR_INVALID_ARG, "NULL pointer");
     if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scale_x) & 3u))
         return fail(CIDER_ERR_INVALID_ARG, "x and q must be 16-byte aligned, scale_x 4-byte aligned");
-    const Range rx = rng(x, static_cast<size_t>(M) * K * 2);
-    if (overlap(rx, rng(q, static_cast<size_t>(M) * K)) || overlap(rx, rng(scale_x, M * 4)) ||
-        overlap(rng(q, static_cast<size_t>(M) * K), rng(scale_x, M * 4)))
+    const Range rx = rng(x, static_cast<size_t>((M - 1) * ldx + K) * 2);
+    const Range rq = rng(q, static_cast<size_t>((M - 1) * ldq + K));
+    if (overlap(rx, rq) || overlap(rx, rng(scale_x, M * 4)) || overlap(rq, rng(scale_x, M * 4)))
         return fail(CIDER_ERR_INVALID_ARG, "x, q and scale_x must not overlap");
     DeviceInfo* d = nullptr;
     cider_status_t s = device_info(&d);
     if (s != CIDER_OK) return s;
-    cudaError_t e = launch_quantize_act(x, xdt, M, static_cast<int>(K), q, scale_x, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_quantize_act(x, xdt, M, static_cast<int>(K), ldx, q, ldq, scale_x, d->num_sms,
+                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "quantize launch");
 }
 
@@ -466,8 +500,36 @@ cider_status_t cider_w8a16_mv_pc(const void* x, cider_dtype_t xdt, int64_t M, in
     DeviceInfo* d = nullptr;
     if ((s = device_info(&d)) != CIDER_OK) return s;
     cudaError_t e = launch_mv_w8a16(x, xdt, static_cast<int>(M), static_cast<int>(K), w, scale_w, static_cast<int>(N),
-                                    y, ydt, d->num_sms, static_cast<cudaStream_t>(stream));
+                                    0, y, ydt, d->num_sms, d->status, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "W8A16 decode kernel launch");
+}
+
+cider_status_t cider_w8a16_mv_pg(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, const int8_t* w,
+                                 const float* scale_w, int64_t N, int64_t gs, void* y, cider_dtype_t ydt,
+                                 void* stream) {
+    t_last_error[0] = '\0';
+    cider_status_t s = check_common(x, M, K, w, scale_w, N, y, xdt, ydt);
+    if (s != CIDER_OK) return s;
+    if ((s = check_gs(K, gs, false)) != CIDER_OK) return s;
+    if (M == 0) return CIDER_OK;
+    if (M > kMaxMvM) return fail(CIDER_ERR_INVALID_ARG, "M = %lld exceeds %d (decode shapes only)", (long long)M, kMaxMvM);
+    if (K > kSmallMaxK) return fail(CIDER_ERR_INVALID_ARG, "K = %lld exceeds %lld", (long long)K, (long long)kSmallMaxK);
+    const Range ry = rng(y, static_cast<size_t>(M) * N * 2);
+    if (overlap(ry, rng(x, static_cast<size_t>(M) * K * 2)) || overlap(ry, rng(w, static_cast<size_t>(N) * K)) ||
+        overlap(ry, rng(scale_w, static_cast<size_t>(K / gs) * N * 4)))
+        return fail(CIDER_ERR_INVALID_ARG, "y overlaps an input");
+    DeviceInfo* d = nullptr;
+    if ((s = device_info(&d)) != CIDER_OK) return s;
+    if (!mv_w8a16_bulk_fits(static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), static_cast<int>(gs),
+                            d->num_sms))
+        return fail(CIDER_ERR_INVALID_ARG,
+                    "M = %lld, K = %lld, N = %lld, gs = %lld: the staged activations, group scales and three weight "
+                    "stages do not fit in shared memory",
+                    (long long)M, (long long)K, (long long)N, (long long)gs);
+    cudaError_t e = launch_mv_w8a16(x, xdt, static_cast<int>(M), static_cast<int>(K), w, scale_w, static_cast<int>(N),
+                                    static_cast<int>(gs), y, ydt, d->num_sms, d->status,
+                                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "W8A16 per-group decode kernel launch");
 }
 
 cider_status_t cider_w8a8_linear_pg(const void* x, cider_dtype_t xdt, int64_t M, int64_t K, const int8_t* w,
@@ -695,9 +757,15 @@ cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8_t* w, int
                     sp, nullptr);
 }
 
+cider_status_t cider_test_set_fused_quantize(int mode) {
+    if (mode < 0 || mode > 2) return fail(CIDER_ERR_INVALID_ARG, "mode %d outside [0, 2]", mode);
+    g_fuse_override.store(mode);
+    return CIDER_OK;
+}
+
 cider_status_t cider_test_set_gemm_variant(int variant) {
-    if (variant < kGemmAuto || variant > kGemmPair)
-        return fail(CIDER_ERR_INVALID_ARG, "variant %d outside [0, 3]", variant);
+    if (variant < kGemmAuto || variant > kGemmSingle80)
+        return fail(CIDER_ERR_INVALID_ARG, "variant %d outside [0, 4]", variant);
     g_gemm_variant.store(variant);
     return CIDER_OK;
 }

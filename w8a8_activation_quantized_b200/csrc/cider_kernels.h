@@ -24,7 +24,12 @@ enum : int {
 
 // Kernel variants of the per-channel GEMM (the grouped modes always use the
 // single-CTA kernel with 128-wide N tiles).
-enum : int { kGemmAuto = 0, kGemmSingle128 = 1, kGemmSingle256 = 2, kGemmPair = 3 };
+enum : int { kGemmAuto = 0, kGemmSingle128 = 1, kGemmSingle256 = 2, kGemmPair = 3, kGemmSingle80 = 4 };
+
+// Grid-barrier slots of the launches that quantize inside the GEMM: the host
+// hands out slots in turn, so launches that run at the same time (up to this
+// many in flight) never share one.
+constexpr int kFuseSlots = 256;
 
 struct GemmLaunch {
     int mode;
@@ -41,6 +46,11 @@ struct GemmLaunch {
     float* part;       // grouped modes with splits > 1: fp32 partial sums, [piece slot][128][128]
     int num_sms;
     unsigned* status;  // device status word
+    // per-channel kernels: quantize x into q / sx inside the GEMM launch
+    // (x == nullptr: q / sx are inputs written by an earlier kernel)
+    const void* x = nullptr;
+    int xdt = 0;
+    int fuse_slot = 0;
 };
 
 // Launches `kern` with programmatic stream serialisation allowed, so that its
@@ -70,8 +80,8 @@ bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t r
                        const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
                        const cuuint32_t* elem_strides, CUtensorMapSwizzle swizzle);
 
-cudaError_t launch_quantize_act(const void* x, int xdt, int64_t M, int K, int8_t* q, float* sx,
-                                cudaStream_t st);
+cudaError_t launch_quantize_act(const void* x, int xdt, int64_t M, int K, int64_t ldx, int8_t* q, int64_t ldq,
+                                float* sx, int num_sms, cudaStream_t st);
 cudaError_t launch_silu_mul_quantize(const void* g, const void* u, int dt, int64_t M, int F,
                                      int8_t* q, float* sx, void* a_out, cudaStream_t st);
 // mode 0: per channel (out = int8 [N][K]); 1: per group int8; 2: per group int4 packed;
@@ -86,9 +96,12 @@ cudaError_t launch_wait_selftest(unsigned* status, unsigned long long limit_ns, 
 cudaError_t launch_unpack_int4(const uint8_t* packed, int64_t N, int K, int8_t* w, cudaStream_t st);
 cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const void* w,
                            const float* sw, int N, int gs, void* y, int ydt, int num_sms,
-                           cudaStream_t st);
-cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* w, const float* sw, int N,
-                            void* y, int ydt, int num_sms, cudaStream_t st);
+                           unsigned* status, cudaStream_t st);
+cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* w, const float* sw, int N, int gs,
+                            void* y, int ydt, int num_sms, unsigned* status, cudaStream_t st);
+// Whether the bulk-staged W8A16 kernel's shared-memory plan fits this shape
+// (the per-group form has no other kernel).
+bool mv_w8a16_bulk_fits(int M, int K, int N, int gs, int num_sms);
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t st);
 cudaError_t launch_gemm_grouped(const GemmLaunch& L, cudaStream_t st);
 

@@ -25,7 +25,104 @@ struct GemmArgs {
     const float* sw;    // [N] or [G][N]
     void* y;            // [M][N] output (fp16/bf16), or int32 acc / acc_g in test modes
     unsigned* status;   // device status word
+    // Fused activation quantization (per-channel kernels): with x set, the
+    // kernel itself quantizes x [M][K] (xdt) into qout [M][K] and sxout [M] --
+    // the buffers its A tensor map and sx point at -- before its first A load,
+    // synchronising the grid on barrier slot fuse_slot.
+    const void* x = nullptr;
+    int xdt = 0;
+    int8_t* qout = nullptr;
+    float* sxout = nullptr;
+    int fuse_slot = 0;
 };
+
+// ---- fused activation quantization -----------------------------------------
+// Barrier slots of the fused launches (kFuseSlots, cider_kernels.h),
+// {arrivals, generation} each.  Zero at load; every launch leaves its slot's
+// arrival count at zero again.  Only the per-channel kernels' translation
+// unit uses them.
+static __device__ unsigned g_fuse_bar[kFuseSlots][2];
+
+__device__ __forceinline__ float fuse_warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Quantizer warp wq of nwq in every CTA: rows r = blockIdx.x + gridDim.x * (wq
+// + nwq * i), one warp per row -- the row's absmax over all of K, then its
+// codes -- with the same arithmetic as cider_quantize_act (act_scale,
+// quant8_codes), so the codes are those of the separate quantize kernel.
+template <typename TX>
+__device__ __forceinline__ void fused_quantize_rows(const GemmArgs& p, int wq, int nwq) {
+    const int lane = threadIdx.x & 31;
+    const int nch = p.K / 8;
+    for (int64_t r = blockIdx.x + static_cast<int64_t>(gridDim.x) * wq; r < p.M;
+         r += static_cast<int64_t>(gridDim.x) * nwq) {
+        const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const TX*>(p.x) + r * p.K);
+        typename Pack2<TX>::type m2 = {};
+#pragma unroll 4
+        for (int c = lane; c < nch; c += 32) m2 = absmax8<TX>(__ldg(xr + c), m2);
+        const float amax = fuse_warp_max(absmax_to_f32<TX>(m2));
+        const float s = act_scale(amax);
+        const float rs = act_rcp(s);
+        if (lane == 0) p.sxout[r] = s;
+        int8_t* qr = p.qout + r * p.K;
+#pragma unroll 4
+        for (int c = lane; c < nch; c += 32) {
+            float f[8];
+            unpack8_f32<TX>(__ldg(xr + c), f);
+            *reinterpret_cast<uint2*>(qr + 8 * c) = quant8_codes(f, s, rs);
+        }
+    }
+    // these generic-proxy writes are read by other CTAs' TMA (async proxy)
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void fused_quantize(const GemmArgs& p, int wq, int nwq) {
+    if (p.xdt == 1)
+        fused_quantize_rows<__nv_bfloat16>(p, wq, nwq);
+    else
+        fused_quantize_rows<__half>(p, wq, nwq);
+}
+
+// Grid-wide barrier of a fused launch, called by one thread per CTA after its
+// CTA's quantizer warps have synchronised.  Every CTA of the grid is resident
+// (one per SM, grid <= SMs).  Sense-reversing on the launch's slot: read the
+// generation, arrive; the last arrival resets the count and bumps the
+// generation, the others wait for that bump -- bounded in time like every
+// other wait.  On timeout it records CIDER_ERR_TIMEOUT in the status word and
+// returns false without aborting the CTA: the kernel then runs to completion
+// on whatever codes are in place, and the caller learns of the failure from
+// cider_device_status().
+__device__ __forceinline__ bool fused_grid_barrier(int slot, unsigned* status, volatile int* abort_flag) {
+    unsigned* cnt = &g_fuse_bar[slot][0];
+    unsigned* gen = &g_fuse_bar[slot][1];
+    unsigned g0;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g0) : "l"(gen) : "memory");
+    __threadfence();
+    const unsigned arrived = atomicAdd(cnt, 1u) + 1u;
+    if (arrived == gridDim.x) {
+        atomicExch(cnt, 0u);
+        __threadfence();
+        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(gen), "r"(g0 + 1u) : "memory");
+        return true;
+    }
+    const unsigned long long t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        unsigned g;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(gen) : "memory");
+        if (g != g0) return true;
+        if ((it & 63u) == 0u) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(status, kStatusTimeout);
+                return false;
+            }
+        }
+        __nanosleep(64);
+    }
+}
 
 // Raster: kGroupM consecutive M-blocks walk the N-blocks together, so the
 // CTAs running at the same time share B tiles in L2.

@@ -41,11 +41,12 @@ struct GemmCfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = (kSmemBudget / STAGE_BYTES) > 8 ? 8 : (kSmemBudget / STAGE_BYTES);
     static constexpr int ACC_BUFS = 2;
-    static constexpr int TMEM_COLS = ACC_BUFS * BN;  // 256 or 512
+    // two accumulators of BN columns, allocated as a power of two (256 or 512)
+    static constexpr int TMEM_COLS = ACC_BUFS * BN <= 256 ? 256 : 512;
     static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * ACC_BUFS) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
-    static_assert(BN % 32 == 0 && BN <= 256, "BN");
-    static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+    static_assert(BN % 16 == 0 && BN <= 256, "BN: a multiple of 16 (the M = 128 MMA shape rule), at most 256");
+    static_assert(ACC_BUFS * BN <= TMEM_COLS, "TMEM");
 };
 
 template <typename TY>
@@ -56,6 +57,35 @@ __device__ __forceinline__ void store_row8(TY* dst, const float (&v)[8]) {
     o.z = pack2_out<TY>(v[4], v[5]);
     o.w = pack2_out<TY>(v[6], v[7]);
     *reinterpret_cast<uint4*>(dst) = o;
+}
+
+// 16 accumulator columns of one row m (the tail chunk of a BN that is not a
+// multiple of 32): the same expression as store_chunk_pc.
+template <int MODE, typename TY>
+__device__ __forceinline__ void store_chunk16_pc(const GemmArgs& p, const uint32_t (&r)[16], int m, int n0,
+                                                 float sxm) {
+    if (MODE == kModeI32) {
+        int32_t* out = static_cast<int32_t*>(p.y) + static_cast<int64_t>(m) * p.N;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (n0 + 4 * j < p.N)
+                *reinterpret_cast<uint4*>(out + n0 + 4 * j) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+    } else {
+        TY* out = static_cast<TY*>(p.y) + static_cast<int64_t>(m) * p.N;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            if (n0 + 8 * j < p.N) {
+                const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.sw + n0 + 8 * j));
+                const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.sw + n0 + 8 * j + 4));
+                const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    v[e] = (static_cast<float>(static_cast<int32_t>(r[8 * j + e])) * sxm) * ws[e];
+                store_row8<TY>(out + n0 + 8 * j, v);
+            }
+        }
+    }
 }
 
 // Per-channel (or INT32) epilogue for 32 accumulator columns of one row m:
@@ -103,6 +133,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     uint64_t* acce = accf + NB;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + NB);
     __shared__ int s_abort;
+    __shared__ uint64_t qready;  // fused launches: the grid's codes are written
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -118,6 +149,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], Cfg::EPI_WARPS * 32);
         }
+        mbar_init(&qready, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_async_smem();
     }
@@ -140,14 +172,35 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            // Fused launch: the weights do not depend on the quantization, so
+            // the first ring's B tiles go out while the grid quantizes x; their
+            // A tiles follow once the codes are written (qready).
+            int pre = 0;
+            if (p.x != nullptr) {
+                for (int t = blockIdx.x; t < num_tiles && pre < S; t += gridDim.x) {
+                    int mb, nb;
+                    tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
+                    for (int kb = 0; kb < p.num_k_blocks && pre < S; ++kb, ++pre) {
+                        mbar_arrive_expect_tx(&full[pre], Cfg::STAGE_BYTES);
+                        tma_load_2d(sB + pre * Cfg::B_BYTES, &tmB, &full[pre], kb * kBK, nb * BN);
+                    }
+                }
+                ok = mbar_wait(&qready, 0, p.status, abort_flag);
+                asm volatile("fence.proxy.async.global;" ::: "memory");  // the codes, for the TMA reads below
+            }
+            int j = 0;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 int mb, nb;
                 tile_coords(t, p.num_m_blocks, p.num_n_blocks, mb, nb);
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-                    tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, &full[stage], kb * kBK, mb * kBM);
-                    tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, &full[stage], kb * kBK, nb * BN);
+                for (int kb = 0; kb < p.num_k_blocks; ++kb, ++j) {
+                    if (j < pre) {  // B already in flight on this stage's first use
+                        tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, &full[stage], kb * kBK, mb * kBM);
+                    } else {
+                        if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+                        tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, &full[stage], kb * kBK, mb * kBM);
+                        tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, &full[stage], kb * kBK, nb * BN);
+                    }
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -185,6 +238,17 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------ epilogue ----------------------------------
+        if (p.x != nullptr) {
+            // fused launch: quantize this CTA's share of the token rows first
+            fused_quantize(p, warp - 2, Cfg::EPI_WARPS);
+            asm volatile("bar.sync 2, %0;" ::"n"(Cfg::EPI_WARPS * 32) : "memory");
+            if (warp == 2 && lane == 0) {
+                // a barrier that runs out leaves the status word set; the
+                // kernel still runs to completion
+                fused_grid_barrier(p.fuse_slot, p.status, abort_flag);
+                mbar_arrive(&qready);
+            }
+        }
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
@@ -199,16 +263,26 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             if (!mbar_wait(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const float sxm = (Cfg::MODE == kModePC && mvalid) ? __ldg(p.sx + m) : 0.0f;
+            constexpr int NC = BN / 32;               // whole 32-column chunks
+            constexpr bool TAIL = (BN % 32) != 0;     // and one 16-column chunk
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = 0; c < NC; ++c) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_base + lane_addr + b * BN + c * 32, r);
                 tmem_ld_wait();
-                if (c == BN / 32 - 1) {
+                if (!TAIL && c == NC - 1) {
                     tc_fence_before();
                     mbar_arrive(&acce[b]);
                 }
                 if (mvalid) store_chunk_pc<Cfg::MODE, TY>(p, r, m, nb * BN + c * 32, sxm);
+            }
+            if constexpr (TAIL) {
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(tmem_base + lane_addr + b * BN + NC * 32, r);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&acce[b]);
+                if (mvalid) store_chunk16_pc<Cfg::MODE, TY>(p, r, m, nb * BN + NC * 32, sxm);
             }
             ++acc_i;
         }
@@ -304,6 +378,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     uint64_t* acce = accf + NB;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + NB);
     __shared__ int s_abort;
+    __shared__ uint64_t qready;  // fused launches: the grid's codes are written
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -323,6 +398,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], 2 * C::EPI_WARPS);  // one arrival per epilogue warp of either CTA
         }
+        mbar_init(&qready, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_async_smem();
     }
@@ -346,14 +422,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            // Fused launch: the first ring's B tiles go out while the grid
+            // quantizes x, their A tiles once this CTA's qready has fired.
+            int pre = 0;
+            if (p.x != nullptr) {
+                for (int u = cid; u < nunits && pre < S; u += ncl) {
+                    const TileUnit w = tile_unit(p, u);
+                    for (int kb = w.kb0; kb < w.kb1 && pre < S; ++kb, ++pre) {
+                        if (leader) mbar_arrive_expect_tx(&full[pre], 2 * C::STAGE_BYTES);
+                        const uint32_t bar = map_to_rank(&full[pre], 0);
+                        tma_load_2d_pair(sB + pre * C::B_BYTES, &tmB, bar, kb * kBK,
+                                         w.nb * C::BN + static_cast<int>(rank) * (C::BN / 2));
+                    }
+                }
+                ok = mbar_wait(&qready, 0, p.status, abort_flag);
+                asm volatile("fence.proxy.async.global;" ::: "memory");  // the codes, for the TMA reads below
+            }
+            int j = 0;
             for (int u = cid; u < nunits && ok; u += ncl) {
                 const TileUnit w = tile_unit(p, u);
-                for (int kb = w.kb0; kb < w.kb1; ++kb) {
-                    if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, p.status, abort_flag)) { ok = false; break; }
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+                for (int kb = w.kb0; kb < w.kb1; ++kb, ++j) {
                     const uint32_t bar = map_to_rank(&full[stage], 0);
+                    if (j >= pre) {
+                        if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, p.status, abort_flag)) { ok = false; break; }
+                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+                    }
                     tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, bar, kb * kBK, w.mb * C::BM + static_cast<int>(rank) * 128);
-                    tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, bar, kb * kBK, w.nb * C::BN + static_cast<int>(rank) * (C::BN / 2));
+                    if (j >= pre)
+                        tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, bar, kb * kBK,
+                                         w.nb * C::BN + static_cast<int>(rank) * (C::BN / 2));
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -395,6 +492,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         // Warp w reads TMEM lanes 32*(w%4).. and columns [half*128, half*128+128) in
         // chunks of 32, loading chunk c+1 (and its scales) before converting chunk c.
         // Per-channel outputs go through a swizzled shared-memory box and a TMA store.
+        if (p.x != nullptr) {
+            // fused launch: quantize this CTA's share of the token rows first
+            fused_quantize(p, warp - 2, C::EPI_WARPS);
+            asm volatile("bar.sync 2, %0;" ::"n"(C::EPI_WARPS * 32) : "memory");
+            if (warp == 2 && lane == 0) {
+                fused_grid_barrier(p.fuse_slot, p.status, abort_flag);
+                mbar_arrive(&qready);
+            }
+        }
         const int ew = warp - 2;
         const int quarter = warp & 3;
         const int half = ew / 4;
@@ -503,6 +609,11 @@ static cudaError_t launch_gemm_cfg(const GemmLaunch& L, cudaStream_t st) {
     a.full_tiles = a.num_m_blocks * a.num_n_blocks;
     a.splits = 1;
     a.kb_per_split = a.num_k_blocks;
+    a.x = L.x;
+    a.xdt = L.xdt;
+    a.qout = const_cast<int8_t*>(L.q);
+    a.sxout = const_cast<float*>(L.sx);
+    a.fuse_slot = L.fuse_slot;
     const int tiles = a.num_m_blocks * a.num_n_blocks;
     const int grid = tiles < L.num_sms ? tiles : L.num_sms;
     auto kern = k_gemm_sm100<Cfg, TY>;
@@ -585,6 +696,11 @@ static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
     a.sw = L.sw;
     a.y = L.y;
     a.status = L.status;
+    a.x = L.x;
+    a.xdt = L.xdt;
+    a.qout = const_cast<int8_t*>(L.q);
+    a.sxout = const_cast<float*>(L.sx);
+    a.fuse_slot = L.fuse_slot;
     const int tiles = a.num_m_blocks * a.num_n_blocks;
     // split K of the tail tiles (per-channel with a partial-sum buffer only)
     int splits = (MODE == kModePC && L.part != nullptr && L.splits > 1) ? L.splits : 1;
@@ -614,6 +730,7 @@ template <int MODE, typename TY>
 static cudaError_t launch_gemm_mode(const GemmLaunch& L, cudaStream_t st) {
     if (L.variant == kGemmPair) return launch_gemm_pair<MODE, TY>(L, st);
     if (L.variant == kGemmSingle128) return launch_gemm_cfg<GemmCfg<128, MODE>, TY>(L, st);
+    if (L.variant == kGemmSingle80) return launch_gemm_cfg<GemmCfg<80, MODE>, TY>(L, st);
     return launch_gemm_cfg<GemmCfg<256, MODE>, TY>(L, st);
 }
 

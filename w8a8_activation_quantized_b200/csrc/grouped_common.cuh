@@ -1,6 +1,5 @@
 // grouped_common.cuh -- pieces of the per-group GEMM kernel: the bias-removing
-// rescale of INT32 partials, 16-column TMEM loads, the cp.async scale ring
-// and the INT32 test store.
+// rescale of INT32 partials, the cp.async scale ring and the INT32 test store.
 #pragma once
 
 #include "gemm_common.cuh"
@@ -13,16 +12,6 @@ constexpr int kScaleSlots = 4;                   // per-warp scale ring depth
 __device__ __forceinline__ uint64_t pack_u32x2(uint32_t lo, uint32_t hi) {
     return (static_cast<uint64_t>(hi) << 32) | lo;
 }
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-}
-
 // 16 bytes global -> shared, zero-filled when `bytes` is 0.
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint32_t bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(bytes)

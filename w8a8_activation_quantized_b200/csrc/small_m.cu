@@ -245,6 +245,253 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
     }
 }
 
+// ---- bulk-staged decode kernel (1 <= M <= 4) --------------------------------
+// The same fused quantize + dot + dequant as k_small_m, organised so that HBM
+// sees as many bytes in flight as it can take.  One CTA per SM owns a
+// contiguous, balanced range of weight rows [n0, n1) -- in the [N][K] layout a
+// single contiguous byte range -- and a producer warp streams it through a
+// ring of shared-memory stages with bulk asynchronous copies, one copy of R
+// whole rows per stage, completion counted on the stage's mbarrier.  With ~20
+// KB stages and the ring filling the rest of shared memory, ~150-200 KB per SM
+// are requested before the first dot product is taken; at the decode shapes
+// of the pages' tables (26 MB of weights over 148 SMs) that is almost the whole
+// of each SM's share, so the copies keep HBM busy while the activations are
+// quantized.  Eight consumer warps form R rows x S K-slices of each stage
+// (R * S = 8); lane l of a slice takes its 16-byte chunks l, l + 32, ... from
+// shared memory, so a warp reads 512 contiguous bytes per step.  Each (row,
+// slice) partial goes to shared memory once; after the last stage the CTA
+// adds the slices in order, dequantizes and writes its outputs, coalesced.
+// With M = 1 the lane's activation codes sit in registers (the lane's chunk
+// positions are the same for every row).  Every wait is bounded; a wait that
+// runs out records the timeout, and the other warps leave their loops through
+// the CTA's abort flag.
+constexpr int kBulkConsumers = 8;                          // consumer warps
+constexpr int kBulkThreads = (kBulkConsumers + 1) * 32;    // + one producer warp
+constexpr int kBulkMaxStages = 16;
+
+struct BulkGeom {
+    int R, S;        // rows per stage, K-slices per row (R * S = 8)
+    int cps, ppl;    // 16-byte chunks per slice, chunks per lane per slice
+    int nstage;      // ring slots
+    int rows_max;    // most rows of any CTA
+    int slot_bytes;  // R * bytes per weight row
+    int q_off, sw_off, part_off, ring_off, smem;  // dynamic shared memory layout
+};
+
+__device__ __forceinline__ void named_sync_consumers() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kBulkConsumers * 32) : "memory");
+}
+
+// The producer thread: stage j holds rows n0 + j*R .. of the CTA (the last
+// stage possibly fewer), one bulk copy each; a slot is refilled once all eight
+// consumer warps have released it.
+__device__ __forceinline__ void bulk_produce(const uint8_t* __restrict__ w, int n0, int rows, int row_bytes,
+                                             const BulkGeom& geo, uint8_t* ring, uint64_t* full, uint64_t* empty,
+                                             unsigned* status, volatile int* abort_flag) {
+    const uint8_t* src = w + static_cast<int64_t>(n0) * row_bytes;
+    const int nst = (rows + geo.R - 1) / geo.R;
+    for (int j = 0; j < nst; ++j) {
+        const int slot = j % geo.nstage;
+        if (j >= geo.nstage && !mbar_wait(&empty[slot], ((j / geo.nstage) - 1) & 1, status, abort_flag)) break;
+        const int nr = min(geo.R, rows - j * geo.R);
+        const uint32_t bytes = static_cast<uint32_t>(nr * row_bytes);
+        mbar_arrive_expect_tx(&full[slot], bytes);
+        bulk_load(ring + slot * geo.slot_bytes, src + static_cast<int64_t>(j) * geo.R * row_bytes, bytes,
+                  &full[slot]);
+    }
+}
+
+template <typename TX, bool PG, bool W4, int MAXM, int PPL>
+__global__ void __launch_bounds__(kBulkThreads, 1) k_small_m_bulk(const TX* __restrict__ x, int M, int K,
+                                                                  const uint8_t* __restrict__ w,
+                                                                  const float* __restrict__ sw, int N, int gs,
+                                                                  void* __restrict__ y, int ydt, BulkGeom geo,
+                                                                  unsigned* status) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t full[kBulkMaxStages], empty[kBulkMaxStages];
+    __shared__ float s_sx[MAXM];
+    __shared__ float s_red[MAXM][kBulkConsumers];
+    __shared__ int s_abort;
+    constexpr int KC = W4 ? 32 : 16;  // weights per 16-byte chunk
+    int8_t* s_q = reinterpret_cast<int8_t*>(smem + geo.q_off);          // [M][K] codes
+    float* s_sw = reinterpret_cast<float*>(smem + geo.sw_off);          // [K/gs][rows_max] group scales
+    float* s_part = reinterpret_cast<float*>(smem + geo.part_off);      // [rows][S][M] partials
+    uint8_t* ring = smem + geo.ring_off;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row_bytes = W4 ? K / 2 : K;
+    const int nch = row_bytes / 16;
+    const int n0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / gridDim.x);
+    const int n1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / gridDim.x);
+    const int rows = n1 - n0;
+    const int nst = (rows + geo.R - 1) / geo.R;
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int i = 0; i < geo.nstage; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kBulkConsumers);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+    volatile int* abort_flag = &s_abort;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == kBulkConsumers) {  // producer
+        if (lane == 0) bulk_produce(w, n0, rows, row_bytes, geo, ring, full, empty, status, abort_flag);
+        return;
+    }
+
+    // consumers: the CTA's group scales (group-major in HBM: one contiguous run
+    // of the CTA's rows per group) and the M activation rows' codes
+    if (PG) {
+        const int G = K / gs;
+        for (int t = threadIdx.x; t < G * rows; t += kBulkConsumers * 32) {
+            const int g = t / rows, r = t - g * rows;
+            s_sw[g * geo.rows_max + r] = __ldg(sw + static_cast<int64_t>(g) * N + n0 + r);
+        }
+    }
+    const int nx = K / 8;  // 16-byte chunks of a row of x
+    for (int m = 0; m < M; ++m) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K);
+        typename Pack2<TX>::type m2 = {};
+        for (int c = threadIdx.x; c < nx; c += kBulkConsumers * 32) m2 = absmax8<TX>(__ldg(xr + c), m2);
+        float amax = absmax_to_f32<TX>(m2);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0) s_red[m][warp] = amax;
+    }
+    named_sync_consumers();
+    for (int m = 0; m < M; ++m) {
+        float amax = s_red[m][0];
+#pragma unroll
+        for (int i = 1; i < kBulkConsumers; ++i) amax = fmaxf(amax, s_red[m][i]);
+        const float s = act_scale(amax);
+        const float rs = act_rcp(s);
+        if (threadIdx.x == 0) s_sx[m] = s;
+        const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K);
+        for (int c = threadIdx.x; c < nx; c += kBulkConsumers * 32) {
+            float f[8];
+            unpack8_f32<TX>(__ldg(xr + c), f);
+            *reinterpret_cast<uint2*>(s_q + static_cast<int64_t>(m) * K + 8 * c) = quant8_codes(f, s, rs);
+        }
+    }
+    named_sync_consumers();
+
+    const int r_in = warp / geo.S, sl = warp % geo.S;
+    const int c_begin = sl * geo.cps, c_end = min(nch, c_begin + geo.cps);
+    // M = 1: this lane's activation codes, the same chunk positions for every row
+    constexpr int XQ = MAXM == 1 ? PPL : 1;
+    uint4 xq[XQ][W4 ? 2 : 1];
+    if constexpr (MAXM == 1) {
+#pragma unroll
+        for (int p = 0; p < PPL; ++p) {
+            const int c = c_begin + 32 * p + lane;
+            const bool ok = p < geo.ppl && c < c_end;
+#pragma unroll
+            for (int h = 0; h < (W4 ? 2 : 1); ++h)
+                xq[p][h] = ok ? *reinterpret_cast<const uint4*>(s_q + c * KC + 16 * h) : make_uint4(0, 0, 0, 0);
+        }
+    }
+    for (int j = 0; j < nst; ++j) {
+        const int slot = j % geo.nstage;
+        if (!mbar_wait(&full[slot], (j / geo.nstage) & 1, status, abort_flag)) break;
+        const int rl = j * geo.R + r_in;  // the CTA-local row this warp takes
+        int iacc[MAXM];
+        float facc[MAXM];
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) { iacc[m] = 0; facc[m] = 0.0f; }
+        if (rl < rows) {
+            const uint8_t* wrow = ring + slot * geo.slot_bytes + r_in * row_bytes;
+#pragma unroll
+            for (int p = 0; p < PPL; ++p) {
+                if (p >= geo.ppl) break;  // warp-uniform
+                const int c = c_begin + 32 * p + lane;
+                if (c < c_end) {
+                    const uint4 wv = *reinterpret_cast<const uint4*>(wrow + 16 * c);
+                    const int k0 = c * KC;
+                    const float gsc = PG ? s_sw[(k0 / gs) * geo.rows_max + rl] : 0.0f;
+#pragma unroll
+                    for (int m = 0; m < MAXM; ++m) {
+                        if (m < M) {
+                            int d;
+                            if constexpr (MAXM == 1) {
+                                if constexpr (!W4) {
+                                    d = dp4a(wv.x, xq[p][0].x, 0);
+                                    d = dp4a(wv.y, xq[p][0].y, d);
+                                    d = dp4a(wv.z, xq[p][0].z, d);
+                                    d = dp4a(wv.w, xq[p][0].w, d);
+                                } else {
+                                    const uint2 u0 = unpack_int4x8(wv.x), u1 = unpack_int4x8(wv.y);
+                                    const uint2 u2 = unpack_int4x8(wv.z), u3 = unpack_int4x8(wv.w);
+                                    d = dp4a(u0.x, xq[p][0].x, 0);
+                                    d = dp4a(u0.y, xq[p][0].y, d);
+                                    d = dp4a(u1.x, xq[p][0].z, d);
+                                    d = dp4a(u1.y, xq[p][0].w, d);
+                                    d = dp4a(u2.x, xq[p][1].x, d);
+                                    d = dp4a(u2.y, xq[p][1].y, d);
+                                    d = dp4a(u3.x, xq[p][1].z, d);
+                                    d = dp4a(u3.y, xq[p][1].w, d);
+                                }
+                            } else {
+                                d = chunk_dot<W4>(wv, s_q + static_cast<int64_t>(m) * K, k0);
+                            }
+                            if (PG)
+                                facc[m] = fmaf(static_cast<float>(d), gsc, facc[m]);
+                            else
+                                iacc[m] += d;
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);  // this warp's reads of the slot are done
+        if (rl < rows) {
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) {
+                if (m < M) {
+                    float v;
+                    if (PG) {
+                        float a = facc[m];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+                        v = a;
+                    } else {
+                        int a = iacc[m];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+                        v = __int_as_float(a);
+                    }
+                    if (lane == 0) s_part[(rl * geo.S + sl) * M + m] = v;
+                }
+            }
+        }
+    }
+    named_sync_consumers();
+    if (*abort_flag) return;
+    // add the slices in order, dequantize, write the CTA's outputs (row-major y)
+    for (int t = threadIdx.x; t < rows * M; t += kBulkConsumers * 32) {
+        const int m = t / rows, r = t - m * rows;
+        float out;
+        if (PG) {
+            float a = 0.0f;
+            for (int q = 0; q < geo.S; ++q) a += s_part[(r * geo.S + q) * M + m];
+            out = a * s_sx[m];
+        } else {
+            int a = 0;
+            for (int q = 0; q < geo.S; ++q) a += __float_as_int(s_part[(r * geo.S + q) * M + m]);
+            out = static_cast<float>(a) * s_sx[m] * __ldg(sw + n0 + r);
+        }
+        const int64_t o = static_cast<int64_t>(m) * N + n0 + r;
+        if (ydt == 1)
+            static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(out);
+        else
+            static_cast<__half*>(y)[o] = __float2half_rn(out);
+    }
+}
+
 // ---- W8A16 decode matrix-vector product ----------------------------------
 // The pages' decode kernel (Cider README, section "Metal Kernel 流水线",
 // Decode): a direct INT8 matrix-vector product with the weights dequantized
@@ -401,6 +648,134 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_mv_w8a16(const TX* __restr
     }
 }
 
+// W8A16 decode product on the bulk-staged layout of k_small_m_bulk (one CTA
+// per SM, a contiguous range of weight rows streamed through a shared-memory
+// ring by a producer warp), per output channel or per group of gs along K.
+// The activation rows are staged once as fp32 pairs in the [pass][pair][lane]
+// layout of k_mv_w8a16 (slices are whole 512-weight passes, so lane l always
+// takes chunks l, l + 32, ... of a pass and its reads are conflict-free).  Per
+// group, each lane multiplies its chunk's fp32 dot by the chunk's group scale
+// scale_w[g][n] (staged per CTA) and accumulates; per channel the row's sum is
+// scaled by scale_w[n] at the end.
+template <typename TX, bool PG, int MAXM, int PPL>
+__global__ void __launch_bounds__(kBulkThreads, 1) k_mv_w8a16_bulk(const TX* __restrict__ x, int M, int K,
+                                                                   const int8_t* __restrict__ w,
+                                                                   const float* __restrict__ sw, int N, int gs,
+                                                                   void* __restrict__ y, int ydt, BulkGeom geo,
+                                                                   unsigned* status) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t full[kBulkMaxStages], empty[kBulkMaxStages];
+    __shared__ int s_abort;
+    uint64_t* s_x = reinterpret_cast<uint64_t*>(smem + geo.q_off);  // [M][pass][8 pairs][32 lanes]
+    float* s_sw = reinterpret_cast<float*>(smem + geo.sw_off);      // [K/gs][rows_max]
+    float* s_part = reinterpret_cast<float*>(smem + geo.part_off);  // [rows][S][M]
+    uint8_t* ring = smem + geo.ring_off;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nch = K / 16;
+    const int npass = (nch + 31) / 32;
+    const int n0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / gridDim.x);
+    const int n1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / gridDim.x);
+    const int rows = n1 - n0;
+    const int nst = (rows + geo.R - 1) / geo.R;
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int i = 0; i < geo.nstage; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kBulkConsumers);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+    volatile int* abort_flag = &s_abort;
+    pdl_wait();
+    pdl_trigger();
+    if (warp == kBulkConsumers) {
+        if (lane == 0)
+            bulk_produce(reinterpret_cast<const uint8_t*>(w), n0, rows, K, geo, ring, full, empty, status, abort_flag);
+        return;
+    }
+    if (PG) {
+        const int G = K / gs;
+        for (int t = threadIdx.x; t < G * rows; t += kBulkConsumers * 32) {
+            const int g = t / rows, r = t - g * rows;
+            s_sw[g * geo.rows_max + r] = __ldg(sw + static_cast<int64_t>(g) * N + n0 + r);
+        }
+    }
+    // the 8 values at k0 = 8t belong to chunk c = t / 2 (pass c / 32, lane
+    // c % 32), pairs (t % 2) * 4 .. + 3
+    const int nx = K / 8;
+    for (int m = 0; m < M; ++m) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K);
+        for (int t = threadIdx.x; t < nx; t += kBulkConsumers * 32) {
+            float f[8];
+            unpack8_f32<TX>(__ldg(xr + t), f);
+            const int c = t >> 1, q = c >> 5, l = c & 31, j0 = (t & 1) * 4;
+            uint64_t* dst = s_x + ((static_cast<int64_t>(m) * npass + q) * 8 + j0) * 32 + l;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[32 * j] = pack_f32x2(f[2 * j], f[2 * j + 1]);
+        }
+    }
+    named_sync_consumers();
+
+    const int r_in = warp / geo.S, sl = warp % geo.S;
+    const int pass0 = sl * (geo.cps / 32);
+    for (int j = 0; j < nst; ++j) {
+        const int slot = j % geo.nstage;
+        if (!mbar_wait(&full[slot], (j / geo.nstage) & 1, status, abort_flag)) break;
+        const int rl = j * geo.R + r_in;
+        float acc[MAXM];
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) acc[m] = 0.0f;
+        if (rl < rows) {
+            const uint8_t* wrow = ring + slot * geo.slot_bytes + r_in * K;
+#pragma unroll
+            for (int p = 0; p < PPL; ++p) {
+                if (p >= geo.ppl) break;  // warp-uniform
+                const int c = (pass0 + p) * 32 + lane;
+                if (c < nch) {
+                    const uint4 wv = *reinterpret_cast<const uint4*>(wrow + 16 * c);
+                    const float gsc = PG ? s_sw[((16 * c) / gs) * geo.rows_max + rl] : 1.0f;
+#pragma unroll
+                    for (int m = 0; m < MAXM; ++m) {
+                        if (m < M) {
+                            const float d =
+                                chunk_dot_f32(wv, s_x + ((static_cast<int64_t>(m) * npass + pass0 + p) * 8) * 32 + lane);
+                            acc[m] = PG ? fmaf(d, gsc, acc[m]) : acc[m] + d;
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (rl < rows) {
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) {
+                if (m < M) {
+                    float a = acc[m];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+                    if (lane == 0) s_part[(rl * geo.S + sl) * M + m] = a;
+                }
+            }
+        }
+    }
+    named_sync_consumers();
+    if (*abort_flag) return;
+    for (int t = threadIdx.x; t < rows * M; t += kBulkConsumers * 32) {
+        const int m = t / rows, r = t - m * rows;
+        float a = 0.0f;
+        for (int q = 0; q < geo.S; ++q) a += s_part[(r * geo.S + q) * M + m];
+        const float out = PG ? a : a * __ldg(sw + n0 + r);
+        const int64_t o = static_cast<int64_t>(m) * N + n0 + r;
+        if (ydt == 1)
+            static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(out);
+        else
+            static_cast<__half*>(y)[o] = __float2half_rn(out);
+    }
+}
+
 // Slices per row: as many as keep at least 4 passes per warp (at most 8).
 static SmallGeom small_geom(int K, int N, bool w4) {
     SmallGeom g;
@@ -449,9 +824,80 @@ static cudaError_t launch_small_m_t(const void* x, int M, int K, const void* w, 
     return launch_small_ppw<TX, PG, W4, 16>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
 }
 
+// Shared-memory plan of k_small_m_bulk: R rows per stage with R * row bytes
+// <= 24 KB (R = 8, 4, 2 or 1), the codes, the CTA's group scales and the
+// partials first, the ring of stages in the rest (at most 16 stages).  Returns
+// false when fewer than three stages fit, or a slice needs more than 8 chunks
+// per lane; those calls take k_small_m.
+constexpr int kBulkSmemBytes = 225 * 1024;
+// With a16 (the W8A16 product) the activation rows are staged as fp32 pairs,
+// M * (whole 512-weight passes) * 2048 bytes, and slices are whole passes.
+static bool bulk_plan(int M, int K, int N, bool pg, bool w4, int gs, int num_sms, BulkGeom& g, int& grid,
+                      bool a16 = false) {
+    const int row_bytes = w4 ? K / 2 : K;
+    int R = 8;
+    while (R > 1 && R * row_bytes > 24 * 1024) R >>= 1;
+    g.R = R;
+    g.S = kBulkConsumers / R;
+    const int nch = row_bytes / 16;
+    g.cps = (nch + g.S - 1) / g.S;
+    if (a16) g.cps = (g.cps + 31) / 32 * 32;
+    g.ppl = (g.cps + 31) / 32;
+    if (g.ppl > 8) return false;
+    g.slot_bytes = R * row_bytes;
+    grid = N / R < num_sms ? (N / R > 0 ? N / R : 1) : num_sms;
+    g.rows_max = (N + grid - 1) / grid;
+    auto al = [](int64_t v) { return static_cast<int>((v + 127) & ~int64_t(127)); };
+    int off = 0;
+    g.q_off = off;
+    off += a16 ? al(static_cast<int64_t>(M) * ((nch + 31) / 32) * 2048) : al(static_cast<int64_t>(M) * K);
+    g.sw_off = off;
+    off += pg ? al(static_cast<int64_t>(K / gs) * g.rows_max * 4) : 0;
+    g.part_off = off;
+    off += al(static_cast<int64_t>(g.rows_max) * g.S * M * 4);
+    g.ring_off = off;
+    if (off >= kBulkSmemBytes) return false;
+    g.nstage = (kBulkSmemBytes - off) / g.slot_bytes;
+    if (g.nstage > kBulkMaxStages) g.nstage = kBulkMaxStages;
+    if (g.nstage < 3) return false;
+    g.smem = off + g.nstage * g.slot_bytes;
+    return true;
+}
+
+template <typename TX, bool PG, bool W4, int MAXM, int PPL>
+static cudaError_t launch_bulk_t(const void* x, int M, int K, const void* w, const float* sw, int N, int gs, void* y,
+                                 int ydt, const BulkGeom& geo, int grid, unsigned* status, cudaStream_t st) {
+    auto kern = k_small_m_bulk<TX, PG, W4, MAXM, PPL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, geo.smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, grid, kBulkThreads, geo.smem, st, static_cast<const TX*>(x), M, K,
+                      static_cast<const uint8_t*>(w), sw, N, gs, y, ydt, geo, status);
+}
+
+template <typename TX, bool PG, bool W4, int MAXM>
+static cudaError_t launch_bulk_ppl(const void* x, int M, int K, const void* w, const float* sw, int N, int gs,
+                                   void* y, int ydt, const BulkGeom& geo, int grid, unsigned* status,
+                                   cudaStream_t st) {
+    if (geo.ppl <= 2) return launch_bulk_t<TX, PG, W4, MAXM, 2>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+    if (geo.ppl <= 4) return launch_bulk_t<TX, PG, W4, MAXM, 4>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+    if (geo.ppl <= 6) return launch_bulk_t<TX, PG, W4, MAXM, 6>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+    return launch_bulk_t<TX, PG, W4, MAXM, 8>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+}
+
 template <bool PG, bool W4>
 static cudaError_t launch_small_m_v(const void* x, int xdt, int M, int K, const void* w, const float* sw, int N,
-                                    int gs, void* y, int ydt, int num_sms, cudaStream_t st) {
+                                    int gs, void* y, int ydt, int num_sms, unsigned* status, cudaStream_t st) {
+    BulkGeom geo;
+    int grid = 0;
+    if (M <= 4 && bulk_plan(M, K, N, PG, W4, gs, num_sms, geo, grid)) {
+        if (xdt == 1) {
+            if (M == 1)
+                return launch_bulk_ppl<__nv_bfloat16, PG, W4, 1>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+            return launch_bulk_ppl<__nv_bfloat16, PG, W4, 4>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+        }
+        if (M == 1) return launch_bulk_ppl<__half, PG, W4, 1>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+        return launch_bulk_ppl<__half, PG, W4, 4>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+    }
     if (xdt == 1) return launch_small_m_t<__nv_bfloat16, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
     return launch_small_m_t<__half, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
 }
@@ -480,8 +926,54 @@ static cudaError_t launch_mv_ppw(const void* x, int M, int K, const int8_t* w, c
     return cudaErrorInvalidValue;  // K beyond the kernel: rejected by the host checks first
 }
 
-cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* w, const float* sw, int N,
-                            void* y, int ydt, int num_sms, cudaStream_t st) {
+template <typename TX, bool PG, int MAXM, int PPL>
+static cudaError_t launch_mv_bulk_t(const void* x, int M, int K, const int8_t* w, const float* sw, int N, int gs,
+                                    void* y, int ydt, const BulkGeom& geo, int grid, unsigned* status,
+                                    cudaStream_t st) {
+    auto kern = k_mv_w8a16_bulk<TX, PG, MAXM, PPL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, geo.smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, grid, kBulkThreads, geo.smem, st, static_cast<const TX*>(x), M, K, w, sw, N, gs, y, ydt,
+                      geo, status);
+}
+
+template <typename TX, bool PG, int MAXM>
+static cudaError_t launch_mv_bulk_ppl(const void* x, int M, int K, const int8_t* w, const float* sw, int N, int gs,
+                                      void* y, int ydt, const BulkGeom& geo, int grid, unsigned* status,
+                                      cudaStream_t st) {
+    if (geo.ppl <= 2) return launch_mv_bulk_t<TX, PG, MAXM, 2>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+    if (geo.ppl <= 4) return launch_mv_bulk_t<TX, PG, MAXM, 4>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+    if (geo.ppl <= 6) return launch_mv_bulk_t<TX, PG, MAXM, 6>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+    return launch_mv_bulk_t<TX, PG, MAXM, 8>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+}
+
+template <typename TX, bool PG>
+static cudaError_t launch_mv_bulk_m(const void* x, int M, int K, const int8_t* w, const float* sw, int N, int gs,
+                                    void* y, int ydt, const BulkGeom& geo, int grid, unsigned* status,
+                                    cudaStream_t st) {
+    if (M <= 1) return launch_mv_bulk_ppl<TX, PG, 1>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+    return launch_mv_bulk_ppl<TX, PG, 4>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+}
+
+bool mv_w8a16_bulk_fits(int M, int K, int N, int gs, int num_sms) {
+    BulkGeom geo;
+    int grid = 0;
+    return bulk_plan(M, K, N, gs > 0, false, gs, num_sms, geo, grid, true);
+}
+
+cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* w, const float* sw, int N, int gs,
+                            void* y, int ydt, int num_sms, unsigned* status, cudaStream_t st) {
+    BulkGeom geo;
+    int grid = 0;
+    if (bulk_plan(M, K, N, gs > 0, false, gs, num_sms, geo, grid, true)) {
+        if (gs > 0) {
+            if (xdt == 1) return launch_mv_bulk_m<__nv_bfloat16, true>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+            return launch_mv_bulk_m<__half, true>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
+        }
+        if (xdt == 1) return launch_mv_bulk_m<__nv_bfloat16, false>(x, M, K, w, sw, N, 0, y, ydt, geo, grid, status, st);
+        return launch_mv_bulk_m<__half, false>(x, M, K, w, sw, N, 0, y, ydt, geo, grid, status, st);
+    }
+    if (gs > 0) return cudaErrorInvalidValue;  // the host checks reject such per-group shapes first
     if (xdt == 1) {
         if (M <= 1) return launch_mv_ppw<__nv_bfloat16, 1>(x, M, K, w, sw, N, y, ydt, num_sms, st);
         return launch_mv_ppw<__nv_bfloat16, 4>(x, M, K, w, sw, N, y, ydt, num_sms, st);
@@ -492,11 +984,11 @@ cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* 
 
 cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const void* w,
                            const float* sw, int N, int gs, void* y, int ydt, int num_sms,
-                           cudaStream_t st) {
+                           unsigned* status, cudaStream_t st) {
     switch (mode) {
-        case kModePC: return launch_small_m_v<false, false>(x, xdt, M, K, w, sw, N, gs, y, ydt, num_sms, st);
-        case kModePG: return launch_small_m_v<true, false>(x, xdt, M, K, w, sw, N, gs, y, ydt, num_sms, st);
-        case kModeW4: return launch_small_m_v<true, true>(x, xdt, M, K, w, sw, N, gs, y, ydt, num_sms, st);
+        case kModePC: return launch_small_m_v<false, false>(x, xdt, M, K, w, sw, N, gs, y, ydt, num_sms, status, st);
+        case kModePG: return launch_small_m_v<true, false>(x, xdt, M, K, w, sw, N, gs, y, ydt, num_sms, status, st);
+        case kModeW4: return launch_small_m_v<true, true>(x, xdt, M, K, w, sw, N, gs, y, ydt, num_sms, status, st);
         default: return cudaErrorInvalidValue;
     }
 }
