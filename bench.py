@@ -653,30 +653,34 @@ def run_row(args):
         print(json.dumps({"row": args.row, "kind": kind, "M": M, "K": K, "ms": ms,
                           "GB/s": (M * K * 3 + M * 4) / (ms * 1e-3) / 1e9}), flush=True)
         return 0
+    cider.cider_test_set_small_m_kernel(args.small_kernel)
     x = torch.from_numpy(synth.activations(M, K, 1000 + M)).to(device)
     W = torch.from_numpy(synth.weights(N, K, 1001)).to(device)
     if kind == "pc":
         w, s = cider.cider_quantize_weight_pc(W)
-        call = lambda y, ws_: cider.cider_w8a8_linear_pc(x, w, s, y=y, workspace=ws_)
+        call = lambda w, y, ws_: cider.cider_w8a8_linear_pc(x, w, s, y=y, workspace=ws_)
     elif kind == "mv":
         w, s = cider.cider_quantize_weight_pc(W)
-        call = lambda y, ws_: cider.cider_w8a16_mv_pc(x, w, s, y=y)
+        call = lambda w, y, ws_: cider.cider_w8a16_mv_pc(x, w, s, y=y)
     elif kind == "pg":
         w, s = cider.cider_quantize_weight_pg(W, gs)
-        call = lambda y, ws_: cider.cider_w8a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)
+        call = lambda w, y, ws_: cider.cider_w8a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)
     elif kind == "mvpg":
         w, s = cider.cider_quantize_weight_pg(W, gs)
-        call = lambda y, ws_: cider.cider_w8a16_mv_pg(x, w, s, gs, y=y)
+        call = lambda w, y, ws_: cider.cider_w8a16_mv_pg(x, w, s, gs, y=y)
     elif kind == "w4pc":
         w, s = cider.cider_pack_weight_int4_pc(W)
-        call = lambda y, ws_: cider.cider_w4a8_linear_pc(x, w, s, y=y, workspace=ws_)
+        call = lambda w, y, ws_: cider.cider_w4a8_linear_pc(x, w, s, y=y, workspace=ws_)
     else:
         w, s = cider.cider_pack_weight_int4_pg(W, gs)
-        call = lambda y, ws_: cider.cider_w4a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)
+        call = lambda w, y, ws_: cider.cider_w4a8_linear_pg(x, w, s, gs, y=y, workspace=ws_)
     del W
-    y = torch.empty((M, N), dtype=torch.float16, device=device)
+    # as in the bench rows: weight copies rotate beyond the L2 cache between calls
+    n = rotating(w.numel() + M * K * 3 + M * N * 2)
+    wr = [w] + [w.roll(i, 0).contiguous() for i in range(1, n)]
+    ys = [torch.empty((M, N), dtype=torch.float16, device=device) for _ in range(min(n, 4))]
     wsp = torch.empty((max(1, cider.cider_workspace_bytes_mnk(M, N, K)),), dtype=torch.uint8, device=device)
-    ms = graph_time(lambda i: call(y, wsp), args.steps, args.warmup)
+    ms = graph_time(lambda i: call(wr[i % n], ys[i % len(ys)], wsp), args.steps, args.warmup)
     cider.cider_device_status()
     print(json.dumps({"row": args.row, "kind": kind, "M": M, "N": N, "K": K, "gs": gs, "ms": ms,
                       "TOPS": 2.0 * M * N * K / (ms * 1e-3) / 1e12}), flush=True)
@@ -694,6 +698,8 @@ def main():
     ap.add_argument("--row", choices=sorted(ROW_CASES), help="time one hot-path row alone (for profiling)")
     ap.add_argument("--fused", choices=["auto", "off", "on"], default="auto",
                     help="with --row: where the per-channel linear quantizes (inside the GEMM launch or not)")
+    ap.add_argument("--small-kernel", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="with --row: decode kernel (0 auto, 1 register ring, 2 bulk, 3 bulk in half of smem)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -163,13 +163,12 @@ CIDER_API cider_status_t cider_w8a16_mv_pc(const void* x, cider_dtype_t xdt, int
  * kernel list).  y[m,n] = round_ydt(sum_g scale_w[g][n] * sum_{k in g}
  * x[m,k] * w[n,k]) with x widened to fp32, each chunk of 16 products summed
  * in fp32, scaled by its group's scale and accumulated in fp32; the
- * activations are NOT quantized.  x: [M][K] (xdt), 1 <= M <= 4, K <= 32768;
- * w: [N][K] int8; scale_w: [K/gs][N] fp32 (group-major, as for the per-group
- * linears); y: [M][N] (ydt).  No workspace.  Besides the common checks,
- * CIDER_ERR_INVALID_ARG when gs is not 64 or 128 or does not divide K, or
- * when the shape's staged activations (M * K * 4 bytes), the group scales of
- * one SM's share of the rows and three weight stages exceed the shared
- * memory of an SM. */
+ * activations are NOT quantized.  x: [M][K] (xdt), 1 <= M <= 4 and
+ * M * ceil(K / 512) * 2048 <= 160 KiB (the rows are staged in shared memory
+ * as fp32), K <= 32768; w: [N][K] int8; scale_w: [K/gs][N] fp32 (group-major,
+ * as for the per-group linears); y: [M][N] (ydt).  No workspace.  Besides the
+ * common checks, CIDER_ERR_INVALID_ARG when gs is not 64 or 128 or does not
+ * divide K. */
 CIDER_API cider_status_t cider_w8a16_mv_pg(const void* x, cider_dtype_t xdt, int64_t M, int64_t K,
                                  const int8_t* w, const float* scale_w, int64_t N, int64_t gs,
                                  void* y, cider_dtype_t ydt, void* stream);
@@ -331,11 +330,18 @@ CIDER_API cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8
  * 2 = single-CTA 128x256 tiles, 3 = CTA-pair 256x256 tiles, 4 = single-CTA
  * 128x80 tiles.  Lets tests cover every variant on small shapes. */
 CIDER_API cider_status_t cider_test_set_gemm_variant(int variant);
+/* Selects the decode-shaped kernel of the small-M path for later calls
+ * (process-wide): 0 = automatic (default), 1 = the register-ring kernel,
+ * 2 = the bulk-staged kernel with the whole shared memory, 3 = the
+ * bulk-staged kernel within half of it.  Shapes a bulk plan cannot hold take
+ * the register-ring kernel either way.  Lets tests and measurements compare
+ * the kernels on the same shapes. */
+CIDER_API cider_status_t cider_test_set_small_m_kernel(int kernel);
 /* Selects, for later calls (process-wide), how the per-channel linear
  * (cider_w8a8_linear_pc and the workspace-free form) quantizes its
- * activations on the tensor-core path: 0 = automatic (default: inside the
- * GEMM launch for M <= 1024, by the separate quantize kernel above), 1 =
- * always the separate kernel, 2 = always inside the GEMM launch.  Either way
+ * activations on the tensor-core path: 0 = automatic (default: the separate
+ * quantize kernel, which measured faster), 1 = always the separate kernel,
+ * 2 = always inside the GEMM launch.  Either way
  * the call leaves the codes q [M][K] at the start of the workspace and
  * scale_x [M] at byte offset align256(M * K), which lets tests check the
  * fused quantization bit for bit.  The fused launch synchronises its grid

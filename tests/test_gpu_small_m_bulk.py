@@ -1,7 +1,8 @@
-"""The decode-shaped linear (1 <= M <= 4) against the oracle, on shapes chosen
-for the corners of its bulk-staged plan (one CTA per SM owns a contiguous
-range of weight rows and streams it through a ring of shared-memory stages of
-R rows, eight warps as R rows x 8/R K-slices):
+"""The bulk-staged decode kernel (1 <= M <= 4; selected by the test switch --
+the register-ring kernel, which measured faster, is the default) against the
+oracle, on shapes chosen for the corners of its plan (one CTA per SM owns a
+contiguous range of weight rows and streams it through a ring of
+shared-memory stages of R rows, eight warps as R rows x 8/R K-slices):
 
 * more stages per CTA than ring slots, so slots are reused (N = 20480);
 * a CTA's last stage only partly filled (rows per CTA not a multiple of R);
@@ -33,7 +34,9 @@ def _device():
         pytest.skip("no CUDA device")
     old = cider.cider_get_small_m_threshold()
     cider.cider_set_small_m_threshold(4)
+    cider.cider_test_set_small_m_kernel(2)
     yield
+    cider.cider_test_set_small_m_kernel(0)
     cider.cider_set_small_m_threshold(old)
     cider.cider_device_status()
 
@@ -104,3 +107,30 @@ def test_small_m_repeated_calls_agree():
     b = cider.cider_w8a8_linear_pg(x, w, s, gs)
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("kernel", [1, 2, 3])
+@pytest.mark.parametrize("mode", ["pc", "pg", "w4"])
+def test_small_m_each_kernel(kernel, mode):
+    """The test switch's three decode kernels (register ring, bulk-staged with
+    the whole shared memory, bulk-staged within half of it) on one shape."""
+    M, N, K, gs = 2, 2056, 4096, 64
+    x = act(M, K, seed=kernel * 10 + len(mode))
+    W = synth.weights(N, K, seed=77)
+    cider.cider_test_set_small_m_kernel(kernel)
+    try:
+        if mode == "pc":
+            qw, sw = oracle.quantize_weight_pc(W)
+            y = cider.cider_w8a8_linear_pc(dev_bits(x, F16), dev(qw), dev(sw))
+            ref = oracle.linear_pc(x, qw, sw)
+        elif mode == "pg":
+            qw, sw = oracle.quantize_weight_pg(W, gs)
+            y = cider.cider_w8a8_linear_pg(dev_bits(x, F16), dev(qw), dev(np.ascontiguousarray(sw.T)), gs)
+            ref = oracle.linear_pg(x, qw, sw, gs)
+        else:
+            packed, sw = oracle.quantize_weight_int4_pg(W, gs)
+            y = cider.cider_w4a8_linear_pg(dev_bits(x, F16), dev(packed), dev(np.ascontiguousarray(sw.T)), gs)
+            ref = oracle.w4a8_linear_pg(x, packed, sw, gs)
+    finally:
+        cider.cider_test_set_small_m_kernel(2)  # this module's setting
+    check_y(y, ref, F16)

@@ -61,23 +61,6 @@ def test_w8a16_mv_zero_token_and_argument_checks():
 
 # ---- per-group weight scales (cider_w8a16_mv_pg) ---------------------------------
 
-def _pg_plan_fits(M, N, K, gs, num_sms):
-    """The kernel's shared-memory plan: stages of R rows (R * K <= 24 KB), one
-    CTA per SM on min(num_sms, N / R) CTAs; fp32 activation pairs of whole
-    512-weight passes, the group scales of the CTA's rows and the slice
-    partials (each rounded up to 128 bytes), then at least three stages in
-    225 KB."""
-    al = lambda v: (v + 127) // 128 * 128
-    R = 8
-    while R > 1 and R * K > 24 * 1024:
-        R //= 2
-    S = 8 // R
-    grid = min(num_sms, max(1, N // R))
-    rows_max = -(-N // grid)
-    used = al(M * ((K // 16 + 31) // 32) * 2048) + al((K // gs) * rows_max * 4) + al(rows_max * S * M * 4)
-    return used < 225 * 1024 and (225 * 1024 - used) // (R * K) >= 3
-
-
 @pytest.mark.parametrize("M", [1, 2, 4])
 @pytest.mark.parametrize("N,K,gs", [(2560, 10240, 64), (2560, 10240, 128), (10240, 2560, 64), (264, 1088, 64),
                                     (20480, 1024, 128), (8, 64, 64), (136, 32768, 128), (136, 16384, 128)])
@@ -85,7 +68,7 @@ def test_w8a16_mv_pg(M, N, K, gs):
     x = act(M, K, seed=M + N + K + gs)
     qw, sw = oracle.quantize_weight_pg(synth.weights(N, K, seed=N + K + gs), gs)
     args = (dev_bits(x, oracle.F16), dev(qw), dev(np.ascontiguousarray(sw.T)), gs)
-    if not _pg_plan_fits(M, N, K, gs, torch.cuda.get_device_properties(0).multi_processor_count):
+    if M * ((K // 16 + 31) // 32) * 2048 > 160 * 1024:  # staged fp32 rows beyond shared memory
         with pytest.raises(cider.CiderError, match="shared memory"):
             cider.cider_w8a16_mv_pg(*args)
         return
@@ -127,6 +110,25 @@ def test_w8a16_mv_pg_argument_checks():
         cider.cider_w8a16_mv_pg(x, w, dev(np.ones((K // 32, N), np.float32)), 32)
     with pytest.raises(cider.CiderError):  # decode shapes only
         cider.cider_w8a16_mv_pg(dev_bits(act(5, K, seed=1), oracle.F16), w, dev(np.ones((K // 64, N), np.float32)), 64)
-    with pytest.raises(cider.CiderError):  # staged rows + scales beyond shared memory
-        cider.cider_w8a16_mv_pg(dev_bits(act(4, 10240, seed=1), oracle.F16), dev(np.zeros((40960, 10240), np.int8)),
-                                dev(np.ones((160, 40960), np.float32)), 64)
+    with pytest.raises(cider.CiderError):  # staged rows beyond shared memory
+        cider.cider_w8a16_mv_pg(dev_bits(act(4, 16384, seed=1), oracle.F16), dev(np.zeros((8, 16384), np.int8)),
+                                dev(np.ones((256, 8), np.float32)), 64)
+
+
+@pytest.mark.parametrize("kernel", [2, 3])
+def test_w8a16_mv_bulk_kernel(kernel):
+    """The bulk-staged W8A16 kernels (selectable by the test switch) on the
+    per-channel and per-group forms."""
+    M, N, K, gs = 2, 2056, 4096, 64
+    x = act(M, K, seed=kernel)
+    W = synth.weights(N, K, seed=kernel + 1)
+    qc, sc = oracle.quantize_weight_pc(W)
+    qg, sg = oracle.quantize_weight_pg(W, gs)
+    cider.cider_test_set_small_m_kernel(kernel)
+    try:
+        y_pc = cider.cider_w8a16_mv_pc(dev_bits(x, oracle.F16), dev(qc), dev(sc))
+        y_pg = cider.cider_w8a16_mv_pg(dev_bits(x, oracle.F16), dev(qg), dev(np.ascontiguousarray(sg.T)), gs)
+    finally:
+        cider.cider_test_set_small_m_kernel(0)
+    check_y(y_pc, oracle.w8a16_linear_pc(x, qc, sc), oracle.F16)
+    check_y(y_pg, oracle.w8a16_linear_pg(x, qg, sg, gs), oracle.F16)

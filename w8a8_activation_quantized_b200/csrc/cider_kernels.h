@@ -99,9 +99,10 @@ cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const
                            unsigned* status, cudaStream_t st);
 cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* w, const float* sw, int N, int gs,
                             void* y, int ydt, int num_sms, unsigned* status, cudaStream_t st);
-// Whether the bulk-staged W8A16 kernel's shared-memory plan fits this shape
-// (the per-group form has no other kernel).
-bool mv_w8a16_bulk_fits(int M, int K, int N, int gs, int num_sms);
+// Test override of the decode-shaped kernel (0 automatic, 1 register ring,
+// 2 bulk-staged, 3 bulk-staged within half of shared memory).
+cudaError_t set_small_m_kernel(int k);
+
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t st);
 cudaError_t launch_gemm_grouped(const GemmLaunch& L, cudaStream_t st);
 

@@ -53,6 +53,10 @@ __device__ __forceinline__ float fuse_warp_max(float v) {
 // + nwq * i), one warp per row -- the row's absmax over all of K, then its
 // codes -- with the same arithmetic as cider_quantize_act (act_scale,
 // quant8_codes), so the codes are those of the separate quantize kernel.
+// Rows of up to 32 * kFuseNV 16-byte chunks (K <= 6144) are loaded once, all
+// loads in flight together, and quantized from registers: one memory round
+// trip per row.  Wider rows take two passes over x (the second from L2).
+constexpr int kFuseNV = 12;
 template <typename TX>
 __device__ __forceinline__ void fused_quantize_rows(const GemmArgs& p, int wq, int nwq) {
     const int lane = threadIdx.x & 31;
@@ -60,19 +64,43 @@ __device__ __forceinline__ void fused_quantize_rows(const GemmArgs& p, int wq, i
     for (int64_t r = blockIdx.x + static_cast<int64_t>(gridDim.x) * wq; r < p.M;
          r += static_cast<int64_t>(gridDim.x) * nwq) {
         const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const TX*>(p.x) + r * p.K);
-        typename Pack2<TX>::type m2 = {};
-#pragma unroll 4
-        for (int c = lane; c < nch; c += 32) m2 = absmax8<TX>(__ldg(xr + c), m2);
-        const float amax = fuse_warp_max(absmax_to_f32<TX>(m2));
-        const float s = act_scale(amax);
-        const float rs = act_rcp(s);
-        if (lane == 0) p.sxout[r] = s;
         int8_t* qr = p.qout + r * p.K;
+        typename Pack2<TX>::type m2 = {};
+        if (nch <= 32 * kFuseNV) {
+            uint4 v[kFuseNV];
+#pragma unroll
+            for (int i = 0; i < kFuseNV; ++i) {
+                const int c = lane + 32 * i;
+                v[i] = c < nch ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < kFuseNV; ++i) m2 = absmax8<TX>(v[i], m2);
+            const float amax = fuse_warp_max(absmax_to_f32<TX>(m2));
+            const float s = act_scale(amax);
+            const float rs = act_rcp(s);
+            if (lane == 0) p.sxout[r] = s;
+#pragma unroll
+            for (int i = 0; i < kFuseNV; ++i) {
+                const int c = lane + 32 * i;
+                if (c < nch) {
+                    float f[8];
+                    unpack8_f32<TX>(v[i], f);
+                    *reinterpret_cast<uint2*>(qr + 8 * c) = quant8_codes(f, s, rs);
+                }
+            }
+        } else {
 #pragma unroll 4
-        for (int c = lane; c < nch; c += 32) {
-            float f[8];
-            unpack8_f32<TX>(__ldg(xr + c), f);
-            *reinterpret_cast<uint2*>(qr + 8 * c) = quant8_codes(f, s, rs);
+            for (int c = lane; c < nch; c += 32) m2 = absmax8<TX>(__ldg(xr + c), m2);
+            const float amax = fuse_warp_max(absmax_to_f32<TX>(m2));
+            const float s = act_scale(amax);
+            const float rs = act_rcp(s);
+            if (lane == 0) p.sxout[r] = s;
+#pragma unroll 4
+            for (int c = lane; c < nch; c += 32) {
+                float f[8];
+                unpack8_f32<TX>(__ldg(xr + c), f);
+                *reinterpret_cast<uint2*>(qr + 8 * c) = quant8_codes(f, s, rs);
+            }
         }
     }
     // these generic-proxy writes are read by other CTAs' TMA (async proxy)

@@ -64,8 +64,15 @@ struct GroupedCfg {
     static constexpr int BN = 128;
     static constexpr int EPI_WARPS = 8;
     static constexpr int EPI_COLS = BN / 2;  // columns per epilogue warp
+    // The W8A8 per-group modes issue their MMAs from two threads (warp 1 and a
+    // last warp), alternating groups, so that one issuer's barrier waits
+    // overlap the other's MMAs in flight (gs = 128 at M = 4096: 0.250 -> 0.210
+    // ms).  W4A8 keeps one issuer: a third warp would cost it a converter warp
+    // (within the register file at 12 warps), and one converter warp measured
+    // slower than the single issuer (0.379 -> 0.522 ms at 2048 x 12288 x 4096).
+    static constexpr int ISSUE2_WARPS = (PC || W4) ? 0 : 1;
     static constexpr int CONV_WARPS = W4 ? 2 : 0;
-    static constexpr int THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
+    static constexpr int THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS + ISSUE2_WARPS);
     static constexpr int A_BYTES = BM * kBK;
     static constexpr int B_BYTES = BN * kBK;
     static constexpr int BP_BYTES = W4 ? BN * kBK / 2 : 0;
@@ -134,7 +141,8 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
         s_abort = 0;
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            // a stage is released by the commit of each issuer whose groups read it
+            mbar_init(&empty[s], (C::ISSUE2_WARPS && gpk == 2) ? 2 : 1);
             if (C::W4) mbar_init(&conv[s], C::CONV_WARPS * 32);
         }
         for (int b = 0; b < NB; ++b) {
@@ -188,8 +196,14 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || (C::ISSUE2_WARPS && warp == 2 + C::EPI_WARPS + C::CONV_WARPS)) {
         // ------------------------------ MMA issuer --------------------------------
+        // Per-group modes: issuer 0 (warp 1) takes the even groups, issuer 1
+        // (the last warp) the odd ones.  A thread that waits on an mbarrier
+        // after issuing MMAs stalls until those MMAs complete, so a single
+        // issuer leaves the tensor pipe idle between groups; with two, one
+        // waits while the other's MMAs run.
+        const int issuer = warp == 1 ? 0 : 1;
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_i8(C::BM, BN);
             constexpr uint32_t idesc_bias = umma_idesc_f16(C::BM, BN);
@@ -229,26 +243,38 @@ __global__ void __launch_bounds__(GroupedCfg<MODE>::THREADS, 1)
                 }
                 int g = w.g0;
                 for (int kb = w.kb0; kb < w.kb1 && ok; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
-                    if (C::W4 && !mbar_wait(&conv[stage], phase, p.status, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
-                    const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
-                    for (int j = 0; j < gpk && g < w.g1; ++j, ++g) {
-                        const uint32_t b = acc_i % NB;
-                        // use u of buffer b waits for phase u: use u-1 read out (or the initial release)
-                        if (!mbar_wait(&acce[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
+                    // this issuer's groups in the k-block: with two issuers and
+                    // two groups per stage one each; with one group per stage,
+                    // every other k-block; a single issuer takes them all
+                    constexpr bool kTwo = C::ISSUE2_WARPS != 0;
+                    const bool mine = (!kTwo || gpk == 2) ? true : ((acc_i & 1u) == static_cast<uint32_t>(issuer));
+                    if (mine) {
+                        if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) { ok = false; break; }
+                        if (C::W4 && !mbar_wait(&conv[stage], phase, p.status, abort_flag)) { ok = false; break; }
                         tc_fence_after();
-                        const uint32_t d = tmem_base + b * BN;
-                        umma_f16_overwrite(d, bias_adesc, bias_bdesc, idesc_bias);  // D = bits of 1.5 * 2^23
-                        for (int kk = 0; kk < steps; ++kk) {
-                            const int off = (j * steps + kk) * kUmmaK;
-                            umma_i8(d, adesc + (off >> 4), bdesc + (off >> 4), idesc, 1u);  // onto the bias
+                        const uint64_t adesc = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
+                        const uint64_t bdesc = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
+                        for (int j = 0; j < gpk && g + j < w.g1; ++j) {
+                            const uint32_t a = acc_i + j;  // this group's buffer use
+                            if (kTwo && (a & 1u) != static_cast<uint32_t>(issuer)) continue;
+                            const uint32_t b = a % NB;
+                            // use u of buffer b waits for phase u: use u-1 read out (or the initial release)
+                            if (!mbar_wait(&acce[b], (a / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
+                            tc_fence_after();
+                            const uint32_t d = tmem_base + b * BN;
+                            umma_f16_overwrite(d, bias_adesc, bias_bdesc, idesc_bias);  // D = bits of 1.5 * 2^23
+                            for (int kk = 0; kk < steps; ++kk) {
+                                const int off = (j * steps + kk) * kUmmaK;
+                                umma_i8(d, adesc + (off >> 4), bdesc + (off >> 4), idesc, 1u);  // onto the bias
+                            }
+                            umma_commit(&accf[b]);
                         }
-                        umma_commit(&accf[b]);
-                        ++acc_i;
+                        if (!ok) break;
+                        umma_commit(&empty[stage]);
                     }
-                    umma_commit(&empty[stage]);
+                    const int ng = min(gpk, w.g1 - g);
+                    g += ng;
+                    acc_i += ng;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
             }

@@ -248,6 +248,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 fused_grid_barrier(p.fuse_slot, p.status, abort_flag);
                 mbar_arrive(&qready);
             }
+            // scale_x was written in this launch by other CTAs: wait for the
+            // barrier's release, and read it from L2 (__ldcg) below
+            mbar_wait(&qready, 0, p.status, abort_flag);
         }
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int row = quarter * 32 + lane;
@@ -262,7 +265,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             const uint32_t b = acc_i % NB;
             if (!mbar_wait(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const float sxm = (Cfg::MODE == kModePC && mvalid) ? __ldg(p.sx + m) : 0.0f;
+            // coherent load: a fused launch writes scale_x itself
+            const float sxm = (Cfg::MODE == kModePC && mvalid) ? __ldcg(p.sx + m) : 0.0f;
             constexpr int NC = BN / 32;               // whole 32-column chunks
             constexpr bool TAIL = (BN % 32) != 0;     // and one 16-column chunk
 #pragma unroll 1
@@ -500,6 +504,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                 fused_grid_barrier(p.fuse_slot, p.status, abort_flag);
                 mbar_arrive(&qready);
             }
+            mbar_wait(&qready, 0, p.status, abort_flag);  // as in k_gemm_sm100: scale_x of this launch
         }
         const int ew = warp - 2;
         const int quarter = warp & 3;
@@ -517,7 +522,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             const int nw = w.nb * C::BN + half * C::EPI_COLS;  // first column of this warp
             const uint32_t b = acc_i % NB;
             const bool piece = w.slot >= 0;  // K piece of a tail tile: INT32 partial sums out
-            const float sxm = (MODE == kModePC && mvalid) ? __ldg(p.sx + m) : 0.0f;
+            // coherent load: a fused launch writes scale_x itself
+            const float sxm = (MODE == kModePC && mvalid) ? __ldcg(p.sx + m) : 0.0f;
             float ws[2][32];
             if (MODE == kModePC && !piece) load_scales32(p.sw, nw, p.N, ws[0]);
             if (!mbar_wait_cluster(&accf[b], (acc_i / NB) & 1u, p.status, abort_flag)) { ok = false; break; }

@@ -25,6 +25,8 @@
 // warp's final shuffle reduction adds the lanes.  With one warp per row
 // (S = 1) a warp writes its outputs directly; otherwise the slices combine
 // through shared memory.
+#include <atomic>
+
 #include "cider_device.cuh"
 #include "cider_kernels.h"
 
@@ -530,10 +532,12 @@ __device__ __forceinline__ float chunk_dot_f32(const uint4& wv, const uint64_t* 
     return lo_f32(acc) + hi_f32(acc);
 }
 
-template <typename TX, int MAXM, int PPW>
+// PG: per-group scales scale_w[g][n] (group-major), applied per 16-weight
+// chunk as its dot is accumulated; otherwise scale_w[n] on the row's sum.
+template <typename TX, bool PG, int MAXM, int PPW>
 __global__ void __launch_bounds__(kSmallThreads, 2) k_mv_w8a16(const TX* __restrict__ x, int M, int K,
                                                                const int8_t* __restrict__ w,
-                                                               const float* __restrict__ sw, int N,
+                                                               const float* __restrict__ sw, int N, int gs,
                                                                void* __restrict__ y, int ydt, SmallGeom geo) {
     extern __shared__ __align__(16) uint64_t s_x[];  // [M][pass][8 pairs][32 lanes] fp32 pairs
     __shared__ float s_part[kSmallWarps][MAXM];
@@ -547,8 +551,8 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_mv_w8a16(const TX* __restr
 
     constexpr int kRing = RingDepth<PPW>::value;
     uint4 ring[kRing][PPW];
-    float ring_s[kRing];
-    auto load = [&](uint4 (&dst)[PPW], float& ds, int blk) {
+    float ring_s[kRing][PG ? PPW : 1];
+    auto load = [&](uint4 (&dst)[PPW], float (&ds)[PG ? PPW : 1], int blk) {
         const int n = blk * geo.R + r_in_blk;
         const bool row_ok = blk < geo.nblocks && n < N;
         const uint4* wr = reinterpret_cast<const uint4*>(w + static_cast<int64_t>(n) * K);
@@ -557,8 +561,9 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_mv_w8a16(const TX* __restr
             const int c = (pass0 + p) * 32 + lane;
             const bool ok = p < geo.ppw && row_ok && c < nch;
             dst[p] = ok ? __ldcs(wr + c) : make_uint4(0, 0, 0, 0);
+            if (PG) ds[p] = ok ? __ldg(sw + static_cast<int64_t>(c * 16 / gs) * N + n) : 0.0f;
         }
-        ds = row_ok ? __ldg(sw + n) : 0.0f;
+        if (!PG) ds[0] = row_ok ? __ldg(sw + n) : 0.0f;
     };
 #pragma unroll
     for (int i = 0; i < kRing - 1; ++i) load(ring[i], ring_s[i], blockIdx.x + i * gridDim.x);
@@ -580,7 +585,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_mv_w8a16(const TX* __restr
     }
     __syncthreads();
 
-    auto step = [&](const uint4 (&cur)[PPW], float cs, int blk) {
+    auto step = [&](const uint4 (&cur)[PPW], const float (&cs)[PG ? PPW : 1], int blk) {
         const int n = blk * geo.R + r_in_blk;
         float acc[MAXM];
 #pragma unroll
@@ -593,8 +598,11 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_mv_w8a16(const TX* __restr
                 if (c < nch) {
 #pragma unroll
                     for (int m = 0; m < MAXM; ++m)
-                        if (m < M)
-                            acc[m] += chunk_dot_f32(cur[p], s_x + ((static_cast<int64_t>(m) * npass + pass0 + p) * 8) * 32 + lane);
+                        if (m < M) {
+                            const float d =
+                                chunk_dot_f32(cur[p], s_x + ((static_cast<int64_t>(m) * npass + pass0 + p) * 8) * 32 + lane);
+                            acc[m] = PG ? fmaf(d, cs[p], acc[m]) : acc[m] + d;
+                        }
                 }
             }
         }
@@ -606,7 +614,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_mv_w8a16(const TX* __restr
                 for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
                 if (geo.S == 1) {
                     if (lane == 0 && n < N) {
-                        const float out = a * cs;
+                        const float out = PG ? a : a * cs[0];
                         if (ydt == 1)
                             static_cast<__nv_bfloat16*>(y)[static_cast<int64_t>(m) * N + n] = __float2bfloat16_rn(out);
                         else
@@ -625,7 +633,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_mv_w8a16(const TX* __restr
                 if (nn < N) {
                     float a = 0.0f;
                     for (int sl = 0; sl < geo.S; ++sl) a += s_part[rr * geo.S + sl][m];
-                    const float out = a * __ldg(sw + nn);
+                    const float out = PG ? a : a * __ldg(sw + nn);
                     if (ydt == 1)
                         static_cast<__nv_bfloat16*>(y)[static_cast<int64_t>(m) * N + nn] = __float2bfloat16_rn(out);
                     else
@@ -830,10 +838,15 @@ static cudaError_t launch_small_m_t(const void* x, int M, int K, const void* w, 
 // false when fewer than three stages fit, or a slice needs more than 8 chunks
 // per lane; those calls take k_small_m.
 constexpr int kBulkSmemBytes = 225 * 1024;
+// test override of the decode kernel: 0 automatic, 1 register ring, 2 bulk
+// with the whole shared memory, 3 bulk within half of it
+static std::atomic<int> g_small_kernel{0};
+static int bulk_smem_budget() { return g_small_kernel.load() == 3 ? 110 * 1024 : kBulkSmemBytes; }
 // With a16 (the W8A16 product) the activation rows are staged as fp32 pairs,
 // M * (whole 512-weight passes) * 2048 bytes, and slices are whole passes.
 static bool bulk_plan(int M, int K, int N, bool pg, bool w4, int gs, int num_sms, BulkGeom& g, int& grid,
                       bool a16 = false) {
+    const int budget = bulk_smem_budget();
     const int row_bytes = w4 ? K / 2 : K;
     int R = 8;
     while (R > 1 && R * row_bytes > 24 * 1024) R >>= 1;
@@ -856,8 +869,8 @@ static bool bulk_plan(int M, int K, int N, bool pg, bool w4, int gs, int num_sms
     g.part_off = off;
     off += al(static_cast<int64_t>(g.rows_max) * g.S * M * 4);
     g.ring_off = off;
-    if (off >= kBulkSmemBytes) return false;
-    g.nstage = (kBulkSmemBytes - off) / g.slot_bytes;
+    if (off >= budget) return false;
+    g.nstage = (budget - off) / g.slot_bytes;
     if (g.nstage > kBulkMaxStages) g.nstage = kBulkMaxStages;
     if (g.nstage < 3) return false;
     g.smem = off + g.nstage * g.slot_bytes;
@@ -889,7 +902,11 @@ static cudaError_t launch_small_m_v(const void* x, int xdt, int M, int K, const 
                                     int gs, void* y, int ydt, int num_sms, unsigned* status, cudaStream_t st) {
     BulkGeom geo;
     int grid = 0;
-    if (M <= 4 && bulk_plan(M, K, N, PG, W4, gs, num_sms, geo, grid)) {
+    // the register-ring kernel is the default: the bulk-staged one measured
+    // slower on B200 (M = 1, N = 10240, K = 2560: 11.3 / 10.0 us with the
+    // whole / half of shared memory against 8.8 us); it stays selectable
+    const int sel = g_small_kernel.load();
+    if (M <= 4 && sel >= 2 && bulk_plan(M, K, N, PG, W4, gs, num_sms, geo, grid)) {
         if (xdt == 1) {
             if (M == 1)
                 return launch_bulk_ppl<__nv_bfloat16, PG, W4, 1>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
@@ -902,28 +919,35 @@ static cudaError_t launch_small_m_v(const void* x, int xdt, int M, int K, const 
     return launch_small_m_t<__half, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
 }
 
-template <typename TX, int MAXM, int PPW>
-static cudaError_t launch_mv_t(const void* x, int M, int K, const int8_t* w, const float* sw, int N, void* y,
+template <typename TX, bool PG, int MAXM, int PPW>
+static cudaError_t launch_mv_t(const void* x, int M, int K, const int8_t* w, const float* sw, int N, int gs, void* y,
                                int ydt, const SmallGeom& geo, int num_sms, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(M) * ((K / 16 + 31) / 32) * 2048;  // whole passes of pairs
-    auto kern = k_mv_w8a16<TX, MAXM, PPW>;
+    auto kern = k_mv_w8a16<TX, PG, MAXM, PPW>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
     const int grid = geo.nblocks < 2 * num_sms ? geo.nblocks : 2 * num_sms;
-    return launch_pdl(kern, grid, kSmallThreads, smem, st, static_cast<const TX*>(x), M, K, w, sw, N, y, ydt, geo);
+    return launch_pdl(kern, grid, kSmallThreads, smem, st, static_cast<const TX*>(x), M, K, w, sw, N, gs, y, ydt, geo);
 }
 
-template <typename TX, int MAXM>
-static cudaError_t launch_mv_ppw(const void* x, int M, int K, const int8_t* w, const float* sw, int N, void* y,
-                                 int ydt, int num_sms, cudaStream_t st) {
+template <typename TX, bool PG, int MAXM>
+static cudaError_t launch_mv_ppw(const void* x, int M, int K, const int8_t* w, const float* sw, int N, int gs,
+                                 void* y, int ydt, int num_sms, cudaStream_t st) {
     const SmallGeom geo = small_geom(K, N, false);
-    if (geo.ppw <= 2) return launch_mv_t<TX, MAXM, 2>(x, M, K, w, sw, N, y, ydt, geo, num_sms, st);
-    if (geo.ppw <= 4) return launch_mv_t<TX, MAXM, 4>(x, M, K, w, sw, N, y, ydt, geo, num_sms, st);
-    if (geo.ppw <= 5) return launch_mv_t<TX, MAXM, 5>(x, M, K, w, sw, N, y, ydt, geo, num_sms, st);
-    if (geo.ppw <= 8) return launch_mv_t<TX, MAXM, 8>(x, M, K, w, sw, N, y, ydt, geo, num_sms, st);
+    if (geo.ppw <= 2) return launch_mv_t<TX, PG, MAXM, 2>(x, M, K, w, sw, N, gs, y, ydt, geo, num_sms, st);
+    if (geo.ppw <= 4) return launch_mv_t<TX, PG, MAXM, 4>(x, M, K, w, sw, N, gs, y, ydt, geo, num_sms, st);
+    if (geo.ppw <= 5) return launch_mv_t<TX, PG, MAXM, 5>(x, M, K, w, sw, N, gs, y, ydt, geo, num_sms, st);
+    if (geo.ppw <= 8) return launch_mv_t<TX, PG, MAXM, 8>(x, M, K, w, sw, N, gs, y, ydt, geo, num_sms, st);
     return cudaErrorInvalidValue;  // K beyond the kernel: rejected by the host checks first
+}
+
+template <typename TX, bool PG>
+static cudaError_t launch_mv_reg(const void* x, int M, int K, const int8_t* w, const float* sw, int N, int gs,
+                                 void* y, int ydt, int num_sms, cudaStream_t st) {
+    if (M <= 1) return launch_mv_ppw<TX, PG, 1>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
+    return launch_mv_ppw<TX, PG, 4>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
 }
 
 template <typename TX, bool PG, int MAXM, int PPL>
@@ -955,17 +979,15 @@ static cudaError_t launch_mv_bulk_m(const void* x, int M, int K, const int8_t* w
     return launch_mv_bulk_ppl<TX, PG, 4>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
 }
 
-bool mv_w8a16_bulk_fits(int M, int K, int N, int gs, int num_sms) {
-    BulkGeom geo;
-    int grid = 0;
-    return bulk_plan(M, K, N, gs > 0, false, gs, num_sms, geo, grid, true);
-}
 
 cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* w, const float* sw, int N, int gs,
                             void* y, int ydt, int num_sms, unsigned* status, cudaStream_t st) {
+    // the register-ring kernel is the default (M = 1, N = 10240, K = 2560:
+    // 7.9 us against 11.3 us for the bulk-staged one); the bulk-staged kernel
+    // runs when the test switch selects it and its plan fits
     BulkGeom geo;
     int grid = 0;
-    if (bulk_plan(M, K, N, gs > 0, false, gs, num_sms, geo, grid, true)) {
+    if (g_small_kernel.load() >= 2 && bulk_plan(M, K, N, gs > 0, false, gs, num_sms, geo, grid, true)) {
         if (gs > 0) {
             if (xdt == 1) return launch_mv_bulk_m<__nv_bfloat16, true>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
             return launch_mv_bulk_m<__half, true>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
@@ -973,13 +995,18 @@ cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* 
         if (xdt == 1) return launch_mv_bulk_m<__nv_bfloat16, false>(x, M, K, w, sw, N, 0, y, ydt, geo, grid, status, st);
         return launch_mv_bulk_m<__half, false>(x, M, K, w, sw, N, 0, y, ydt, geo, grid, status, st);
     }
-    if (gs > 0) return cudaErrorInvalidValue;  // the host checks reject such per-group shapes first
-    if (xdt == 1) {
-        if (M <= 1) return launch_mv_ppw<__nv_bfloat16, 1>(x, M, K, w, sw, N, y, ydt, num_sms, st);
-        return launch_mv_ppw<__nv_bfloat16, 4>(x, M, K, w, sw, N, y, ydt, num_sms, st);
+    if (gs > 0) {
+        if (xdt == 1) return launch_mv_reg<__nv_bfloat16, true>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
+        return launch_mv_reg<__half, true>(x, M, K, w, sw, N, gs, y, ydt, num_sms, st);
     }
-    if (M <= 1) return launch_mv_ppw<__half, 1>(x, M, K, w, sw, N, y, ydt, num_sms, st);
-    return launch_mv_ppw<__half, 4>(x, M, K, w, sw, N, y, ydt, num_sms, st);
+    if (xdt == 1) return launch_mv_reg<__nv_bfloat16, false>(x, M, K, w, sw, N, 0, y, ydt, num_sms, st);
+    return launch_mv_reg<__half, false>(x, M, K, w, sw, N, 0, y, ydt, num_sms, st);
+}
+
+cudaError_t set_small_m_kernel(int k) {
+    if (k < 0 || k > 3) return cudaErrorInvalidValue;
+    g_small_kernel.store(k);
+    return cudaSuccess;
 }
 
 cudaError_t launch_small_m(int mode, const void* x, int xdt, int M, int K, const void* w,
