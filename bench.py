@@ -625,6 +625,7 @@ def run_row(args):
     device = torch.device("cuda", 0)
     cider.cider_test_set_fused_quantize({"auto": 0, "off": 1, "on": 2}[args.fused])
     if kind == "sdpa":  # decode attention alone, K/V rotated beyond L2
+        cider.cider_test_set_sdpa_kernel(args.sdpa_kernel)
         H_q, H_kv, Nk, D = 32, M, N, 128
         kv_bytes = 2 * H_kv * Nk * D * 2
         n = rotating(kv_bytes)
@@ -700,6 +701,8 @@ def main():
                     help="with --row: where the per-channel linear quantizes (inside the GEMM launch or not)")
     ap.add_argument("--small-kernel", type=int, default=0, choices=[0, 1, 2, 3],
                     help="with --row: decode kernel (0 auto, 1 register ring, 2 bulk, 3 bulk in half of smem)")
+    ap.add_argument("--sdpa-kernel", type=int, default=0, choices=[0, 1, 2],
+                    help="with --row: decode attention (0 auto, 1 CUDA cores, 2 tensor cores)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -330,6 +330,14 @@ CIDER_API cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8
  * 2 = single-CTA 128x256 tiles, 3 = CTA-pair 256x256 tiles, 4 = single-CTA
  * 128x80 tiles.  Lets tests cover every variant on small shapes. */
 CIDER_API cider_status_t cider_test_set_gemm_variant(int variant);
+/* Selects the decode-attention kernels for later calls (process-wide):
+ * 0 = automatic (default: the tensor-core kernel when 2 <= H_q / H_kv <= 16,
+ * the CUDA-core kernels otherwise), 1 = the CUDA-core kernels only, 2 = the
+ * tensor-core kernel wherever it applies, 3 = the same with the two offset
+ * fields of the V operand's shared-memory descriptor exchanged (a layout
+ * probe for tests).  The workspace size follows the selection: query
+ * cider_sdpa_decode_workspace_bytes after setting it. */
+CIDER_API cider_status_t cider_test_set_sdpa_kernel(int kernel);
 /* Selects the decode-shaped kernel of the small-M path for later calls
  * (process-wide): 0 = automatic (default), 1 = the register-ring kernel,
  * 2 = the bulk-staged kernel with the whole shared memory, 3 = the

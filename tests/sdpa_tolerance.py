@@ -14,13 +14,18 @@ values, plus F, a bound on the fp32 error |o' - o|:
 
     eps_rel = 2 ln2 (E_s + u S) + 4 depth 2^-21
 
-* E_s: error of one score in the log2 domain.  The kernel rounds q * log2(e)
-  / sqrt(D) once per element, sums 8 products with fused multiply-adds and 4
-  shuffle additions: at most 13 roundings, E_s <= 13 u c max_j sum_d |q_d
-  k_jd| with c = log2(e) / sqrt(D) and u = 2^-24.  The subtraction s - max
-  adds u S, S = the largest |s_j - max s|.  A weight's relative error is at
-  most ln2 times its exponent's error, and normalising by the sum of the
-  weights at most doubles it.
+* E_s: error of one score in the log2 domain.  The CUDA-core kernel rounds
+  q * log2(e) / sqrt(D) once per element, sums 8 products with fused
+  multiply-adds and 4 shuffle additions (13 roundings); the tensor-core
+  kernel forms the D exact products of 16-bit values and adds them in fp32
+  in an order of its own (at most D - 1 roundings), then scales once.  Both
+  are within D + 2 roundings: E_s <= (D + 2) u c max_j sum_d |q_d k_jd| with
+  c = log2(e) / sqrt(D) and u = 2^-24.  The subtraction s - max adds u S,
+  S = the largest |s_j - max s|.  A weight's relative error is at most ln2
+  times its exponent's error, and normalising by the sum of the weights at
+  most doubles it.  (The tensor-core kernel hands P to its second product as
+  a sum of 16-bit parts exact to 2^-22 of each weight, inside the 2^-21 per
+  step below.)
 * The rest: every hardware exp2 (relative error below 2^-22), every rescale
   of the running state, every fp32 addition of the running sums and every
   merge of streams and chunks costs at most 2^-21 relative; along any path
@@ -67,7 +72,7 @@ def fp32_bound(q, k, v, dt, keys_per_stream, chunks):
     for h in range(H_q):
         g = h // G
         s = (kf[g] @ qf[h]) * C                      # scores in the log2 domain
-        e_s = 13 * U * C * np.max(np.abs(kf[g]) @ np.abs(qf[h]))
+        e_s = (D + 2) * U * C * np.max(np.abs(kf[g]) @ np.abs(qf[h]))
         spread = float(s.max() - s.min())
         eps_rel = 2 * math.log(2) * (e_s + U * spread) + 4 * depth * 2.0 ** -21
         p = np.exp2(s - s.max())

@@ -52,6 +52,38 @@ def _check(H_q, H_kv, N, seed, dt=oracle.F16, kind="diffuse"):
     return out
 
 
+def test_sdpa_tc_operand_layout_probe():
+    """The tensor-core kernel reads V as an MN-major operand; of the two orders
+    of the descriptor's offset fields (mode 2: atoms along MN in the leading
+    field; mode 3: exchanged) exactly one reproduces the oracle.  The default
+    (mode 0) uses mode 2's order, so this test also pins the default."""
+    q, k, v = tl.make_inputs("peaked", 32, 8, 1024, seed=11)
+    ref = sdpa.sdpa_decode(q, k, v, oracle.F16)
+    ok = {}
+    for mode in (2, 3):
+        cider.cider_test_set_sdpa_kernel(mode)
+        try:
+            out = cider.cider_sdpa_decode(dev_bits(q, oracle.F16), dev_bits(k, oracle.F16), dev_bits(v, oracle.F16))
+            torch.cuda.synchronize()
+        finally:
+            cider.cider_test_set_sdpa_kernel(0)
+        n_bad, _ = tl.violations(ref, host_bits(out), q, k, v, oracle.F16, _num_sms())
+        ok[mode] = n_bad == 0
+    print(f"\ntensor-core V descriptor: mode 2 {'ok' if ok[2] else 'wrong'}, mode 3 {'ok' if ok[3] else 'wrong'}")
+    assert ok[2] and not ok[3]
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("H_kv,N", [(8, 4096), (4, 32768), (16, 3001)])
+def test_sdpa_both_kernels(kernel, H_kv, N):
+    """GQA shapes on the CUDA-core kernels (1) and the tensor-core kernel (2)."""
+    cider.cider_test_set_sdpa_kernel(kernel)
+    try:
+        _check(32, H_kv, N, seed=17 * kernel + N, kind="last_max")
+    finally:
+        cider.cider_test_set_sdpa_kernel(0)
+
+
 @pytest.mark.parametrize("H_kv", [32, 8, 4])
 @pytest.mark.parametrize("N", [1024, 4096, 32768])
 def test_sdpa_pages_configs(H_kv, N):

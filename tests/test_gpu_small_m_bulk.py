@@ -134,3 +134,22 @@ def test_small_m_each_kernel(kernel, mode):
     finally:
         cider.cider_test_set_small_m_kernel(2)  # this module's setting
     check_y(y, ref, F16)
+
+
+@pytest.mark.parametrize("M,K", [(12, 4096), (3, 16384), (16, 3072)])
+def test_register_ring_at_48k_of_codes(M, K):
+    """The register-ring kernel stages M x K codes in shared memory; at exactly
+    48 KB (plus its static shared memory) the launch must opt in to more than
+    the default, or it is refused."""
+    N = 264
+    x = act(M, K, seed=M + K)
+    qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed=K))
+    old = cider.cider_get_small_m_threshold()
+    cider.cider_set_small_m_threshold(16)
+    cider.cider_test_set_small_m_kernel(1)
+    try:
+        y = cider.cider_w8a8_linear_pc(dev_bits(x, F16), dev(qw), dev(sw))
+    finally:
+        cider.cider_test_set_small_m_kernel(2)  # this module's setting
+        cider.cider_set_small_m_threshold(old)
+    check_y(y, oracle.linear_pc(x, qw, sw), F16)

@@ -72,6 +72,7 @@ _SIGNATURES = {
     "cider_test_set_split_k": (_INT, [_INT]),
     "cider_test_set_fused_quantize": (_INT, [_INT]),
     "cider_test_set_small_m_kernel": (_INT, [_INT]),
+    "cider_test_set_sdpa_kernel": (_INT, [_INT]),
     "cider_test_bounded_wait": (_INT, [_I64, _P]),
 }
 EXPORTS = tuple(_SIGNATURES)
@@ -437,6 +438,11 @@ def cider_test_gemm_i32_grouped(q, w, gs, acc_g=None, stream=None):
 def cider_test_set_gemm_variant(variant: int):
     """0 automatic, 1 single-CTA 128x128, 2 single-CTA 128x256, 3 CTA-pair 256x256, 4 single-CTA 128x80."""
     _check("cider_test_set_gemm_variant", lib().cider_test_set_gemm_variant(variant))
+
+
+def cider_test_set_sdpa_kernel(kernel: int):
+    """0 automatic, 1 CUDA cores only, 2 tensor cores, 3 tensor cores with the V descriptor fields swapped."""
+    _check("cider_test_set_sdpa_kernel", lib().cider_test_set_sdpa_kernel(kernel))
 
 
 def cider_test_set_small_m_kernel(kernel: int):

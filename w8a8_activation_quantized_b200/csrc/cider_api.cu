@@ -721,7 +721,7 @@ cider_status_t cider_sdpa_decode(const void* q, const void* k, const void* v, ci
         overlap(ro, rng(workspace, need)))
         return fail(CIDER_ERR_INVALID_ARG, "out overlaps an input or the workspace");
     cudaError_t e = launch_sdpa_decode(q, k, v, dt == CIDER_BF16 ? 1 : 0, static_cast<int>(H_q), static_cast<int>(H_kv),
-                                       static_cast<int>(N), plan, static_cast<float*>(workspace), out,
+                                       static_cast<int>(N), plan, static_cast<float*>(workspace), out, d->status,
                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CIDER_OK : cuda_fail(e, "decode-attention launch");
 }
@@ -752,6 +752,11 @@ cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8_t* w, int
     const SplitPlan sp{0, forced > 1 ? forced : 1, 0, 0};
     return run_gemm(kModeI32G, q, nullptr, M, K, w, nullptr, N, gs, acc_g, 0, d, static_cast<cudaStream_t>(stream),
                     sp, nullptr);
+}
+
+cider_status_t cider_test_set_sdpa_kernel(int kernel) {
+    if (set_sdpa_kernel(kernel) != cudaSuccess) return fail(CIDER_ERR_INVALID_ARG, "kernel %d outside [0, 3]", kernel);
+    return CIDER_OK;
 }
 
 cider_status_t cider_test_set_small_m_kernel(int kernel) {

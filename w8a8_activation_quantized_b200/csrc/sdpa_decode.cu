@@ -300,6 +300,7 @@ cudaError_t launch_dt(const void* q, const void* k, const void* v, int H_q, int 
 }  // namespace
 
 SdpaPlan sdpa_plan(int64_t H_q, int64_t H_kv, int64_t N, int num_sms) {
+    if (sdpa_tc_applies(H_q, H_kv, N)) return sdpa_tc_plan(H_q, H_kv, N, num_sms);
     SdpaPlan p{};
     const int64_t G = H_q / H_kv;
     p.th = G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1);
@@ -321,9 +322,18 @@ size_t sdpa_part_bytes(int64_t H_q, const SdpaPlan& p) {
 }
 
 cudaError_t launch_sdpa_decode(const void* q, const void* k, const void* v, int dt, int H_q, int H_kv, int N,
-                               const SdpaPlan& plan, float* part, void* out, cudaStream_t st) {
+                               const SdpaPlan& plan, float* part, void* out, unsigned* status, cudaStream_t st) {
+    if (plan.tc) return launch_sdpa_tc(q, k, v, dt, H_q, H_kv, N, plan, part, out, status, st);
     return dt == 1 ? launch_dt<__nv_bfloat16>(q, k, v, H_q, H_kv, N, plan, part, out, st)
                    : launch_dt<__half>(q, k, v, H_q, H_kv, N, plan, part, out, st);
+}
+
+cudaError_t launch_sdpa_merge(const float* part, int chunks, void* out, int H_q, int dt, cudaStream_t st) {
+    if (dt == 1)
+        return launch_pdl(k_sdpa_decode_merge<__nv_bfloat16>, static_cast<unsigned>(H_q), kSdpaD, 0, st, part, chunks,
+                          static_cast<__nv_bfloat16*>(out));
+    return launch_pdl(k_sdpa_decode_merge<__half>, static_cast<unsigned>(H_q), kSdpaD, 0, st, part, chunks,
+                      static_cast<__half*>(out));
 }
 
 }  // namespace cider
