@@ -9,6 +9,9 @@
 namespace cider {
 
 constexpr int kSdpaD = 128;  // head dimension of the kernels
+// One chunk's partial result: o [D], then its max and its sum, padded to a
+// multiple of four floats so that every row starts 16-byte aligned.
+constexpr int kSdpaPartStride = kSdpaD + 4;
 
 // How a decode-attention call is cut: TH query heads per CTA (a head tile of
 // one KV group), C chunks of `chunk` keys along the sequence.
@@ -19,7 +22,7 @@ struct SdpaPlan {
     int tc = 0;
 };
 SdpaPlan sdpa_plan(int64_t H_q, int64_t H_kv, int64_t N, int num_sms);
-// fp32 partial results [H_q][chunks][D + 2] (o, then max and sum)
+// fp32 partial results [H_q][chunks][kSdpaPartStride] (o, then max and sum)
 size_t sdpa_part_bytes(int64_t H_q, const SdpaPlan& p);
 cudaError_t launch_sdpa_decode(const void* q, const void* k, const void* v, int dt, int H_q, int H_kv, int N,
                                const SdpaPlan& plan, float* part, void* out, unsigned* status, cudaStream_t st);

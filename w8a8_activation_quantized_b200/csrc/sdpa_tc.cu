@@ -96,6 +96,14 @@ __device__ __forceinline__ uint32_t kmaj_offset(int row, int k, int rows) {
     return atom * rows * 128 + (row >> 3) * 1024 + r8 * 128 + ((((kk >> 3) ^ r8) & 7) << 4) + (kk & 7) * 2;
 }
 
+// 2^x by the hardware approximation (PTX ex2.approx: relative error near
+// 2^-22, 2^-inf = +0), as in the CUDA-core kernels.
+__device__ __forceinline__ float ex2_tc(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <typename T>
 __device__ __forceinline__ uint16_t to_bits(T v) {
     return *reinterpret_cast<uint16_t*>(&v);
@@ -248,11 +256,14 @@ __global__ void __launch_bounds__(kTcThreads) k_sdpa_tc(const __grid_constant__ 
                 m[h] = fmaxf(m[h], sv[t][h]);
             }
         }
-        // the chunk's maximum per head, over the 128 threads
+        // the chunk's maximum per head, over the 128 threads (heads beyond the
+        // group are padding: no reductions, no weights)
 #pragma unroll
         for (int h = 0; h < kTcHeads; ++h) {
+            if (h < G) {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], o));
+                for (int o = 16; o > 0; o >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], o));
+            }
         }
         if (lane < kTcHeads) {
             float v = m[0];
@@ -271,11 +282,11 @@ __global__ void __launch_bounds__(kTcThreads) k_sdpa_tc(const __grid_constant__ 
             const int key = t * kTcKeys + wq * 32 + lane;  // within the chunk
 #pragma unroll
             for (int h = 0; h < kTcHeads; ++h) {
-                const float p = sv[t][h] == -INFINITY ? 0.0f : exp2f(sv[t][h] - m[h]);
-                l[h] += p;
-                uint16_t pt[NP];
-                split_parts<T, NP>(p, pt);
-                if (t < nt) {
+                if (h < G && t < nt) {
+                    const float p = ex2_tc(sv[t][h] - m[h]);  // 0 for keys past the chunk (-inf)
+                    l[h] += p;
+                    uint16_t pt[NP];
+                    split_parts<T, NP>(p, pt);
                     const uint32_t off = kmaj_offset(h, key, kTcHeads);
 #pragma unroll
                     for (int pp = 0; pp < NP; ++pp) *reinterpret_cast<uint16_t*>(sP + pp * kTcPPartBytes + off) = pt[pp];
@@ -287,8 +298,10 @@ __global__ void __launch_bounds__(kTcThreads) k_sdpa_tc(const __grid_constant__ 
         // the chunk's sum of weights per head
 #pragma unroll
         for (int h = 0; h < kTcHeads; ++h) {
+            if (h < G) {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], o);
+                for (int o = 16; o > 0; o >>= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], o);
+            }
         }
         if (lane < kTcHeads) {
             float v = l[0];
@@ -306,7 +319,7 @@ __global__ void __launch_bounds__(kTcThreads) k_sdpa_tc(const __grid_constant__ 
             tmem_ld_wait();
             const int d = wq * 32 + lane;
             for (int h = 0; h < G; ++h) {
-                float* pp = part + (static_cast<int64_t>(hk * G + h) * chunks + c) * (kSdpaD + 2);
+                float* pp = part + (static_cast<int64_t>(hk * G + h) * chunks + c) * kSdpaPartStride;
                 pp[d] = __uint_as_float(o[h]);
                 if (d == 0) {
                     pp[kSdpaD] = m[h];

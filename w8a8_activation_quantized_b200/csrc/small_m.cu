@@ -117,56 +117,11 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
 #pragma unroll
     for (int i = 0; i < kRing - 1; ++i) load(ring[i], ring_s[i], blockIdx.x + i * gridDim.x);
 
-    // M = 1 with whole rows per warp (S = 1): every warp quantizes the token by
-    // itself -- each lane loads the x values of exactly its own weight chunks,
-    // one warp max gives the row's absmax, and the lane keeps its codes in
-    // registers -- with no shared memory and no CTA barrier before the first
-    // dot product.  Otherwise all warps quantize the M rows into shared memory.
-    // (int8 weights and at most 5 passes per lane: the W4 and 8-pass forms
-    // would spill the extra x and code registers)
-    const bool warp_quant = MAXM == 1 && !W4 && PPW <= 5 && geo.S == 1;
-    constexpr int XQ = MAXM == 1 ? PPW : 1;
-    constexpr int XH = W4 ? 2 : 1;    // 16-byte code vectors per chunk
-    uint4 xq[XQ][XH];
-    float sx_warp = 0.0f;
-    if constexpr (MAXM == 1 && !W4 && PPW <= 5) {
-        if (warp_quant) {
-            constexpr int XV = KC / 8;  // 16-byte vectors of x per chunk
-            const uint4* xr = reinterpret_cast<const uint4*>(x);
-            uint4 xv[PPW][XV];
-#pragma unroll
-            for (int p = 0; p < PPW; ++p) {
-                const int c = p * 32 + lane;
-                const bool ok = p < geo.ppw && c < nch;
-#pragma unroll
-                for (int h = 0; h < XV; ++h) xv[p][h] = ok ? __ldg(xr + c * XV + h) : make_uint4(0, 0, 0, 0);
-            }
-            typename Pack2<TX>::type m2 = {};
-#pragma unroll
-            for (int p = 0; p < PPW; ++p)
-#pragma unroll
-                for (int h = 0; h < XV; ++h) m2 = absmax8<TX>(xv[p][h], m2);
-            float amax = absmax_to_f32<TX>(m2);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            const float sc = act_scale(amax);
-            const float rs = act_rcp(sc);
-            sx_warp = sc;
-#pragma unroll
-            for (int p = 0; p < PPW; ++p) {
-#pragma unroll
-                for (int h = 0; h < XH; ++h) {
-                    float f0[8], f1[8];
-                    unpack8_f32<TX>(xv[p][2 * h], f0);
-                    unpack8_f32<TX>(xv[p][2 * h + 1], f1);
-                    const uint2 lo = quant8_codes(f0, sc, rs), hi = quant8_codes(f1, sc, rs);
-                    xq[p][h] = make_uint4(lo.x, lo.y, hi.x, hi.y);
-                }
-            }
-        }
-    }
+    // Quantize the M activation rows into shared memory, all warps on every row.
+    // (Quantizing per warp in registers at M = 1 -- each lane loading the x of
+    // its own chunks, no CTA barrier -- measured slower: 12.9 against 10.7 us
+    // per launch under ncu, with 4x the L2 reads of x and 122 registers.)
     const int nx = K / 8;  // 16-byte chunks of a row of x
-    if (!warp_quant) {
     for (int m = 0; m < M; ++m) {
         const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K);
         typename Pack2<TX>::type m2 = {};
@@ -192,34 +147,6 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
         }
     }
     __syncthreads();
-    }  // !warp_quant
-    // INT32 dot of a chunk with the token's codes: from this lane's registers
-    // (warp_quant) or from shared memory
-    auto dot = [&](const uint4& wv, int m, int p, int k0) -> int {
-        if constexpr (MAXM == 1 && !W4 && PPW <= 5) {
-            if (warp_quant) {
-                if constexpr (!W4) {
-                    int a = dp4a(wv.x, xq[p][0].x, 0);
-                    a = dp4a(wv.y, xq[p][0].y, a);
-                    a = dp4a(wv.z, xq[p][0].z, a);
-                    return dp4a(wv.w, xq[p][0].w, a);
-                } else {
-                    const uint2 u0 = unpack_int4x8(wv.x), u1 = unpack_int4x8(wv.y);
-                    const uint2 u2 = unpack_int4x8(wv.z), u3 = unpack_int4x8(wv.w);
-                    int a = dp4a(u0.x, xq[p][0].x, 0);
-                    a = dp4a(u0.y, xq[p][0].y, a);
-                    a = dp4a(u1.x, xq[p][0].z, a);
-                    a = dp4a(u1.y, xq[p][0].w, a);
-                    a = dp4a(u2.x, xq[p][1].x, a);
-                    a = dp4a(u2.y, xq[p][1].y, a);
-                    a = dp4a(u3.x, xq[p][1].z, a);
-                    return dp4a(u3.y, xq[p][1].w, a);
-                }
-            }
-        }
-        return chunk_dot<W4>(wv, s_q + static_cast<int64_t>(m) * K, k0);
-    };
-    auto sxm = [&](int m) -> float { return warp_quant ? sx_warp : s_sx[m]; };
 
     auto step = [&](const uint4 (&cur)[PPW], const float (&cs)[PG ? PPW : 1], int blk) {
         const int n = blk * geo.R + r_in_blk;
@@ -237,7 +164,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
                 if (!PG) {
 #pragma unroll
                     for (int m = 0; m < MAXM; ++m)
-                        if (m < M && valid) iacc[m] = dot(cur[p], m, p, k0) + iacc[m];
+                        if (m < M && valid) iacc[m] = chunk_dot<W4>(cur[p], s_q + static_cast<int64_t>(m) * K, k0) + iacc[m];
                 } else {
                     // Each lane scales its own chunk's exact INT32 dot by the chunk's
                     // group scale: summed over the group's lanes that is
@@ -246,7 +173,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
 #pragma unroll
                     for (int m = 0; m < MAXM; ++m) {
                         if (m < M) {
-                            const int pp = valid ? dot(cur[p], m, p, k0) : 0;
+                            const int pp = valid ? chunk_dot<W4>(cur[p], s_q + static_cast<int64_t>(m) * K, k0) : 0;
                             facc[m] = fmaf(static_cast<float>(pp), s, facc[m]);
                         }
                     }
@@ -272,7 +199,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
                 }
                 if (geo.S == 1) {
                     if (lane == 0 && n < N) {
-                        const float out = PG ? v * sxm(m) : static_cast<float>(__float_as_int(v)) * sxm(m) * cs[0];
+                        const float out = PG ? v * s_sx[m] : static_cast<float>(__float_as_int(v)) * s_sx[m] * cs[0];
                         if (ydt == 1)
                             static_cast<__nv_bfloat16*>(y)[static_cast<int64_t>(m) * N + n] = __float2bfloat16_rn(out);
                         else
