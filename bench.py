@@ -699,8 +699,8 @@ def main():
     ap.add_argument("--row", choices=sorted(ROW_CASES), help="time one hot-path row alone (for profiling)")
     ap.add_argument("--fused", choices=["auto", "off", "on"], default="auto",
                     help="with --row: where the per-channel linear quantizes (inside the GEMM launch or not)")
-    ap.add_argument("--small-kernel", type=int, default=0, choices=[0, 1, 2, 3],
-                    help="with --row: decode kernel (0 auto, 1 register ring, 2 bulk, 3 bulk in half of smem)")
+    ap.add_argument("--small-kernel", type=int, default=0, choices=[0, 1, 2, 3, 4],
+                    help="with --row: decode kernel (0 auto, 1 register ring, 2 bulk, 3 bulk in half of smem, 4 one-shot)")
     ap.add_argument("--sdpa-kernel", type=int, default=0, choices=[0, 1, 2],
                     help="with --row: decode attention (0 auto, 1 CUDA cores, 2 tensor cores)")
     args = ap.parse_args()

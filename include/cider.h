@@ -339,11 +339,15 @@ CIDER_API cider_status_t cider_test_set_gemm_variant(int variant);
  * cider_sdpa_decode_workspace_bytes after setting it. */
 CIDER_API cider_status_t cider_test_set_sdpa_kernel(int kernel);
 /* Selects the decode-shaped kernel of the small-M path for later calls
- * (process-wide): 0 = automatic (default), 1 = the register-ring kernel,
- * 2 = the bulk-staged kernel with the whole shared memory, 3 = the
- * bulk-staged kernel within half of it.  Shapes a bulk plan cannot hold take
- * the register-ring kernel either way.  Lets tests and measurements compare
- * the kernels on the same shapes. */
+ * (process-wide): 0 = automatic (default: the one-shot kernel, which requests
+ * all of a CTA's weights before using any, where its plan fits -- M <= 4 and
+ * at most 12 passes of 512 weights per warp -- else the register-ring
+ * kernel), 1 = the register-ring kernel, 2 = the bulk-staged kernel with the
+ * whole shared memory, 3 = the bulk-staged kernel within half of it, 4 = the
+ * one-shot kernel where its plan fits.  Shapes a selected kernel's plan
+ * cannot hold take the register-ring kernel.  The W8A16 products have no
+ * one-shot form (0, 1 and 4 select their register-ring kernel).  Lets tests
+ * and measurements compare the kernels on the same shapes. */
 CIDER_API cider_status_t cider_test_set_small_m_kernel(int kernel);
 /* Selects, for later calls (process-wide), how the per-channel linear
  * (cider_w8a8_linear_pc and the workspace-free form) quantizes its

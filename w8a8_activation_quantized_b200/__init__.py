@@ -446,7 +446,7 @@ def cider_test_set_sdpa_kernel(kernel: int):
 
 
 def cider_test_set_small_m_kernel(kernel: int):
-    """0 automatic, 1 register ring, 2 bulk-staged, 3 bulk-staged within half of shared memory."""
+    """0 automatic, 1 register ring, 2 bulk-staged, 3 bulk-staged within half of shared memory, 4 one-shot."""
     _check("cider_test_set_small_m_kernel", lib().cider_test_set_small_m_kernel(kernel))
 
 

@@ -761,7 +761,7 @@ cider_status_t cider_test_set_sdpa_kernel(int kernel) {
 
 cider_status_t cider_test_set_small_m_kernel(int kernel) {
     if (set_small_m_kernel(kernel) != cudaSuccess)
-        return fail(CIDER_ERR_INVALID_ARG, "kernel %d outside [0, 3]", kernel);
+        return fail(CIDER_ERR_INVALID_ARG, "kernel %d outside [0, 4]", kernel);
     return CIDER_OK;
 }
 

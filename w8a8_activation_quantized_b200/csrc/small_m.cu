@@ -25,6 +25,7 @@
 // warp's final shuffle reduction adds the lanes.  With one warp per row
 // (S = 1) a warp writes its outputs directly; otherwise the slices combine
 // through shared memory.
+#include <algorithm>
 #include <atomic>
 
 #include "cider_device.cuh"
@@ -246,6 +247,265 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
                 step(ring[r], ring_s[r], blk);
             }
             blk += gridDim.x;
+        }
+    }
+}
+
+// ---- one-shot decode kernel (1 <= M <= 4) ----------------------------------
+// The same quantize + dot + dequant, organised so that all of a CTA's weight
+// bytes are requested at once, before any is used.  Measured on B200 (a 26 MB
+// weight matrix, launches back to back in a CUDA graph): with each SM's whole
+// share in flight at once the bytes land in about 4.2 us; loads issued in
+// rounds (a ring of a few loads per thread) take 6-9 us, each round adding a
+// DRAM round trip.  The weights come by bulk copies (the copy engine), not
+// per-thread loads: as many per-thread loads as that needs fill the SM's
+// load/store queue faster than DRAM drains it, and every later load, store
+// or shared-memory access of the CTA then waits behind them (a global load
+// issued behind them took ~3 us, the quantization of x ~2.4 us).
+//
+// Work split.  One CTA of 1024 threads per SM; CTA b owns the contiguous
+// weight rows [b N / G, (b+1) N / G), so the CTAs differ by at most one row.
+// Thread 0 requests the activation rows (one bulk copy) and then the CTA's
+// weight rows in pieces of at most 16 KB, each on its own mbarrier; the
+// weight scales follow as 4-byte cp.async copies.  The CTA quantizes the
+// activation rows as soon as they land.  The weight rows are cut into passes
+// (32 consecutive 16-byte chunks of one row, the last pass of a row possibly
+// partial) and the 32 warps take equal contiguous runs of passes, so a run
+// may start and end inside a row; a warp waits only for the pieces its
+// passes lie in.  A lane adds up the dot products of its chunks of one row;
+// at the end of a row (or of its run) the warp reduces and lane 0 writes the
+// row's partial sum into a per-row slot indexed by the warp's place among the
+// warps that meet the row.  The output pass adds a row's slots in warp order,
+// so results do not depend on timing.  Per group, each lane scales its
+// chunk's exact INT32 dot by its group's scale (scale_w[g] * acc_g, summed in
+// another order).
+constexpr int kShotThreads = 1024;
+constexpr int kShotWarps = kShotThreads / 32;
+constexpr int kShotPieceBytes = 16 * 1024;  // weight bytes per bulk copy
+constexpr int kShotMaxPieces = 15;          // 15 x 16 KB covers the shared memory
+constexpr int kShotSmemBytes = 226 * 1024;  // dynamic shared memory (the static part stays below 1 KB)
+
+struct ShotGeom {
+    int ppr;       // passes per weight row
+    int slots;     // per-row slots for the partial sums of the warps that meet the row
+    int ngroups;   // per-group modes: K / gs
+    int x_off;     // shared-memory byte offsets (the weight rows start at 0): activation rows, then their codes;
+    int sw_off;    // weight scales;
+    int part_off;  // row partial sums
+};
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <typename TX, bool PG, bool W4, int MAXM>
+__global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __restrict__ x, int M, int K,
+                                                                  const uint8_t* __restrict__ w,
+                                                                  const float* __restrict__ sw, int N, int gs,
+                                                                  void* __restrict__ y, int ydt, ShotGeom geo,
+                                                                  unsigned* status) {
+    extern __shared__ __align__(128) uint8_t s_raw[];
+    const uint8_t* s_w = s_raw;                                      // [rows][row bytes]
+    uint8_t* s_x = s_raw + geo.x_off;                                // [M][K] of TX, then [M][K] codes
+    int8_t* s_q = reinterpret_cast<int8_t*>(s_x);
+    float* s_sw = reinterpret_cast<float*>(s_raw + geo.sw_off);      // per group [rows][K / gs], per channel [rows]
+    float* s_part = reinterpret_cast<float*>(s_raw + geo.part_off);  // [rows][slots][MAXM]
+    __shared__ float s_sx[MAXM];
+    __shared__ float s_red[MAXM][kShotWarps];
+    __shared__ __align__(8) uint64_t s_bar[kShotMaxPieces + 1];      // the weight pieces, then the activation rows
+    __shared__ int s_abort;
+    volatile int* abort_flag = &s_abort;
+    uint64_t* xbar = &s_bar[kShotMaxPieces];
+    constexpr int KC = W4 ? 32 : 16;  // weights per 16-byte chunk
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row_bytes = W4 ? K / 2 : K;
+    const int nch = K / KC;
+    const int ppr = geo.ppr;
+    const int n0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / gridDim.x);
+    const int n1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / gridDim.x);
+    const int rows = n1 - n0;
+    const int wbytes = rows * row_bytes;                             // < 226 KB, by the plan
+    const int npieces = (wbytes + kShotPieceBytes - 1) / kShotPieceBytes;
+    const int P = rows * ppr;                          // passes of this CTA
+    const int pw = (P + kShotWarps - 1) / kShotWarps;  // passes per warp
+    const int q0 = warp * pw;
+    const int np = min(pw, P - q0);                    // this warp's passes (may be <= 0)
+    const int r0 = np > 0 ? q0 / ppr : 0;              // the row, and the pass within it, where the run starts
+    const int kp0 = np > 0 ? q0 - r0 * ppr : 0;
+    const int nx = K / 8;                              // 16-byte chunks of a row of x (M * nx <= 2 * threads, by the plan)
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int i = 0; i <= kShotMaxPieces; ++i) mbar_init(&s_bar[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
+
+    if (threadIdx.x == 0) {
+        const uint32_t xbytes = static_cast<uint32_t>(M) * K * sizeof(TX);
+        mbar_arrive_expect_tx(xbar, xbytes);
+        bulk_load(s_x, x, xbytes, xbar);
+        const uint8_t* src = w + static_cast<int64_t>(n0) * row_bytes;
+        for (int c = 0; c < npieces; ++c) {
+            const int off = c * kShotPieceBytes;
+            const int sz = min(kShotPieceBytes, wbytes - off);
+            mbar_arrive_expect_tx(&s_bar[c], sz);
+            bulk_load(s_raw + off, src + off, sz, &s_bar[c]);
+        }
+    }
+    {
+        const int ns = PG ? rows * geo.ngroups : rows;
+        const uint32_t sw0 = smem_u32(s_sw);
+        for (int i = threadIdx.x; i < ns; i += kShotThreads) {
+            if (PG) {
+                const int g = i / rows, r = i - g * rows;  // read along n (contiguous)
+                cp_async4(sw0 + (r * geo.ngroups + g) * 4u, sw + static_cast<int64_t>(g) * N + n0 + r);
+            } else {
+                cp_async4(sw0 + i * 4u, sw + n0 + i);
+            }
+        }
+        cp_async_commit();
+    }
+
+    // quantize the M activation rows: each thread takes (at most) two 16-byte
+    // chunks into registers, so the codes can overwrite the rows afterwards
+    const bool x_ok = mbar_wait(xbar, 0, status, abort_flag);
+    uint4 xv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+    float amax[MAXM];
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) amax[m] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int i = threadIdx.x + j * kShotThreads;  // chunk i % nx of row i / nx
+        if (i < M * nx && x_ok) {
+            xv[j] = *reinterpret_cast<const uint4*>(s_x + static_cast<int64_t>(i) * 16);
+            const int m = i / nx;
+            const float a = absmax_to_f32<TX>(absmax8<TX>(xv[j], typename Pack2<TX>::type{}));
+#pragma unroll
+            for (int mm = 0; mm < MAXM; ++mm)
+                if (mm == m) amax[mm] = fmaxf(amax[mm], a);
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) {
+        if (m < M) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax[m] = fmaxf(amax[m], __shfl_xor_sync(0xffffffffu, amax[m], o));
+            if (lane == 0) s_red[m][warp] = amax[m];
+        }
+    }
+    __syncthreads();  // every read of the staged rows is done: the codes may overwrite them
+    if (threadIdx.x < M) {
+        float a = s_red[threadIdx.x][0];
+        for (int i = 1; i < kShotWarps; ++i) a = fmaxf(a, s_red[threadIdx.x][i]);
+        s_sx[threadIdx.x] = act_scale(a);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int i = threadIdx.x + j * kShotThreads;
+        if (i < M * nx) {
+            const int m = i / nx, c = i - m * nx;
+            const float sc = s_sx[m];
+            float f[8];
+            unpack8_f32<TX>(xv[j], f);
+            *reinterpret_cast<uint2*>(s_q + static_cast<int64_t>(m) * K + 8 * c) = quant8_codes(f, sc, act_rcp(sc));
+        }
+    }
+    cp_async_wait_all();  // this thread's scale copies
+    __syncthreads();      // codes and every thread's scales visible to the CTA
+
+    // dot products, one row segment of the run at a time: wait for the pieces
+    // the segment lies in, walk its passes, then reduce over the warp and
+    // store the row's partial sum (every condition below is warp-uniform)
+    if (np > 0) {
+        const int r_last = (q0 + np - 1) / ppr;
+        int ready = (r0 * row_bytes + kp0 * 512) / kShotPieceBytes;  // the first piece not yet waited for
+        bool ok = true;
+        for (int r = r0; r <= r_last; ++r) {
+            const int kp_lo = max(q0, r * ppr) - r * ppr;
+            const int kp_hi = min(q0 + np, (r + 1) * ppr) - r * ppr;
+            const int seg_end = r * row_bytes + min(kp_hi * 512, row_bytes);  // one past the segment's last byte
+            while (ok && ready <= (seg_end - 1) / kShotPieceBytes) ok = mbar_wait(&s_bar[ready++], 0, status, abort_flag);
+            int iacc[MAXM];
+            float facc[MAXM];
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) { iacc[m] = 0; facc[m] = 0.0f; }
+            if (ok) {
+                const uint8_t* wrow = s_w + r * row_bytes + lane * 16;
+                const float* srow = s_sw + r * geo.ngroups;
+#pragma unroll 4
+                for (int kp = kp_lo; kp < kp_hi; ++kp) {
+                    const int kc = kp * 32 + lane;
+                    if (kc < nch) {
+                        const uint4 wv = *reinterpret_cast<const uint4*>(wrow + kp * 512);
+                        const int k0 = kc * KC;
+                        const float gsc = PG ? srow[k0 / gs] : 0.0f;
+#pragma unroll
+                        for (int m = 0; m < MAXM; ++m) {
+                            if (m < M) {
+                                const int d = chunk_dot<W4>(wv, s_q + static_cast<int64_t>(m) * K, k0);
+                                if (PG)
+                                    facc[m] = fmaf(static_cast<float>(d), gsc, facc[m]);
+                                else
+                                    iacc[m] += d;
+                            }
+                        }
+                    }
+                }
+            }
+            const int slot = warp - (r * ppr) / pw;  // this warp's place among the row's warps
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) {
+                if (m < M) {
+                    float v;
+                    if (PG) {
+                        float a = facc[m];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+                        v = a;
+                    } else {
+                        v = __int_as_float(__reduce_add_sync(0xffffffffu, iacc[m]));
+                    }
+                    if (lane == 0) s_part[(r * geo.slots + slot) * MAXM + m] = v;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // outputs: a row's partial sums in warp order, then the dequant
+    for (int t = threadIdx.x; t < rows * M; t += kShotThreads) {
+        const int m = t / rows, r = t - m * rows;
+        const int wa = (r * ppr) / pw, wb = ((r + 1) * ppr - 1) / pw;
+        float out;
+        if (PG) {
+            float a = 0.0f;
+            for (int wi = wa; wi <= wb; ++wi) a += s_part[(r * geo.slots + (wi - wa)) * MAXM + m];
+            out = a * s_sx[m];
+        } else {
+            int a = 0;
+            for (int wi = wa; wi <= wb; ++wi) a += __float_as_int(s_part[(r * geo.slots + (wi - wa)) * MAXM + m]);
+            out = static_cast<float>(a) * s_sx[m] * s_sw[r];
+        }
+        const int64_t o = static_cast<int64_t>(m) * N + n0 + r;
+        if (ydt == 1)
+            static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(out);
+        else
+            static_cast<__half*>(y)[o] = __float2half_rn(out);
+    }
+    // A timed-out wait left the status flagged and the CTA's waits skipped;
+    // bulk copies may still be in flight, so give them (bounded) time to land
+    // before the CTA's shared memory is released.
+    if (*abort_flag && threadIdx.x == 0) {
+        const unsigned long long t0 = global_timer_ns();
+        for (int c = 0; c <= kShotMaxPieces; ++c) {
+            if (c < npieces || c == kShotMaxPieces)
+                while (!mbar_try_wait(&s_bar[c], 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+                }
         }
     }
 }
@@ -842,8 +1102,9 @@ static cudaError_t launch_small_m_t(const void* x, int M, int K, const void* w, 
 // false when fewer than three stages fit, or a slice needs more than 8 chunks
 // per lane; those calls take k_small_m.
 constexpr int kBulkSmemBytes = 225 * 1024;
-// test override of the decode kernel: 0 automatic, 1 register ring, 2 bulk
-// with the whole shared memory, 3 bulk within half of it
+// test override of the decode kernel: 0 automatic (one-shot where its plan
+// fits, else the register ring), 1 register ring, 2 bulk with the whole shared
+// memory, 3 bulk within half of it, 4 one-shot where its plan fits
 static std::atomic<int> g_small_kernel{0};
 static int bulk_smem_budget() { return g_small_kernel.load() == 3 ? 110 * 1024 : kBulkSmemBytes; }
 // With a16 (the W8A16 product) the activation rows are staged as fp32 pairs,
@@ -901,6 +1162,59 @@ static cudaError_t launch_bulk_ppl(const void* x, int M, int K, const void* w, c
     return launch_bulk_t<TX, PG, W4, MAXM, 8>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
 }
 
+// Plan of k_small_m_shot: one CTA per SM (at most one per row), at most two
+// 16-byte chunks of x per thread, and the CTA's weight rows, activation rows,
+// weight scales and row partial sums within one CTA's shared memory; false
+// otherwise (those calls take the register-ring kernel).
+static bool shot_plan(int M, int K, int N, bool pg, bool w4, int gs, int num_sms, ShotGeom& g, int& grid,
+                      int& smem) {
+    if (M < 1 || M > 4 || N < 1) return false;
+    if (M * (K / 8) > 2 * kShotThreads) return false;
+    const int64_t row_bytes = w4 ? K / 2 : K;
+    const int nch = K / (w4 ? 32 : 16);
+    g.ppr = (nch + 31) / 32;
+    grid = std::min(num_sms, N);
+    const int64_t rows_max = (N + grid - 1) / grid, rows_min = N / grid;
+    const int64_t wbytes = rows_max * row_bytes;
+    if (wbytes > static_cast<int64_t>(kShotMaxPieces) * kShotPieceBytes) return false;
+    const int64_t pw_min = std::max<int64_t>(1, (rows_min * g.ppr + kShotWarps - 1) / kShotWarps);
+    // a row's ppr passes meet at most ceil(ppr / pw) + 1 warps' runs
+    g.slots = static_cast<int>(std::min<int64_t>(kShotWarps, (g.ppr + pw_min - 1) / pw_min + 1));
+    g.ngroups = pg ? K / gs : 0;
+    auto al = [](int64_t v) { return (v + 127) & ~int64_t(127); };
+    int64_t off = al(wbytes);
+    g.x_off = static_cast<int>(off);
+    off += al(static_cast<int64_t>(M) * K * 2);  // the activation rows (16-bit), then their codes
+    g.sw_off = static_cast<int>(off);
+    off += al(rows_max * (pg ? g.ngroups : 1) * 4);
+    g.part_off = static_cast<int>(off);
+    off += al(rows_max * g.slots * 4 * 4);  // MAXM <= 4 partial sums per slot
+    if (off > kShotSmemBytes) return false;
+    smem = static_cast<int>(off);
+    return true;
+}
+
+template <typename TX, bool PG, bool W4, int MAXM>
+static cudaError_t launch_shot_t(const void* x, int M, int K, const void* w, const float* sw, int N, int gs, void* y,
+                                 int ydt, const ShotGeom& geo, int grid, int smem, unsigned* status,
+                                 cudaStream_t st) {
+    auto kern = k_small_m_shot<TX, PG, W4, MAXM>;
+    if (smem > 32 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(kern, grid, kShotThreads, smem, st, static_cast<const TX*>(x), M, K,
+                      static_cast<const uint8_t*>(w), sw, N, gs, y, ydt, geo, status);
+}
+
+template <typename TX, bool PG, bool W4>
+static cudaError_t launch_shot_m(const void* x, int M, int K, const void* w, const float* sw, int N, int gs, void* y,
+                                 int ydt, const ShotGeom& geo, int grid, int smem, unsigned* status,
+                                 cudaStream_t st) {
+    if (M == 1) return launch_shot_t<TX, PG, W4, 1>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, smem, status, st);
+    return launch_shot_t<TX, PG, W4, 4>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, smem, status, st);
+}
+
 template <bool PG, bool W4>
 static cudaError_t launch_small_m_v(const void* x, int xdt, int M, int K, const void* w, const float* sw, int N,
                                     int gs, void* y, int ydt, int num_sms, unsigned* status, cudaStream_t st) {
@@ -910,7 +1224,14 @@ static cudaError_t launch_small_m_v(const void* x, int xdt, int M, int K, const 
     // slower on B200 (M = 1, N = 10240, K = 2560: 11.3 / 10.0 us with the
     // whole / half of shared memory against 8.8 us); it stays selectable
     const int sel = g_small_kernel.load();
-    if (M <= 4 && sel >= 2 && bulk_plan(M, K, N, PG, W4, gs, num_sms, geo, grid)) {
+    ShotGeom sg;
+    int sgrid = 0, ssmem = 0;
+    if ((sel == 0 || sel == 4) && shot_plan(M, K, N, PG, W4, gs, num_sms, sg, sgrid, ssmem)) {
+        if (xdt == 1)
+            return launch_shot_m<__nv_bfloat16, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, sg, sgrid, ssmem, status, st);
+        return launch_shot_m<__half, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, sg, sgrid, ssmem, status, st);
+    }
+    if (M <= 4 && (sel == 2 || sel == 3) && bulk_plan(M, K, N, PG, W4, gs, num_sms, geo, grid)) {
         if (xdt == 1) {
             if (M == 1)
                 return launch_bulk_ppl<__nv_bfloat16, PG, W4, 1>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
@@ -992,7 +1313,8 @@ cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* 
     // runs when the test switch selects it and its plan fits
     BulkGeom geo;
     int grid = 0;
-    if (g_small_kernel.load() >= 2 && bulk_plan(M, K, N, gs > 0, false, gs, num_sms, geo, grid, true)) {
+    const int sel = g_small_kernel.load();
+    if ((sel == 2 || sel == 3) && bulk_plan(M, K, N, gs > 0, false, gs, num_sms, geo, grid, true)) {
         if (gs > 0) {
             if (xdt == 1) return launch_mv_bulk_m<__nv_bfloat16, true>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
             return launch_mv_bulk_m<__half, true>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
@@ -1009,7 +1331,7 @@ cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* 
 }
 
 cudaError_t set_small_m_kernel(int k) {
-    if (k < 0 || k > 3) return cudaErrorInvalidValue;
+    if (k < 0 || k > 4) return cudaErrorInvalidValue;
     g_small_kernel.store(k);
     return cudaSuccess;
 }
