@@ -261,16 +261,26 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
 // per-thread loads: as many per-thread loads as that needs fill the SM's
 // load/store queue faster than DRAM drains it, and every later load, store
 // or shared-memory access of the CTA then waits behind them (a global load
-// issued behind them took ~3 us, the quantization of x ~2.4 us).
+// issued behind them took ~3 us, the quantization of x ~2.4 us).  At most
+// kShotWindow pieces are in flight per CTA: with every piece requested at
+// once, all of an SM's pieces land within the last ~0.5 us and the dot
+// products (bound by shared-memory bandwidth) start only then; with a window
+// of a few 16 KB pieces the first lands after ~1.4 us, the rest follow at the
+// SM's share of DRAM bandwidth, and the arithmetic overlaps the stream
+// (measured on B200: 6.6 against 7.0 us per launch for the copies and the
+// same shared-memory reads; windows of 2 to 8 pieces of 8 to 32 KB were
+// within 0.4 us of each other on the decode shapes, 6 x 16 KB among the best).
 //
 // Work split.  One CTA of 1024 threads per SM; CTA b owns the contiguous
 // weight rows [b N / G, (b+1) N / G), so the CTAs differ by at most one row.
-// Thread 0 requests the activation rows (one bulk copy) and then the CTA's
-// weight rows in pieces of at most 16 KB, each on its own mbarrier; the
-// weight scales follow as 4-byte cp.async copies.  The CTA quantizes the
+// The last warp is the producer: one lane requests the activation rows (one
+// bulk copy) and then the CTA's weight rows in pieces of at most 16 KB, each
+// on its own mbarrier, issuing piece c once piece c - kShotWindow has landed.
+// The other 31 warps (synchronising among themselves on a named barrier)
+// stage the weight scales as 4-byte cp.async copies and quantize the
 // activation rows as soon as they land.  The weight rows are cut into passes
 // (32 consecutive 16-byte chunks of one row, the last pass of a row possibly
-// partial) and the 32 warps take equal contiguous runs of passes, so a run
+// partial) and the 31 warps take equal contiguous runs of passes, so a run
 // may start and end inside a row; a warp waits only for the pieces its
 // passes lie in.  A lane adds up the dot products of its chunks of one row;
 // at the end of a row (or of its run) the warp reduces and lane 0 writes the
@@ -281,6 +291,9 @@ __global__ void __launch_bounds__(kSmallThreads, 2) k_small_m(const TX* __restri
 // another order).
 constexpr int kShotThreads = 1024;
 constexpr int kShotWarps = kShotThreads / 32;
+constexpr int kShotCompute = kShotWarps - 1;       // compute warps (the last warp is the producer)
+constexpr int kShotComputeThreads = kShotCompute * 32;
+constexpr int kShotWindow = 6;                     // weight pieces in flight per CTA
 constexpr int kShotPieceBytes = 16 * 1024;  // weight bytes per bulk copy
 constexpr int kShotMaxPieces = 15;          // 15 x 16 KB covers the shared memory
 constexpr int kShotSmemBytes = 226 * 1024;  // dynamic shared memory (the static part stays below 1 KB)
@@ -299,6 +312,10 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// barrier of the compute warps only (the producer warp never joins it)
+__device__ __forceinline__ void shot_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kShotComputeThreads) : "memory");
+}
 
 template <typename TX, bool PG, bool W4, int MAXM>
 __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __restrict__ x, int M, int K,
@@ -313,7 +330,7 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
     float* s_sw = reinterpret_cast<float*>(s_raw + geo.sw_off);      // per group [rows][K / gs], per channel [rows]
     float* s_part = reinterpret_cast<float*>(s_raw + geo.part_off);  // [rows][slots][MAXM]
     __shared__ float s_sx[MAXM];
-    __shared__ float s_red[MAXM][kShotWarps];
+    __shared__ float s_red[MAXM][kShotCompute];
     __shared__ __align__(8) uint64_t s_bar[kShotMaxPieces + 1];      // the weight pieces, then the activation rows
     __shared__ int s_abort;
     volatile int* abort_flag = &s_abort;
@@ -328,13 +345,13 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
     const int rows = n1 - n0;
     const int wbytes = rows * row_bytes;                             // < 226 KB, by the plan
     const int npieces = (wbytes + kShotPieceBytes - 1) / kShotPieceBytes;
-    const int P = rows * ppr;                          // passes of this CTA
-    const int pw = (P + kShotWarps - 1) / kShotWarps;  // passes per warp
+    const int P = rows * ppr;                              // passes of this CTA
+    const int pw = (P + kShotCompute - 1) / kShotCompute;  // passes per compute warp
     const int q0 = warp * pw;
     const int np = min(pw, P - q0);                    // this warp's passes (may be <= 0)
     const int r0 = np > 0 ? q0 / ppr : 0;              // the row, and the pass within it, where the run starts
     const int kp0 = np > 0 ? q0 - r0 * ppr : 0;
-    const int nx = K / 8;                              // 16-byte chunks of a row of x (M * nx <= 2 * threads, by the plan)
+    const int nx = K / 8;  // 16-byte chunks of a row of x (M * nx <= 2 * compute threads, by the plan)
     if (threadIdx.x == 0) {
         s_abort = 0;
         for (int i = 0; i <= kShotMaxPieces; ++i) mbar_init(&s_bar[i], 1);
@@ -344,22 +361,40 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
     pdl_wait();
     pdl_trigger();
 
-    if (threadIdx.x == 0) {
-        const uint32_t xbytes = static_cast<uint32_t>(M) * K * sizeof(TX);
-        mbar_arrive_expect_tx(xbar, xbytes);
-        bulk_load(s_x, x, xbytes, xbar);
-        const uint8_t* src = w + static_cast<int64_t>(n0) * row_bytes;
-        for (int c = 0; c < npieces; ++c) {
-            const int off = c * kShotPieceBytes;
-            const int sz = min(kShotPieceBytes, wbytes - off);
-            mbar_arrive_expect_tx(&s_bar[c], sz);
-            bulk_load(s_raw + off, src + off, sz, &s_bar[c]);
+    if (warp == kShotCompute) {
+        // the producer: the activation rows, then the weight pieces through the window
+        if (lane == 0) {
+            const uint32_t xbytes = static_cast<uint32_t>(M) * K * sizeof(TX);
+            mbar_arrive_expect_tx(xbar, xbytes);
+            bulk_load(s_x, x, xbytes, xbar);
+            const uint8_t* src = w + static_cast<int64_t>(n0) * row_bytes;
+            int issued = 0;
+            for (int c = 0; c < npieces; ++c) {
+                if (c >= kShotWindow && !mbar_wait(&s_bar[c - kShotWindow], 0, status, abort_flag)) break;
+                const int off = c * kShotPieceBytes;
+                const int sz = min(kShotPieceBytes, wbytes - off);
+                mbar_arrive_expect_tx(&s_bar[c], sz);
+                bulk_load(s_raw + off, src + off, sz, &s_bar[c]);
+                issued = c + 1;
+            }
+            if (*abort_flag) {
+                // a wait timed out (the status is flagged): let every issued
+                // copy land, within a bound, before the CTA's shared memory
+                // is released
+                const unsigned long long t0 = global_timer_ns();
+                for (int c = 0; c <= issued; ++c) {
+                    uint64_t* bar = c < issued ? &s_bar[c] : xbar;
+                    while (!mbar_try_wait(bar, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+                    }
+                }
+            }
         }
+        return;
     }
     {
         const int ns = PG ? rows * geo.ngroups : rows;
         const uint32_t sw0 = smem_u32(s_sw);
-        for (int i = threadIdx.x; i < ns; i += kShotThreads) {
+        for (int i = threadIdx.x; i < ns; i += kShotComputeThreads) {
             if (PG) {
                 const int g = i / rows, r = i - g * rows;  // read along n (contiguous)
                 cp_async4(sw0 + (r * geo.ngroups + g) * 4u, sw + static_cast<int64_t>(g) * N + n0 + r);
@@ -379,7 +414,7 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
     for (int m = 0; m < MAXM; ++m) amax[m] = 0.0f;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        const int i = threadIdx.x + j * kShotThreads;  // chunk i % nx of row i / nx
+        const int i = threadIdx.x + j * kShotComputeThreads;  // chunk i % nx of row i / nx
         if (i < M * nx && x_ok) {
             xv[j] = *reinterpret_cast<const uint4*>(s_x + static_cast<int64_t>(i) * 16);
             const int m = i / nx;
@@ -397,16 +432,16 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
             if (lane == 0) s_red[m][warp] = amax[m];
         }
     }
-    __syncthreads();  // every read of the staged rows is done: the codes may overwrite them
+    shot_sync();  // every read of the staged rows is done: the codes may overwrite them
     if (threadIdx.x < M) {
         float a = s_red[threadIdx.x][0];
-        for (int i = 1; i < kShotWarps; ++i) a = fmaxf(a, s_red[threadIdx.x][i]);
+        for (int i = 1; i < kShotCompute; ++i) a = fmaxf(a, s_red[threadIdx.x][i]);
         s_sx[threadIdx.x] = act_scale(a);
     }
-    __syncthreads();
+    shot_sync();
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        const int i = threadIdx.x + j * kShotThreads;
+        const int i = threadIdx.x + j * kShotComputeThreads;
         if (i < M * nx) {
             const int m = i / nx, c = i - m * nx;
             const float sc = s_sx[m];
@@ -416,7 +451,7 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
         }
     }
     cp_async_wait_all();  // this thread's scale copies
-    __syncthreads();      // codes and every thread's scales visible to the CTA
+    shot_sync();          // codes and every thread's scales visible to the compute warps
 
     // dot products, one row segment of the run at a time: wait for the pieces
     // the segment lies in, walk its passes, then reduce over the warp and
@@ -475,10 +510,10 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
             }
         }
     }
-    __syncthreads();
+    shot_sync();
 
     // outputs: a row's partial sums in warp order, then the dequant
-    for (int t = threadIdx.x; t < rows * M; t += kShotThreads) {
+    for (int t = threadIdx.x; t < rows * M; t += kShotComputeThreads) {
         const int m = t / rows, r = t - m * rows;
         const int wa = (r * ppr) / pw, wb = ((r + 1) * ppr - 1) / pw;
         float out;
@@ -496,17 +531,6 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
             static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(out);
         else
             static_cast<__half*>(y)[o] = __float2half_rn(out);
-    }
-    // A timed-out wait left the status flagged and the CTA's waits skipped;
-    // bulk copies may still be in flight, so give them (bounded) time to land
-    // before the CTA's shared memory is released.
-    if (*abort_flag && threadIdx.x == 0) {
-        const unsigned long long t0 = global_timer_ns();
-        for (int c = 0; c <= kShotMaxPieces; ++c) {
-            if (c < npieces || c == kShotMaxPieces)
-                while (!mbar_try_wait(&s_bar[c], 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-                }
-        }
     }
 }
 
@@ -1169,7 +1193,7 @@ static cudaError_t launch_bulk_ppl(const void* x, int M, int K, const void* w, c
 static bool shot_plan(int M, int K, int N, bool pg, bool w4, int gs, int num_sms, ShotGeom& g, int& grid,
                       int& smem) {
     if (M < 1 || M > 4 || N < 1) return false;
-    if (M * (K / 8) > 2 * kShotThreads) return false;
+    if (M * (K / 8) > 2 * kShotComputeThreads) return false;
     const int64_t row_bytes = w4 ? K / 2 : K;
     const int nch = K / (w4 ? 32 : 16);
     g.ppr = (nch + 31) / 32;
@@ -1177,9 +1201,9 @@ static bool shot_plan(int M, int K, int N, bool pg, bool w4, int gs, int num_sms
     const int64_t rows_max = (N + grid - 1) / grid, rows_min = N / grid;
     const int64_t wbytes = rows_max * row_bytes;
     if (wbytes > static_cast<int64_t>(kShotMaxPieces) * kShotPieceBytes) return false;
-    const int64_t pw_min = std::max<int64_t>(1, (rows_min * g.ppr + kShotWarps - 1) / kShotWarps);
+    const int64_t pw_min = std::max<int64_t>(1, (rows_min * g.ppr + kShotCompute - 1) / kShotCompute);
     // a row's ppr passes meet at most ceil(ppr / pw) + 1 warps' runs
-    g.slots = static_cast<int>(std::min<int64_t>(kShotWarps, (g.ppr + pw_min - 1) / pw_min + 1));
+    g.slots = static_cast<int>(std::min<int64_t>(kShotCompute, (g.ppr + pw_min - 1) / pw_min + 1));
     g.ngroups = pg ? K / gs : 0;
     auto al = [](int64_t v) { return (v + 127) & ~int64_t(127); };
     int64_t off = al(wbytes);
