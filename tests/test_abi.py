@@ -146,23 +146,25 @@ def test_sdpa_plan_covers_every_key(H_q, H_kv, N, sms, kernel):
     """kernel 1: the CUDA-core kernels' cut (head tiles of 1, 2 or 4 query
     heads, chunks of whole 16-key streams); kernel 0 (automatic) takes the
     tensor-core cut for 2 <= H_q / H_kv <= 16 (one CTA per KV head and chunk
-    of 128 .. 512 keys, in whole 128-key tiles) when its chunks fit the merge."""
+    of 1 .. 15 whole 128-key tiles: the fewest tiles that put every CTA in one
+    wave of one CTA per SM) when its chunks fit the merge."""
     cider.cider_test_set_sdpa_kernel(kernel)
     try:
         th, tiles, chunk, chunks = cider.cider_test_sdpa_plan(H_q, H_kv, N, sms)
     finally:
         cider.cider_test_set_sdpa_kernel(0)
     G = H_q // H_kv
-    tc = kernel == 0 and 2 <= G <= 16 and -(-N // 512) <= 1024
+    tc = kernel == 0 and 2 <= G <= 16 and -(-N // 1920) <= 1024
     assert 1 <= chunks <= 1024
     assert (chunks - 1) * chunk < N <= chunks * chunk  # every chunk has a key; every key has a chunk
     if tc:
         assert th == G and tiles == 1
-        assert chunk % 128 == 0 and 128 <= chunk <= 512
-        # about two CTAs per SM: the keys over ceil(2 * SMs / H_kv) chunks, rounded up
-        # to whole 128-key tiles, between one and four tiles
-        target = -(-2 * sms // H_kv)
-        assert chunk == min(max(-(-(-(-N // target)) // 128) * 128, 128), 512)
+        assert chunk % 128 == 0 and 128 <= chunk <= 1920
+        tiles, t = -(-N // 128), 1
+        while t < 15 and H_kv * -(-tiles // t) > sms:
+            t += 1
+        assert chunk == 128 * t
+        assert H_kv * chunks <= sms or t == 15
     else:
         assert th in (1, 2, 4) and th * tiles == G
         assert th == (4 if G % 4 == 0 else 2 if G % 2 == 0 else 1)
