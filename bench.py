@@ -84,7 +84,8 @@ class ClockSampler:
     def __init__(self, device_index, period_s=0.002):
         self.dev = device_index
         self.period = period_s
-        self.samples = []  # (sm_mhz, reasons_mask)
+        self.samples = []  # (sm_mhz, reasons_mask): background samples
+        self.polled = []   # samples taken by poll_until, while the timed work runs
         self.max_mhz = None
         self._stop = threading.Event()
         self._nvml = None
@@ -130,6 +131,8 @@ class ClockSampler:
     def __enter__(self):
         try:
             pynvml, h = self._handle()
+            self._nvml = (pynvml, h)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
             self._t = threading.Thread(target=self._loop_nvml, args=(pynvml, h), daemon=True)
         except Exception:
             self._t = threading.Thread(target=self._loop_smi, daemon=True)
@@ -137,19 +140,41 @@ class ClockSampler:
         time.sleep(0.01)
         return self
 
+    def _sample_nvml(self):
+        pynvml, h = self._nvml
+        clk = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        try:
+            rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except AttributeError:
+            rs = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        self.polled.append((float(clk), int(rs)))
+
+    def poll_until(self, event):
+        """Samples from this thread while queued GPU work runs, until `event`
+        completes: a timed region shorter than the background period still
+        gets samples taken under load (at least one, before the first check)."""
+        if self._nvml is None:
+            return
+        while True:
+            self._sample_nvml()
+            if event.query():
+                return
+
     def __exit__(self, *a):
         self._stop.set()
         self._t.join(timeout=10)
 
     def summary(self):
-        if not self.samples:
+        # samples taken while the timed work ran, when there are any
+        samples = self.polled or self.samples
+        if not samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
         mask = 0
-        for _, m in self.samples:
+        for _, m in samples:
             mask |= m
-        return {"sm_mhz": statistics.median(c for c, _ in self.samples), "sm_max_mhz": self.max_mhz,
+        return {"sm_mhz": statistics.median(c for c, _ in samples), "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(n for n, b in self.REASONS.items() if mask & b),
-                "samples": len(self.samples)}
+                "samples": len(samples)}
 
 
 # ----------------------------------------------------------------------------- timing
@@ -309,6 +334,7 @@ def run_cider(args):
         a.record(st)
         g.replay()
         b.record(st)
+        clk.poll_until(b)
         torch.cuda.synchronize()
     _barrier(ws)
     ms = _max_over_ranks(a.elapsed_time(b) / args.steps, ws, device)
