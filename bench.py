@@ -681,6 +681,7 @@ def run_row(args):
                           "GB/s": (M * K * 3 + M * 4) / (ms * 1e-3) / 1e9}), flush=True)
         return 0
     cider.cider_test_set_small_m_kernel(args.small_kernel)
+    cider.cider_test_set_gemm_variant(args.gemm_variant)
     x = torch.from_numpy(synth.activations(M, K, 1000 + M)).to(device)
     W = torch.from_numpy(synth.weights(N, K, 1001)).to(device)
     if kind == "pc":
@@ -727,6 +728,8 @@ def main():
                     help="with --row: where the per-channel linear quantizes (inside the GEMM launch or not)")
     ap.add_argument("--small-kernel", type=int, default=0, choices=[0, 1, 2, 3, 4],
                     help="with --row: decode kernel (0 auto, 1 register ring, 2 bulk, 3 bulk in half of smem, 4 one-shot)")
+    ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1, 2, 3, 4],
+                    help="with --row: per-channel GEMM (0 auto, 1 128x128, 2 128x256, 3 CTA pair, 4 128x80)")
     ap.add_argument("--sdpa-kernel", type=int, default=0, choices=[0, 1, 2],
                     help="with --row: decode attention (0 auto, 1 CUDA cores, 2 tensor cores)")
     args = ap.parse_args()
