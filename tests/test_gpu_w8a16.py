@@ -3,7 +3,8 @@
 kernels) against the oracle's W8A16 modes, within the row-relative
 tolerance, for 1 <= M <= 4, both input dtypes and both output dtypes,
 including shapes whose K is split across warps, whose rows wrap the ring of
-shared-memory stages, and the argument checks."""
+shared-memory stages, the one-shot kernel's corners (forced against the
+register ring), and the argument checks."""
 import numpy as np
 import pytest
 import torch
@@ -132,3 +133,52 @@ def test_w8a16_mv_bulk_kernel(kernel):
         cider.cider_test_set_small_m_kernel(0)
     check_y(y_pc, oracle.w8a16_linear_pc(x, qc, sc), oracle.F16)
     check_y(y_pg, oracle.w8a16_linear_pg(x, qg, sg, gs), oracle.F16)
+
+
+# ---- the one-shot kernel (A16 mode) against the register ring -----------------
+
+@pytest.mark.parametrize("kernel", [1, 4])
+@pytest.mark.parametrize("M", [1, 3])
+@pytest.mark.parametrize("mode,N,K,gs", [("pc", 10240, 2560, 0), ("pg", 2560, 10240, 64), ("pg", 2560, 10240, 128),
+                                         ("pc", 144, 16384, 0), ("pg", 264, 16384, 128), ("pc", 152, 1040, 0),
+                                         ("pg", 296, 1088, 64), ("pg", 8, 128, 64)])
+def test_w8a16_one_shot_and_register_ring(kernel, M, mode, N, K, gs):
+    """Both W8A16 kernels on the one-shot kernel's corners: the decode shapes,
+    rows met by many warps (K = 16384), partial last passes (K = 1040, 1088)
+    and fewer rows than SMs."""
+    if K == 16384 and M > 1:
+        pytest.skip("M x K beyond the staged activations of the register-ring kernel")
+    x = act(M, K, seed=M + N + K + gs + kernel)
+    W = synth.weights(N, K, seed=N + K + gs)
+    cider.cider_test_set_small_m_kernel(kernel)
+    try:
+        if mode == "pc":
+            qw, sw = oracle.quantize_weight_pc(W)
+            y = cider.cider_w8a16_mv_pc(dev_bits(x, oracle.F16), dev(qw), dev(sw))
+            ref = oracle.w8a16_linear_pc(x, qw, sw)
+        else:
+            qw, sw = oracle.quantize_weight_pg(W, gs)
+            y = cider.cider_w8a16_mv_pg(dev_bits(x, oracle.F16), dev(qw), dev(np.ascontiguousarray(sw.T)), gs)
+            ref = oracle.w8a16_linear_pg(x, qw, sw, gs)
+    finally:
+        cider.cider_test_set_small_m_kernel(0)
+    check_y(y, ref, oracle.F16)
+
+
+@pytest.mark.parametrize("mode", ["pc", "pg"])
+def test_w8a16_one_shot_bf16(mode):
+    M, N, K, gs = 2, 2056, 4096, 64
+    x = act(M, K, seed=5, dt=oracle.BF16)
+    x[1] = 0
+    W = synth.weights(N, K, seed=6)
+    if mode == "pc":
+        qw, sw = oracle.quantize_weight_pc(W)
+        y = cider.cider_w8a16_mv_pc(dev_bits(x, oracle.BF16), dev(qw), dev(sw), out_dtype=torch.bfloat16)
+        ref = oracle.w8a16_linear_pc(x, qw, sw, xdt=oracle.BF16, ydt=oracle.BF16)
+    else:
+        qw, sw = oracle.quantize_weight_pg(W, gs)
+        y = cider.cider_w8a16_mv_pg(dev_bits(x, oracle.BF16), dev(qw), dev(np.ascontiguousarray(sw.T)), gs,
+                                    out_dtype=torch.bfloat16)
+        ref = oracle.w8a16_linear_pg(x, qw, sw, gs, xdt=oracle.BF16, ydt=oracle.BF16)
+    check_y(y, ref, oracle.BF16)
+    assert not y[1].any()

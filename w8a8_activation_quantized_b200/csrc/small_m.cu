@@ -27,6 +27,7 @@
 // through shared memory.
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 
 #include "cider_device.cuh"
 #include "cider_kernels.h"
@@ -312,12 +313,51 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// fp32 dot of one 16-byte weight chunk with 16 activations of type TX read
+// from shared memory (W8A16): each weight is widened exactly (its sign bit
+// flipped, the byte placed under the exponent of 2^23 by one permute, 2^23 +
+// 128 subtracted), each activation pair converted to an fp32 pair, and the
+// products summed by packed FMAs, two per instruction.
+template <typename TX>
+__device__ __forceinline__ float chunk_dot_x16(const uint4& wv, const uint8_t* xs) {
+    constexpr float kOff = 8388608.0f + 128.0f;  // 2^23 + 128
+    const uint64_t neg_off = pack_f32x2(-kOff, -kOff);
+    const uint4 xa = *reinterpret_cast<const uint4*>(xs);
+    const uint4 xb = *reinterpret_cast<const uint4*>(xs + 16);
+    const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+    const uint32_t wd[4] = {wv.x ^ 0x80808080u, wv.y ^ 0x80808080u, wv.z ^ 0x80808080u, wv.w ^ 0x80808080u};
+    uint64_t acc = 0;  // two fp32 partial sums
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t v = wd[i];
+        const uint64_t w01 = f32x2_add(
+            (static_cast<uint64_t>(__byte_perm(v, 0x4B000000u, 0x7651)) << 32) | __byte_perm(v, 0x4B000000u, 0x7650),
+            neg_off);
+        const uint64_t w23 = f32x2_add(
+            (static_cast<uint64_t>(__byte_perm(v, 0x4B000000u, 0x7653)) << 32) | __byte_perm(v, 0x4B000000u, 0x7652),
+            neg_off);
+        float2 x01, x23;
+        if constexpr (std::is_same<TX, __half>::value) {
+            x01 = __half22float2(*reinterpret_cast<const __half2*>(&xw[2 * i]));
+            x23 = __half22float2(*reinterpret_cast<const __half2*>(&xw[2 * i + 1]));
+        } else {
+            x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[2 * i]));
+            x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[2 * i + 1]));
+        }
+        acc = f32x2_fma(w01, pack_f32x2(x01.x, x01.y), acc);
+        acc = f32x2_fma(w23, pack_f32x2(x23.x, x23.y), acc);
+    }
+    return lo_f32(acc) + hi_f32(acc);
+}
+
 // barrier of the compute warps only (the producer warp never joins it)
 __device__ __forceinline__ void shot_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kShotComputeThreads) : "memory");
 }
 
-template <typename TX, bool PG, bool W4, int MAXM>
+// A16: the W8A16 product (no activation quantization): the rows of x stay in
+// shared memory as they arrive and the dot products are taken in fp32.
+template <typename TX, bool PG, bool W4, int MAXM, bool A16 = false>
 __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __restrict__ x, int M, int K,
                                                                   const uint8_t* __restrict__ w,
                                                                   const float* __restrict__ sw, int N, int gs,
@@ -405,9 +445,10 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
         cp_async_commit();
     }
 
+    const bool x_ok = mbar_wait(xbar, 0, status, abort_flag);
+    if constexpr (!A16) {
     // quantize the M activation rows: each thread takes (at most) two 16-byte
     // chunks into registers, so the codes can overwrite the rows afterwards
-    const bool x_ok = mbar_wait(xbar, 0, status, abort_flag);
     uint4 xv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
     float amax[MAXM];
 #pragma unroll
@@ -450,6 +491,7 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
             *reinterpret_cast<uint2*>(s_q + static_cast<int64_t>(m) * K + 8 * c) = quant8_codes(f, sc, act_rcp(sc));
         }
     }
+    }
     cp_async_wait_all();  // this thread's scale copies
     shot_sync();          // codes and every thread's scales visible to the compute warps
 
@@ -482,11 +524,17 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
 #pragma unroll
                         for (int m = 0; m < MAXM; ++m) {
                             if (m < M) {
-                                const int d = chunk_dot<W4>(wv, s_q + static_cast<int64_t>(m) * K, k0);
-                                if (PG)
-                                    facc[m] = fmaf(static_cast<float>(d), gsc, facc[m]);
-                                else
-                                    iacc[m] += d;
+                                if constexpr (A16) {
+                                    const float d = chunk_dot_x16<TX>(
+                                        wv, s_x + (static_cast<int64_t>(m) * K + k0) * static_cast<int64_t>(sizeof(TX)));
+                                    facc[m] = PG ? fmaf(d, gsc, facc[m]) : facc[m] + d;
+                                } else {
+                                    const int d = chunk_dot<W4>(wv, s_q + static_cast<int64_t>(m) * K, k0);
+                                    if (PG)
+                                        facc[m] = fmaf(static_cast<float>(d), gsc, facc[m]);
+                                    else
+                                        iacc[m] += d;
+                                }
                             }
                         }
                     }
@@ -497,7 +545,7 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
             for (int m = 0; m < MAXM; ++m) {
                 if (m < M) {
                     float v;
-                    if (PG) {
+                    if (PG || A16) {
                         float a = facc[m];
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
@@ -517,7 +565,11 @@ __global__ void __launch_bounds__(kShotThreads, 1) k_small_m_shot(const TX* __re
         const int m = t / rows, r = t - m * rows;
         const int wa = (r * ppr) / pw, wb = ((r + 1) * ppr - 1) / pw;
         float out;
-        if (PG) {
+        if (A16) {
+            float a = 0.0f;
+            for (int wi = wa; wi <= wb; ++wi) a += s_part[(r * geo.slots + (wi - wa)) * MAXM + m];
+            out = PG ? a : a * s_sw[r];
+        } else if (PG) {
             float a = 0.0f;
             for (int wi = wa; wi <= wb; ++wi) a += s_part[(r * geo.slots + (wi - wa)) * MAXM + m];
             out = a * s_sx[m];
@@ -1191,9 +1243,9 @@ static cudaError_t launch_bulk_ppl(const void* x, int M, int K, const void* w, c
 // weight scales and row partial sums within one CTA's shared memory; false
 // otherwise (those calls take the register-ring kernel).
 static bool shot_plan(int M, int K, int N, bool pg, bool w4, int gs, int num_sms, ShotGeom& g, int& grid,
-                      int& smem) {
+                      int& smem, bool a16 = false) {
     if (M < 1 || M > 4 || N < 1) return false;
-    if (M * (K / 8) > 2 * kShotComputeThreads) return false;
+    if (!a16 && M * (K / 8) > 2 * kShotComputeThreads) return false;  // the quantizer's two chunks a thread
     const int64_t row_bytes = w4 ? K / 2 : K;
     const int nch = K / (w4 ? 32 : 16);
     g.ppr = (nch + 31) / 32;
@@ -1218,11 +1270,11 @@ static bool shot_plan(int M, int K, int N, bool pg, bool w4, int gs, int num_sms
     return true;
 }
 
-template <typename TX, bool PG, bool W4, int MAXM>
+template <typename TX, bool PG, bool W4, int MAXM, bool A16 = false>
 static cudaError_t launch_shot_t(const void* x, int M, int K, const void* w, const float* sw, int N, int gs, void* y,
                                  int ydt, const ShotGeom& geo, int grid, int smem, unsigned* status,
                                  cudaStream_t st) {
-    auto kern = k_small_m_shot<TX, PG, W4, MAXM>;
+    auto kern = k_small_m_shot<TX, PG, W4, MAXM, A16>;
     if (smem > 32 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
@@ -1330,14 +1382,37 @@ static cudaError_t launch_mv_bulk_m(const void* x, int M, int K, const int8_t* w
 }
 
 
+template <typename TX, bool PG>
+static cudaError_t launch_mv_shot(const void* x, int M, int K, const int8_t* w, const float* sw, int N, int gs, void* y,
+                                  int ydt, const ShotGeom& geo, int grid, int smem, unsigned* status, cudaStream_t st) {
+    if (M == 1) return launch_shot_t<TX, PG, false, 1, true>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, smem, status, st);
+    return launch_shot_t<TX, PG, false, 4, true>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, smem, status, st);
+}
+
 cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* w, const float* sw, int N, int gs,
                             void* y, int ydt, int num_sms, unsigned* status, cudaStream_t st) {
-    // the register-ring kernel is the default (M = 1, N = 10240, K = 2560:
-    // 7.9 us against 11.3 us for the bulk-staged one); the bulk-staged kernel
-    // runs when the test switch selects it and its plan fits
+    // Per group, the one-shot kernel (A16 mode) where its plan fits (M = 1,
+    // N = 2560, K = 10240: 11.5 / 12.2 us at gs = 128 / 64 against 14.9 /
+    // 15.2 us for the register ring); per channel the register ring, whose
+    // fp32 activation pairs are staged once (M = 1, N = 10240, K = 2560:
+    // 9.95 us against 10.1 us for the one-shot kernel, which widens the
+    // activations for every chunk).  The test switch's 4 forces the one-shot
+    // kernel for both; the bulk-staged kernel (11.3 us per channel) runs when
+    // the switch selects it and its plan fits.
     BulkGeom geo;
     int grid = 0;
     const int sel = g_small_kernel.load();
+    ShotGeom sg;
+    int sgrid = 0, ssmem = 0;
+    if (((sel == 0 && gs > 0) || sel == 4) &&
+        shot_plan(M, K, N, gs > 0, false, gs > 0 ? gs : 64, num_sms, sg, sgrid, ssmem, true)) {
+        if (gs > 0) {
+            if (xdt == 1) return launch_mv_shot<__nv_bfloat16, true>(x, M, K, w, sw, N, gs, y, ydt, sg, sgrid, ssmem, status, st);
+            return launch_mv_shot<__half, true>(x, M, K, w, sw, N, gs, y, ydt, sg, sgrid, ssmem, status, st);
+        }
+        if (xdt == 1) return launch_mv_shot<__nv_bfloat16, false>(x, M, K, w, sw, N, 0, y, ydt, sg, sgrid, ssmem, status, st);
+        return launch_mv_shot<__half, false>(x, M, K, w, sw, N, 0, y, ydt, sg, sgrid, ssmem, status, st);
+    }
     if ((sel == 2 || sel == 3) && bulk_plan(M, K, N, gs > 0, false, gs, num_sms, geo, grid, true)) {
         if (gs > 0) {
             if (xdt == 1) return launch_mv_bulk_m<__nv_bfloat16, true>(x, M, K, w, sw, N, gs, y, ydt, geo, grid, status, st);
