@@ -621,7 +621,8 @@ def bench_stack(device, pk, steps, warmup, layers=36, M=2048):
 ROW_CASES = {
     # name: (kind, M, N, K, gs)
     "pc_m1": ("pc", 1, 10240, 2560, 0), "pc_m128": ("pc", 128, 10240, 2560, 0),
-    "pc_m1024": ("pc", 1024, 10240, 2560, 0), "pc_m4096": ("pc", 4096, 10240, 2560, 0),
+    "pc_m512": ("pc", 512, 10240, 2560, 0), "pc_m1024": ("pc", 1024, 10240, 2560, 0),
+    "pc_m2048": ("pc", 2048, 10240, 2560, 0), "pc_m4096": ("pc", 4096, 10240, 2560, 0),
     "pc_m8192": ("pc", 8192, 10240, 2560, 0),
     "pg128_m1": ("pg", 1, 2560, 10240, 128), "pg128_m4096": ("pg", 4096, 2560, 10240, 128),
     "mv_m1": ("mv", 1, 10240, 2560, 0), "mvpg64_m1": ("mvpg", 1, 2560, 10240, 64),
@@ -728,8 +729,9 @@ def main():
                     help="with --row: where the per-channel linear quantizes (inside the GEMM launch or not)")
     ap.add_argument("--small-kernel", type=int, default=0, choices=[0, 1, 2, 3, 4],
                     help="with --row: decode kernel (0 auto, 1 register ring, 2 bulk, 3 bulk in half of smem, 4 one-shot)")
-    ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1, 2, 3, 4],
-                    help="with --row: per-channel GEMM (0 auto, 1 128x128, 2 128x256, 3 CTA pair, 4 128x80)")
+    ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1, 2, 3, 4, 5],
+                    help="with --row: per-channel GEMM (0 auto, 1 128x128, 2 128x256, 3 CTA pair 256x256, "
+                         "4 128x80, 5 CTA pair 256x192)")
     ap.add_argument("--sdpa-kernel", type=int, default=0, choices=[0, 1, 2],
                     help="with --row: decode attention (0 auto, 1 CUDA cores, 2 tensor cores)")
     args = ap.parse_args()

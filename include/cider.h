@@ -328,7 +328,8 @@ CIDER_API cider_status_t cider_test_gemm_i32_grouped(const int8_t* q, const int8
 /* Forces the kernel variant of the per-channel and INT32 GEMM for later calls
  * (process-wide): 0 = automatic (default), 1 = single-CTA 128x128 tiles,
  * 2 = single-CTA 128x256 tiles, 3 = CTA-pair 256x256 tiles, 4 = single-CTA
- * 128x80 tiles.  Lets tests cover every variant on small shapes. */
+ * 128x80 tiles, 5 = CTA-pair 256x192 tiles.  Lets tests cover every variant
+ * on small shapes.  Outside [0, 5]: CIDER_ERR_INVALID_ARG, nothing changes. */
 CIDER_API cider_status_t cider_test_set_gemm_variant(int variant);
 /* Selects the decode-attention kernels for later calls (process-wide):
  * 0 = automatic (default: the tensor-core kernel when 2 <= H_q / H_kv <= 16,

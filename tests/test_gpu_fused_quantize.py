@@ -83,7 +83,7 @@ def test_fused_codes_and_outputs(M, N, K):
     assert torch.equal(y.view(torch.int16), y_plain.view(torch.int16))
 
 
-@pytest.mark.parametrize("variant", [1, 2, 3, 4])
+@pytest.mark.parametrize("variant", [1, 2, 3, 4, 5])
 def test_fused_every_variant(variant):
     M, N, K = 300, 1032, 2560
     x = act(M, K, seed=variant)

@@ -1,6 +1,6 @@
 """Every kernel variant of the per-channel GEMM against the oracle on small and
 ragged shapes: single-CTA 128x80, 128x128 and 128x256 tiles, and the CTA-pair
-256x256 tile (tcgen05.mma.cta_group::2).  Bit-exact INT32 accumulators, and
+256x256 and 256x192 tiles (tcgen05.mma.cta_group::2).  Bit-exact INT32 accumulators, and
 the fused dequant within the row-relative tolerance."""
 import numpy as np
 import pytest
@@ -13,7 +13,7 @@ from tests.parity import act, check_y, dev, dev_bits
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = {"single128": 1, "single256": 2, "pair256": 3, "single80": 4}
+VARIANTS = {"single128": 1, "single256": 2, "pair256": 3, "single80": 4, "pair192": 5}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -73,6 +73,29 @@ def test_pair_is_chosen_for_large_m():
     assert torch.equal(y_pair, y_single) and torch.equal(y_auto, y_pair)
     rows = np.arange(0, M, 97)
     check_y(y_auto, oracle.linear_pc(x[rows], qw, sw), oracle.F16, rows=rows)
+
+
+@pytest.mark.parametrize("dt", [oracle.F16, oracle.BF16])
+def test_pair192_is_chosen_at_m1024(dt):
+    """M = 1024, N = 10240, K = 2560: 160 square pair tiles leave the 74 SM
+    pairs a last round of 12 tiles, so the automatic choice takes the 256 x 192
+    tile (216 tiles, three full rounds of narrower tiles).  Exact INT32 sums and
+    the same dequant expression: equal to the square tile bit for bit; the
+    last N tile holds 64 valid columns of 192."""
+    M, N, K = 1024, 10240, 2560
+    cider.cider_set_small_m_threshold(4)
+    x = act(M, K, seed=1024, dt=dt)
+    qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed=1025))
+    xd, wd, sd = dev_bits(x, dt), dev(qw), dev(sw)
+    outs = {}
+    for name, v in (("auto", 0), ("pair192", 5), ("pair256", 3)):
+        cider.cider_test_set_gemm_variant(v)
+        outs[name] = cider.cider_w8a8_linear_pc(xd, wd, sd)
+    cider.cider_test_set_gemm_variant(0)
+    torch.cuda.synchronize()
+    assert torch.equal(outs["auto"], outs["pair192"]) and torch.equal(outs["pair192"], outs["pair256"])
+    rows = np.concatenate([np.arange(0, M, 61), [M - 1]])
+    check_y(outs["auto"], oracle.linear_pc(x[rows], qw, sw, xdt=dt, ydt=dt), dt, rows=rows)
 
 
 # ---------------------------------------------------------------- split K of the pair kernel

@@ -436,7 +436,8 @@ def cider_test_gemm_i32_grouped(q, w, gs, acc_g=None, stream=None):
 
 
 def cider_test_set_gemm_variant(variant: int):
-    """0 automatic, 1 single-CTA 128x128, 2 single-CTA 128x256, 3 CTA-pair 256x256, 4 single-CTA 128x80."""
+    """0 automatic, 1 single-CTA 128x128, 2 single-CTA 128x256, 3 CTA-pair 256x256, 4 single-CTA 128x80,
+    5 CTA-pair 256x192."""
     _check("cider_test_set_gemm_variant", lib().cider_test_set_gemm_variant(variant))
 
 

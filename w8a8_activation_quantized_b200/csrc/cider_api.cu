@@ -164,7 +164,7 @@ bool use_fused_quantize(int mode, int64_t M) {
 }
 constexpr int kMaxSplits = 16;
 
-int pick_variant(int64_t M, int64_t N, int num_sms);
+int pick_variant(int64_t M, int64_t N, int64_t K, int num_sms);
 
 // Split-K plan of a persistent GEMM with `slots` resident tiles (SMs, or SM
 // pairs): the tiles that fill whole rounds run over all of K; the R tiles of
@@ -198,9 +198,12 @@ SplitPlan grouped_split_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
 // Per-channel GEMM: only on the CTA-pair 256 x 256 tile, whose k-block takes
 // ~0.27 us; measured at K = 2560 (M = 1024 and 8192) the split does not pay,
 // so it needs >= 32 saved k-blocks (K of roughly 5120 and more).
-SplitPlan pc_split_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
-    if (pick_variant(M, N, num_sms) != kGemmPair) return {0, 1, 0, 0};
+SplitPlan pair_split_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
     return split_plan(((M + 255) / 256) * ((N + 255) / 256), 256 * 256, num_sms / 2, K, 32);
+}
+SplitPlan pc_split_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
+    if (pick_variant(M, N, K, num_sms) != kGemmPair) return {0, 1, 0, 0};
+    return pair_split_plan(M, N, K, num_sms);
 }
 
 // Bytes of 32-bit partial sums: one tile-sized slot per K piece of a tail tile.
@@ -213,12 +216,23 @@ size_t part_bytes(const SplitPlan& sp) {
 // leave SMs idle -- 128x128 or 128x80, whichever gives the busiest SM fewer
 // weight rows to stream (rounds of the persistent grid x tile width; at
 // M <= 128, N = 10240 that is one round of 128 tiles of 80 rows instead of
-// 80 tiles of 128 rows on 80 SMs).
-int pick_variant(int64_t M, int64_t N, int num_sms) {
+// 80 tiles of 128 rows on 80 SMs).  Among the pair tiles, 256x192 replaces
+// 256x256 when the square tile's tail is not split along K and the busiest
+// pair streams fewer operand bytes: rounds x (128 rows of A + BN / 2 rows of B)
+// per k-block and CTA.  Measured on B200 (N = 10240, K = 2560) the time per
+// round follows those bytes: M = 512 and 1024 (2 and 3 rounds either way)
+// gain 3.7% and 2.0% with 192 columns, M = 2048 (5 rounds of 256 against 6 of
+// 192) loses 10% and M = 4096 (9 against 12) 16% -- which this rule avoids.
+int pick_variant(int64_t M, int64_t N, int64_t K, int num_sms) {
     const int forced = g_gemm_variant.load();
     if (forced != kGemmAuto) return forced;
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
-    if (M > 128 && pair_tiles >= num_sms / 2) return kGemmPair;
+    if (M > 128 && pair_tiles >= num_sms / 2) {
+        const int64_t pairs = num_sms / 2, mbp = (M + 255) / 256;
+        auto bytes_per_pair = [&](int64_t bn) { return (mbp * ((N + bn - 1) / bn) + pairs - 1) / pairs * (128 + bn / 2); };
+        if (pair_split_plan(M, N, K, num_sms).splits == 1 && bytes_per_pair(192) < bytes_per_pair(256)) return kGemmPair192;
+        return kGemmPair;
+    }
     const int64_t mb = (M + 127) / 128;
     const int64_t tiles256 = mb * ((N + 255) / 256);
     if (tiles256 >= num_sms) return kGemmSingle256;
@@ -245,7 +259,7 @@ cider_status_t run_gemm(int mode, const int8_t* q, const float* sx, int64_t M, i
     L.K = static_cast<int>(K);
     L.gs = static_cast<int>(gs);
     L.ydt = ydt;
-    L.variant = (mode == kModePC || mode == kModeI32) ? pick_variant(M, N, d->num_sms) : kGemmSingle128;
+    L.variant = (mode == kModePC || mode == kModeI32) ? pick_variant(M, N, K, d->num_sms) : kGemmSingle128;
     L.full_tiles = sp.full_tiles;
     L.splits = sp.splits;
     L.part = part;
@@ -772,8 +786,8 @@ cider_status_t cider_test_set_fused_quantize(int mode) {
 }
 
 cider_status_t cider_test_set_gemm_variant(int variant) {
-    if (variant < kGemmAuto || variant > kGemmSingle80)
-        return fail(CIDER_ERR_INVALID_ARG, "variant %d outside [0, 4]", variant);
+    if (variant < kGemmAuto || variant > kGemmPair192)
+        return fail(CIDER_ERR_INVALID_ARG, "variant %d outside [0, 5]", variant);
     g_gemm_variant.store(variant);
     return CIDER_OK;
 }

@@ -206,6 +206,23 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
                  "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
+// L2 prefetches.  They write neither shared memory nor registers, only bring
+// global lines into the L2, which every SM reads through (the point of
+// coherence), so a kernel may issue them before its grid-dependency wait: a
+// load after the wait still sees every write of the kernel before it.  Used
+// for the streamed operands of the HBM-bound kernels, so the next launch's
+// CTAs start pulling their bytes while the previous launch drains.
+// Untiled: `gsrc` 16-byte aligned, `bytes` a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* gsrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gsrc), "r"(bytes) : "memory");
+}
+// One box of a 2-D tensor map (no multicast; c0 innermost, as in tma_load_2d).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N of this thread's bulk groups still read shared memory.
 template <int N>

@@ -24,7 +24,7 @@ enum : int {
 
 // Kernel variants of the per-channel GEMM (the grouped modes always use the
 // single-CTA kernel with 128-wide N tiles).
-enum : int { kGemmAuto = 0, kGemmSingle128 = 1, kGemmSingle256 = 2, kGemmPair = 3, kGemmSingle80 = 4 };
+enum : int { kGemmAuto = 0, kGemmSingle128 = 1, kGemmSingle256 = 2, kGemmPair = 3, kGemmSingle80 = 4, kGemmPair192 = 5 };
 
 // Grid-barrier slots of the launches that quantize inside the GEMM: the host
 // hands out slots in turn, so launches that run at the same time (up to this
@@ -40,7 +40,7 @@ struct GemmLaunch {
     void* y;           // output
     int M, N, K, gs;
     int ydt;           // 0 fp16, 1 bf16
-    int variant;       // per-channel modes: kGemmSingle128, kGemmSingle256 or kGemmPair
+    int variant;       // per-channel modes: one of the kGemm* kernel variants above
     int full_tiles;    // grouped modes: tiles that run over all of K (the rest are split)
     int splits;        // grouped modes: K pieces of each later tile (1 = no split)
     float* part;       // grouped modes with splits > 1: fp32 partial sums, [piece slot][128][128]

@@ -12,6 +12,9 @@ constexpr int kBK = 128;          // int8 K values per stage = one 128-byte swiz
 constexpr int kUmmaK = 32;        // K per kind::i8 MMA
 constexpr int kGroupM = 8;        // tile raster: 8 M-blocks share each N-block in turn
 constexpr int kSmemBudget = 196608;
+// k-blocks of a CTA's first weight tile requested into L2 before its
+// grid-dependency wait (one 128-wide k-block per request).
+constexpr int kPrefetchKBlocks = 32;
 constexpr int kSmemMax = 232448;  // dynamic shared memory per CTA on sm_100
 
 struct GemmArgs {

@@ -156,6 +156,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        // With one block row of A (M <= 128: the weights are nearly all the
+        // bytes), the first tile's weight tiles go into L2 before the wait on
+        // the previous kernel (the quantizer that writes A), so they stream
+        // while it runs (see prefetch_l2_bulk for why this is safe).
+        // Measured on B200, N = 10240, K = 2560: M = 128 15.2 -> 14.4 us; at
+        // M = 1024 and 4096 (the quantizer already streaming at full rate)
+        // it cost 0.7-0.9%, so larger M does not prefetch.
+        if (p.num_m_blocks == 1 && blockIdx.x < num_tiles) {
+            int mb, nb;
+            tile_coords(blockIdx.x, p.num_m_blocks, p.num_n_blocks, mb, nb);
+            for (int kb = 0; kb < p.num_k_blocks && kb < kPrefetchKBlocks; ++kb) tma_prefetch_l2_2d(&tmB, kb * kBK, nb * BN);
+        }
     }
     if (warp == 1) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tc_fence_before();
@@ -301,22 +313,24 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// CTA-pair kernel (per-channel and INT32 modes): one 256 x 256 output tile per
-// cluster of two CTAs with tcgen05.mma.cta_group::2.  Each CTA stages its own
-// 128 rows of A and its half (128 rows) of B, so per multiply-add a CTA moves
-// two thirds of the bytes of the single-CTA 128 x 256 tile.  The even CTA
-// (the pair's leader) issues the MMAs; its full barrier counts the TMA bytes of
-// both CTAs, the MMA commits arrive on both CTAs' barriers, and the epilogue
-// warps of both CTAs report to the leader's accumulator-empty barriers.
-// Each CTA's TMEM holds the accumulator rows of its own 128 rows of A.
+// CTA-pair kernel (per-channel and INT32 modes): one 256 x BN output tile per
+// cluster of two CTAs with tcgen05.mma.cta_group::2 (BN = 256, or 192 where
+// the narrower tile fills the SM pairs' last round better).  Each CTA stages
+// its own 128 rows of A and its half (BN / 2 rows) of B, so per multiply-add
+// a CTA moves two thirds of the bytes of the single-CTA 128 x 256 tile.  The
+// even CTA (the pair's leader) issues the MMAs; its full barrier counts the
+// TMA bytes of both CTAs, the MMA commits arrive on both CTAs' barriers, and
+// the epilogue warps of both CTAs report to the leader's accumulator-empty
+// barriers.  Each CTA's TMEM holds the accumulator rows of its own 128 rows of A.
 // ---------------------------------------------------------------------------
-struct PairCfg {
+template <int BN_>
+struct PairCfgN {
     static constexpr int BM = 256;                   // rows of the pair tile
-    static constexpr int BN = 256;                   // columns of the pair tile
+    static constexpr int BN = BN_;                   // columns of the pair tile
     static constexpr int A_BYTES = 128 * kBK;        // this CTA's rows of A
     static constexpr int B_BYTES = (BN / 2) * kBK;   // this CTA's half of B
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = kSmemBudget / STAGE_BYTES;  // 6
+    static constexpr int STAGES = kSmemBudget / STAGE_BYTES;  // 6 (BN 256), 7 (BN 192)
     static constexpr int ACC_BUFS = 2;
     static constexpr int TMEM_COLS = 512;
     static constexpr int EPI_WARPS = 8;                 // two per TMEM lane quarter
@@ -327,7 +341,12 @@ struct PairCfg {
     static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * ACC_BUFS) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_WARPS * STG_PER_WARP * STG_BYTES + BAR_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
+    // 32-column epilogue chunks per warp; the cta_group::2 M = 256 shape takes N % 16 == 0, N <= 256
+    static_assert(BN % 64 == 0 && BN <= 256, "pair tile width");
+    static_assert(ACC_BUFS * BN <= TMEM_COLS, "TMEM");
+    static_assert(B_BYTES % 1024 == 0, "stage bases on the 1024-byte swizzle atom");
 };
+using PairCfg = PairCfgN<256>;  // the split-K tail and its reduce use the square tile
 
 // 32 accumulators of one row -> 32 outputs, written as 4 swizzled 16-byte
 // chunks into row `r` of a 32 x 32 staging box laid out for the TMA 64-byte
@@ -364,11 +383,11 @@ __device__ __forceinline__ void load_scales32(const float* sw, int n0, int N, fl
     }
 }
 
-template <int MODE, typename TY>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
+template <int MODE, typename TY, int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfgN<BN>::THREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmP, GemmArgs p) {
-    using C = PairCfg;
+    using C = PairCfgN<BN>;
     constexpr int S = C::STAGES;
     constexpr int NB = C::ACC_BUFS;
     extern __shared__ uint8_t smem_raw[];
@@ -492,8 +511,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         }
         __syncwarp();
     } else {
-        // ---------------- epilogue (both CTAs): this CTA's 128 rows x 256 columns ----------------
-        // Warp w reads TMEM lanes 32*(w%4).. and columns [half*128, half*128+128) in
+        // ---------------- epilogue (both CTAs): this CTA's 128 rows x BN columns ----------------
+        // Warp w reads TMEM lanes 32*(w%4).. and columns [half*BN/2, (half+1)*BN/2) in
         // chunks of 32, loading chunk c+1 (and its scales) before converting chunk c.
         // Per-channel outputs go through a swizzled shared-memory box and a TMA store.
         if (p.x != nullptr) {
@@ -680,11 +699,12 @@ __global__ void __launch_bounds__(256) k_splitk_reduce_pc(const int32_t* __restr
     store_row8<TY>(y + static_cast<int64_t>(m) * p.N + n, v);
 }
 
-template <int MODE, typename TY>
+template <int MODE, typename TY, int BN>
 static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
+    using C = PairCfgN<BN>;
     CUtensorMap tmA, tmB, tmY, tmP;
     if (!make_map_2d(&tmA, L.q, L.K, L.M, kBK, 128, true)) return cudaErrorInvalidValue;
-    if (!make_map_2d(&tmB, L.w, L.K, L.N, kBK, PairCfg::BN / 2, true)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&tmB, L.w, L.K, L.N, kBK, C::BN / 2, true)) return cudaErrorInvalidValue;
     if (MODE == kModePC) {
         if (!make_map_out(&tmY, L.y, L.M, L.N, L.ydt)) return cudaErrorInvalidValue;
     } else {
@@ -695,8 +715,8 @@ static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
     a.N = L.N;
     a.K = L.K;
     a.gs = 0;
-    a.num_m_blocks = (L.M + PairCfg::BM - 1) / PairCfg::BM;
-    a.num_n_blocks = (L.N + PairCfg::BN - 1) / PairCfg::BN;
+    a.num_m_blocks = (L.M + C::BM - 1) / C::BM;
+    a.num_n_blocks = (L.N + C::BN - 1) / C::BN;
     a.num_k_blocks = (L.K + kBK - 1) / kBK;
     a.sx = L.sx;
     a.sw = L.sw;
@@ -708,8 +728,8 @@ static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
     a.sxout = const_cast<float*>(L.sx);
     a.fuse_slot = L.fuse_slot;
     const int tiles = a.num_m_blocks * a.num_n_blocks;
-    // split K of the tail tiles (per-channel with a partial-sum buffer only)
-    int splits = (MODE == kModePC && L.part != nullptr && L.splits > 1) ? L.splits : 1;
+    // split K of the tail tiles (per-channel square tiles with a partial-sum buffer only)
+    int splits = (MODE == kModePC && BN == PairCfg::BN && L.part != nullptr && L.splits > 1) ? L.splits : 1;
     const int full = splits > 1 ? std::min(std::max(L.full_tiles, 0), tiles) : tiles;
     a.kb_per_split = (a.num_k_blocks + splits - 1) / splits;
     a.splits = (a.num_k_blocks + a.kb_per_split - 1) / a.kb_per_split;
@@ -723,10 +743,10 @@ static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
     }
     const int units = a.full_tiles + (tiles - a.full_tiles) * a.splits;
     const int clusters = units < L.num_sms / 2 ? units : L.num_sms / 2;
-    auto kern = k_gemm_pair<MODE, TY>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
+    auto kern = k_gemm_pair<MODE, TY, BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(kern, 2 * clusters, PairCfg::THREADS, PairCfg::SMEM_BYTES, st, tmA, tmB, tmY, tmP, a);
+    e = launch_pdl(kern, 2 * clusters, C::THREADS, C::SMEM_BYTES, st, tmA, tmB, tmY, tmP, a);
     if (e != cudaSuccess || a.splits == 1) return e;
     return launch_pdl(k_splitk_reduce_pc<TY>, (tiles - a.full_tiles) * (PairCfg::BM / 8), 256, 0, st,
                       reinterpret_cast<const int32_t*>(L.part), a, static_cast<TY*>(L.y));
@@ -734,7 +754,8 @@ static cudaError_t launch_gemm_pair(const GemmLaunch& L, cudaStream_t st) {
 
 template <int MODE, typename TY>
 static cudaError_t launch_gemm_mode(const GemmLaunch& L, cudaStream_t st) {
-    if (L.variant == kGemmPair) return launch_gemm_pair<MODE, TY>(L, st);
+    if (L.variant == kGemmPair) return launch_gemm_pair<MODE, TY, 256>(L, st);
+    if (L.variant == kGemmPair192) return launch_gemm_pair<MODE, TY, 192>(L, st);
     if (L.variant == kGemmSingle128) return launch_gemm_cfg<GemmCfg<128, MODE>, TY>(L, st);
     if (L.variant == kGemmSingle80) return launch_gemm_cfg<GemmCfg<80, MODE>, TY>(L, st);
     return launch_gemm_cfg<GemmCfg<256, MODE>, TY>(L, st);

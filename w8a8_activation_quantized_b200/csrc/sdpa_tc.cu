@@ -142,7 +142,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sdpa_tc(const __grid_constant
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const T* __restrict__ q, int G, int N, int chunk,
                                                            int chunks, float qscale, float* __restrict__ part,
-                                                           uint32_t v_lbo, uint32_t v_sbo, unsigned* status) {
+                                                           uint32_t v_lbo, uint32_t v_sbo, int npre,
+                                                           unsigned* status) {
     constexpr bool BF = std::is_same<T, __nv_bfloat16>::value;
     constexpr int NP = BF ? 3 : 2;  // 16-bit parts of P
     extern __shared__ uint8_t smem_raw[];
@@ -176,6 +177,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sdpa_tc(const __grid_constant
         mbar_init(&odone, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_async_smem();
+        // The ring's first npre tiles into L2 before the wait on the previous
+        // kernel (a prefetch writes no shared memory, and the loads after the
+        // wait still see that kernel's writes): a CTA that starts while the
+        // previous launch drains streams meanwhile.
+        for (int i = 0; i < 2 * nt && i < npre; ++i) {
+            const CUtensorMap* map = i < nt ? &tmK : &tmV;
+            const int row = row0 + (i % nt) * kTcKeys;
+            tma_prefetch_l2_2d(map, 0, row);
+            tma_prefetch_l2_2d(map, 128, row);
+        }
     }
     if (warp == 1) tmem_alloc(&tmem_slot, kTcTmemCols);
     pdl_wait();
@@ -398,9 +409,17 @@ cudaError_t launch_tc(const void* q, const void* k, const void* v, int H_q, int 
     const bool swap = g_sdpa_kernel.load() == 3;
     const uint32_t lbo = swap ? 1024u : static_cast<uint32_t>(kTcTileBytes / 2);
     const uint32_t sbo = swap ? static_cast<uint32_t>(kTcTileBytes / 2) : 1024u;
+    // Prefetch the ring's first stages before the grid-dependency wait only
+    // when all of K and V fit in L2.  Measured on B200 (32 query heads,
+    // D = 128): GQA8 19.9 -> 19.4 us at N = 32K (67 MB) and 9.6 -> 9.0 us at
+    // 4K; GQA4 at 32K (134 MB, more than L2) 29.7 -> 30.4 us, so not there.
+    int dev = 0, l2 = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev)) != cudaSuccess) return e;
+    const int npre = 2 * rows * kSdpaD * 2 <= static_cast<uint64_t>(l2) ? kTcStages : 0;
     const dim3 grid(static_cast<unsigned>(p.chunks), static_cast<unsigned>(H_kv));
     e = launch_pdl(kern, grid, kTcThreads, smem, st, tmK, tmV, static_cast<const T*>(q), H_q / H_kv, N, p.chunk,
-                   p.chunks, qscale, part, lbo, sbo, status);
+                   p.chunks, qscale, part, lbo, sbo, npre, status);
     if (e != cudaSuccess) return e;
     return launch_sdpa_merge(part, p.chunks, out, H_q, std::is_same<T, __nv_bfloat16>::value ? 1 : 0, st);
 }
