@@ -633,6 +633,8 @@ ROW_CASES = {
     "w4a8_m2048": ("w4", 2048, 12288, 4096, 64), "w4a8pc_m2048": ("w4pc", 2048, 12288, 4096, 0),
     "stack_8b": ("stack", 2048, 0, 0, 0),
     "quant_m4096_k2560": ("quant", 4096, 0, 2560, 0), "quant_m8192_k10240": ("quant", 8192, 0, 10240, 0),
+    # offline conversion with percentile-clipped scales (p = 99.9): (kind, 0, N, K, gs)
+    "clip_pc": ("clip", 0, 10240, 2560, 0), "clip_pg64": ("clip", 0, 2560, 10240, 64),
     # decode attention: (kind, H_kv, N keys, 0, 0) with H_q = 32, D = 128
     "sdpa_mha_n32k": ("sdpa", 32, 32768, 0, 0), "sdpa_gqa4_n32k": ("sdpa", 8, 32768, 0, 0),
     "sdpa_gqa8_n32k": ("sdpa", 4, 32768, 0, 0), "sdpa_gqa8_n4k": ("sdpa", 4, 4096, 0, 0),
@@ -669,6 +671,19 @@ def run_row(args):
         cider.cider_device_status()
         print(json.dumps({"row": args.row, "kind": kind, "H_q": H_q, "H_kv": H_kv, "N": Nk, "ms": ms,
                           "GB/s": (kv_bytes + 2 * H_q * D * 2) / (ms * 1e-3) / 1e9}), flush=True)
+        return 0
+    if kind == "clip":  # percentile-clipped weight quantizer alone, weights rotated beyond L2
+        n = rotating(N * K * 5)
+        Ws = [torch.from_numpy(synth.weights(N, K, 4000 + i)).to(device) for i in range(n)]
+        if gs == 0:
+            ms = graph_time(lambda i: cider.cider_quantize_weight_pc_clip(Ws[i % n], 99.9), args.steps, args.warmup)
+        else:
+            ms = graph_time(lambda i: cider.cider_quantize_weight_pg_clip(Ws[i % n], gs, 99.9), args.steps,
+                            args.warmup)
+        cider.cider_device_status()
+        nbytes = N * K * 5 + N * (K // gs if gs else 1) * 4
+        print(json.dumps({"row": args.row, "kind": kind, "N": N, "K": K, "gs": gs, "ms": ms,
+                          "GB/s": nbytes / (ms * 1e-3) / 1e9}), flush=True)
         return 0
     if kind == "quant":  # activation quantization alone, inputs rotated beyond L2
         n = rotating(M * K * 3)

@@ -391,8 +391,8 @@ cudaError_t launch_quantize_weight(int mode, const float* W, int64_t N, int K, i
 // magnitude is the largest pattern r with at most k magnitudes below it
 // (|x| as an unsigned bit pattern orders like |x|).  Each of the 31 counting
 // passes (bit 31 of |x| is 0) counts for both statistics at once.  Exact for
-// any slab length; the conversion runs once per model, so the passes read
-// the row through L1 rather than holding it on chip.
+// any slab length.  A row of up to 4096 weights is held in registers for the
+// passes; a longer one is read through L1 each pass.
 
 __device__ __forceinline__ float clip_value(uint32_t r0, uint32_t r1, bool two, float t, float amax) {
     const float a = __uint_as_float(r0);
@@ -402,11 +402,193 @@ __device__ __forceinline__ float clip_value(uint32_t r0, uint32_t r1, bool two, 
 __device__ __forceinline__ int8_t clip_code(float x, float s) {
     return static_cast<int8_t>(max(quant_code(x, s), -127));
 }
+// clip_code without the division.  With r = 1/s correctly rounded, t = x * r
+// lies within a relative 1.5 * 2^-23 of the correctly rounded quotient (three
+// roundings of at most 2^-24 each), i.e. within 2^-15 of it below 128.  So
+// wherever t is more than 2^-14 from a halfway point k + 1/2 below 127.5,
+// rint(t) (taken by adding 1.5 * 2^23, as in quant8_codes) is the code, and
+// halfway points never reach this path, so ties-to-even and round-half-away
+// cannot differ.  Beyond 127.5 + 2^-14 every rounding of the quotient
+// saturates at +-127.  Anything else -- a near tie, s = 0, a NaN -- takes the
+// exact clip_code.
+__device__ __forceinline__ int8_t clip_code_fast(float x, float s, float r) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    constexpr float kMargin = 0x1p-14f;
+    const float t = __fmul_rn(x, r);
+    const float at = fabsf(t);
+    if (at < 127.5f - kMargin) {
+        const float v = __fadd_rn(t, kMagic);
+        const float d = __fsub_rn(t, __fsub_rn(v, kMagic));
+        if (fabsf(d) < 0.5f - kMargin) return static_cast<int8_t>(static_cast<int>(__fsub_rn(v, kMagic)));
+    } else if (at > 127.5f + kMargin && s != 0.0f) {
+        return static_cast<int8_t>(t > 0.0f ? 127 : -127);
+    }
+    return clip_code(x, s);
+}
+
+// High percentiles (the pages' 99.9) sit a few ranks below the maximum.  With
+// j = len - 1 - k0 the rank of the first statistic counted from the top, a
+// slab with j <= kClipTop is walked down through its distinct magnitudes
+// instead: the largest magnitude below the previous one, then how many
+// elements equal it, until the run of equal values that holds rank j.  That
+// takes at most j + 1 steps of two reductions (every step passes at least
+// one element) and gives the same order statistics, ties included; rank
+// j - 1 (the second statistic) is in the same run or is the previous value.
+constexpr int kClipTop = 12;
+
+// 256-thread block reductions: warp redux, then the 8 warps' values through
+// shared memory.  Two buffers alternate, so a call's writes never meet the
+// previous call's reads (the barrier of the call between them orders them).
+__device__ __forceinline__ uint32_t clip_block_max(uint32_t v, uint32_t (&buf)[2][8], int& par) {
+    v = __reduce_max_sync(0xffffffffu, v);
+    if ((threadIdx.x & 31) == 0) buf[par][threadIdx.x >> 5] = v;
+    __syncthreads();
+    uint32_t r = buf[par][0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) r = max(r, buf[par][i]);
+    par ^= 1;
+    return r;
+}
+__device__ __forceinline__ uint32_t clip_block_sum(uint32_t v, uint32_t (&buf)[2][8], int& par) {
+    v = __reduce_add_sync(0xffffffffu, v);
+    if ((threadIdx.x & 31) == 0) buf[par][threadIdx.x >> 5] = v;
+    __syncthreads();
+    uint32_t r = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r += buf[par][i];
+    par ^= 1;
+    return r;
+}
+__device__ __forceinline__ uint32_t mag_bits(float x) { return __float_as_uint(x) & 0x7FFFFFFFu; }
+
+// The order statistics r0 = k0-th and r1 = (k0+1)-th smallest magnitude of a
+// slab of `len` values held by one warp.  `each(f)` calls f(u, q) for every
+// valid magnitude pattern u the lane holds, q in [0, 4) spreading them over
+// four independent accumulators (one chain of dependent max / add operations
+// per accumulator instead of one for the whole lane).
+template <typename Each>
+__device__ __forceinline__ void warp_select2(int len, int k0, Each&& each, uint32_t& r0, uint32_t& r1) {
+    r0 = r1 = 0;
+    const int j = len - 1 - k0;
+    if (j <= kClipTop) {
+        // the maximum, then per step one pass for both the count of the
+        // current value m and the largest magnitude below it
+        uint32_t lm[4] = {0, 0, 0, 0};
+        each([&](uint32_t u, int q) { lm[q] = max(lm[q], u); });
+        uint32_t m = __reduce_max_sync(0xffffffffu, max(max(lm[0], lm[1]), max(lm[2], lm[3])));
+        int above = 0;  // elements above m
+        uint32_t prev = 0;
+        for (int it = 0; it <= kClipTop; ++it) {
+            uint32_t lc[4] = {0, 0, 0, 0}, lb[4] = {0, 0, 0, 0};
+            each([&](uint32_t u, int q) {
+                lc[q] += u == m;
+                if (u < m) lb[q] = max(lb[q], u);
+            });
+            const int c = static_cast<int>(__reduce_add_sync(0xffffffffu, (lc[0] + lc[1]) + (lc[2] + lc[3])));
+            const uint32_t below = __reduce_max_sync(0xffffffffu, max(max(lb[0], lb[1]), max(lb[2], lb[3])));
+            if (j < above + c) {
+                r0 = m;
+                r1 = (j >= 1 && j - 1 < above) ? prev : m;
+                return;
+            }
+            above += c;
+            prev = m;
+            m = below;
+        }
+    } else {
+        for (int b = 30; b >= 0; --b) {
+            const uint32_t t0 = r0 | (1u << b), t1 = r1 | (1u << b);
+            uint32_t c0[4] = {0, 0, 0, 0}, c1[4] = {0, 0, 0, 0};
+            each([&](uint32_t u, int q) {
+                c0[q] += u < t0;
+                c1[q] += u < t1;
+            });
+            const uint32_t n0 = __reduce_add_sync(0xffffffffu, (c0[0] + c0[1]) + (c0[2] + c0[3]));
+            const uint32_t n1 = __reduce_add_sync(0xffffffffu, (c1[0] + c1[1]) + (c1[2] + c1[3]));
+            if (static_cast<int>(n0) <= k0) r0 = t0;
+            if (static_cast<int>(n1) <= k0 + 1) r1 = t1;
+        }
+    }
+}
+
+// Per channel, rows of K <= 32 * VPL weights with K % 4 == 0 (16-byte aligned
+// rows): one warp per output row, the row in registers (lane l holds the
+// 16-byte chunks l, l + 32, ...), every reduction a warp redux -- no block
+// barriers, and eight rows per 256-thread CTA in flight at once.
+template <int VPL>
+__global__ void __launch_bounds__(256) k_quantize_weight_pc_clip_warp(const float* __restrict__ W, int64_t N, int K,
+                                                                      int k0, float t, int8_t* __restrict__ w,
+                                                                      float* __restrict__ sw) {
+    static_assert(VPL % 4 == 0, "whole 16-byte chunks per lane");
+    pdl_wait();
+    pdl_trigger();
+    const int64_t n = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (n >= N) return;  // whole warps
+    const float* wr = W + n * K;
+    float x[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL / 4; ++i) {
+        const int k = 4 * (lane + 32 * i);
+        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (k < K) v = __ldg(reinterpret_cast<const float4*>(wr + k));
+        x[4 * i] = v.x;
+        x[4 * i + 1] = v.y;
+        x[4 * i + 2] = v.z;
+        x[4 * i + 3] = v.w;
+    }
+    float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int i = 0; i < VPL / 4; ++i)
+        if (4 * (lane + 32 * i) < K)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) am[c] = fmaxf(am[c], fabsf(x[4 * i + c]));
+    const float amax = warp_max(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])));
+    auto each = [&](auto&& f) {
+#pragma unroll
+        for (int i = 0; i < VPL / 4; ++i)
+            if (4 * (lane + 32 * i) < K)  // K % 4 == 0: a chunk is wholly inside the row or wholly past it
+#pragma unroll
+                for (int c = 0; c < 4; ++c) f(mag_bits(x[4 * i + c]), c);
+    };
+    uint32_t r0, r1;
+    warp_select2(K, k0, each, r0, r1);
+    const float c = clip_value(r0, r1, t != 0.0f && k0 + 1 < K, t, amax);
+    const float s = act_scale(c);
+    const float r = __frcp_rn(s);
+    if (lane == 0) sw[n] = s;
+#pragma unroll
+    for (int i = 0; i < VPL / 4; ++i) {
+        const int k = 4 * (lane + 32 * i);
+        if (k < K) {
+            const uint32_t b0 = static_cast<uint8_t>(clip_code_fast(x[4 * i], s, r));
+            const uint32_t b1 = static_cast<uint8_t>(clip_code_fast(x[4 * i + 1], s, r));
+            const uint32_t b2 = static_cast<uint8_t>(clip_code_fast(x[4 * i + 2], s, r));
+            const uint32_t b3 = static_cast<uint8_t>(clip_code_fast(x[4 * i + 3], s, r));
+            *reinterpret_cast<uint32_t*>(w + n * K + k) = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        }
+    }
+}
+
+// This thread's elements of a row (k = tid, tid + 256, ...): held in
+// registers when VPT > 0 (K <= 256 * VPT), else read through L1 each time.
+template <int VPT, typename F>
+__device__ __forceinline__ void clip_each(const float* wr, int K, const float (&x)[VPT > 0 ? VPT : 1], F&& f) {
+    if constexpr (VPT > 0) {
+#pragma unroll
+        for (int i = 0; i < VPT; ++i)
+            if (static_cast<int>(threadIdx.x) + 256 * i < K) f(x[i]);
+    } else {
+        for (int k = threadIdx.x; k < K; k += 256) f(__ldg(wr + k));
+    }
+}
 
 // Per channel: one CTA of 256 threads per output row.
+template <int VPT>
 __global__ void __launch_bounds__(256) k_quantize_weight_pc_clip(const float* __restrict__ W, int K, int k0,
                                                                  float t, int8_t* __restrict__ w,
                                                                  float* __restrict__ sw) {
+    __shared__ uint32_t buf[2][8];
     __shared__ int red[2][8][2];
     __shared__ float redm[8];
     pdl_wait();
@@ -414,47 +596,87 @@ __global__ void __launch_bounds__(256) k_quantize_weight_pc_clip(const float* __
     const int64_t n = blockIdx.x;
     const float* wr = W + n * K;
     const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    float x[VPT > 0 ? VPT : 1];
+    if constexpr (VPT > 0) {
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) x[i] = tid + 256 * i < K ? wr[tid + 256 * i] : 0.0f;
+    }
     float amax = 0.0f;
-    for (int k = tid; k < K; k += 256) amax = fmaxf(amax, fabsf(wr[k]));
+    clip_each<VPT>(wr, K, x, [&](float v) { amax = fmaxf(amax, fabsf(v)); });
     amax = warp_max(amax);
     if (lane == 0) redm[wp] = amax;
     __syncthreads();
     amax = redm[0];
     for (int i = 1; i < 8; ++i) amax = fmaxf(amax, redm[i]);
     uint32_t r0 = 0, r1 = 0;
-    for (int b = 30; b >= 0; --b) {
-        const uint32_t t0 = r0 | (1u << b), t1 = r1 | (1u << b);
-        int c0 = 0, c1 = 0;
-        for (int k = tid; k < K; k += 256) {
-            const uint32_t u = __float_as_uint(fabsf(__ldg(wr + k)));
-            c0 += u < t0;
-            c1 += u < t1;
+    const int j = K - 1 - k0;
+    if (j <= kClipTop) {
+        int par = 0, above = 0;  // elements at or above the current value
+        uint32_t thr = 0xFFFFFFFFu, prev = 0;
+        for (int it = 0; it <= kClipTop; ++it) {
+            uint32_t lm = 0;
+            clip_each<VPT>(wr, K, x, [&](float v) {
+                const uint32_t u = mag_bits(v);
+                if (u < thr) lm = max(lm, u);
+            });
+            const uint32_t m = clip_block_max(lm, buf, par);
+            uint32_t lc = 0;
+            clip_each<VPT>(wr, K, x, [&](float v) { lc += mag_bits(v) == m; });
+            const int c = static_cast<int>(clip_block_sum(lc, buf, par));
+            if (j < above + c) {
+                r0 = m;
+                r1 = (j >= 1 && j - 1 < above) ? prev : m;
+                break;
+            }
+            above += c;
+            prev = m;
+            thr = m;
         }
-        c0 = __reduce_add_sync(0xffffffffu, c0);
-        c1 = __reduce_add_sync(0xffffffffu, c1);
-        // two buffers: a pass's writes never meet the previous pass's reads
-        int(*rb)[2] = red[b & 1];
-        if (lane == 0) {
-            rb[wp][0] = c0;
-            rb[wp][1] = c1;
+    } else {
+        for (int b = 30; b >= 0; --b) {
+            const uint32_t t0 = r0 | (1u << b), t1 = r1 | (1u << b);
+            int c0 = 0, c1 = 0;
+            clip_each<VPT>(wr, K, x, [&](float v) {
+                const uint32_t u = mag_bits(v);
+                c0 += u < t0;
+                c1 += u < t1;
+            });
+            c0 = __reduce_add_sync(0xffffffffu, c0);
+            c1 = __reduce_add_sync(0xffffffffu, c1);
+            // two buffers: a pass's writes never meet the previous pass's reads
+            int(*rb)[2] = red[b & 1];
+            if (lane == 0) {
+                rb[wp][0] = c0;
+                rb[wp][1] = c1;
+            }
+            __syncthreads();
+            c0 = c1 = 0;
+            for (int i = 0; i < 8; ++i) {
+                c0 += rb[i][0];
+                c1 += rb[i][1];
+            }
+            if (c0 <= k0) r0 = t0;
+            if (c1 <= k0 + 1) r1 = t1;
         }
-        __syncthreads();
-        c0 = c1 = 0;
-        for (int i = 0; i < 8; ++i) {
-            c0 += rb[i][0];
-            c1 += rb[i][1];
-        }
-        if (c0 <= k0) r0 = t0;
-        if (c1 <= k0 + 1) r1 = t1;
     }
     const float c = clip_value(r0, r1, t != 0.0f && k0 + 1 < K, t, amax);
     const float s = act_scale(c);
+    const float rs = __frcp_rn(s);
     if (tid == 0) sw[n] = s;
-    for (int k = tid; k < K; k += 256) w[n * K + k] = clip_code(wr[k], s);
+    if constexpr (VPT > 0) {
+#pragma unroll
+        for (int i = 0; i < VPT; ++i)
+            if (tid + 256 * i < K) w[n * K + tid + 256 * i] = clip_code_fast(x[i], s, rs);
+    } else {
+        for (int k = tid; k < K; k += 256) w[n * K + k] = clip_code_fast(wr[k], s, rs);
+    }
 }
 
-// Per group: one warp per (row n, group g), the group's gs = 32 * VPL
-// magnitudes held in registers; scales group-major [G][N].
+// Per group: one warp per GPW consecutive groups of a row (group g of row n
+// and the next ones), each group's gs = 32 * VPL magnitudes held in
+// registers; all the groups' loads go out before the first selection, so a
+// warp has GPW * gs * 4 bytes in flight.  Scales group-major [G][N].
+constexpr int kClipGroupsPerWarp = 4;
 template <int VPL>
 __global__ void __launch_bounds__(256) k_quantize_weight_pg_clip(const float* __restrict__ W, int64_t N, int K,
                                                                  int k0, float t, int8_t* __restrict__ out,
@@ -462,50 +684,63 @@ __global__ void __launch_bounds__(256) k_quantize_weight_pg_clip(const float* __
     pdl_wait();
     pdl_trigger();
     constexpr int GS = 32 * VPL;
+    constexpr int GPW = kClipGroupsPerWarp;
     const int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     const int G = K / GS;
-    if (item >= N * G) return;  // whole warps
-    const int64_t n = item / G;
-    const int g = static_cast<int>(item % G);
-    const float* wg = W + n * K + static_cast<int64_t>(g) * GS;
-    float x[VPL];
-    uint32_t u[VPL];
-    float amax = 0.0f;
+    const int wpr = (G + GPW - 1) / GPW;  // warps per row
+    if (item >= N * wpr) return;  // whole warps
+    const int64_t n = item / wpr;
+    const int g0 = static_cast<int>(item % wpr) * GPW;
+    float x[GPW][VPL];
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-        x[j] = wg[lane + 32 * j];
-        u[j] = __float_as_uint(fabsf(x[j]));
-        amax = fmaxf(amax, fabsf(x[j]));
-    }
-    amax = warp_max(amax);
-    uint32_t r0 = 0, r1 = 0;
-    for (int b = 30; b >= 0; --b) {
-        const uint32_t t0 = r0 | (1u << b), t1 = r1 | (1u << b);
-        int c0 = 0, c1 = 0;
+    for (int h = 0; h < GPW; ++h)
+        if (g0 + h < G) {
+            const float* wg = W + n * K + static_cast<int64_t>(g0 + h) * GS;
 #pragma unroll
-        for (int j = 0; j < VPL; ++j) {
-            c0 += u[j] < t0;
-            c1 += u[j] < t1;
+            for (int i = 0; i < VPL; ++i) x[h][i] = wg[lane + 32 * i];
         }
-        c0 = __reduce_add_sync(0xffffffffu, c0);
-        c1 = __reduce_add_sync(0xffffffffu, c1);
-        if (c0 <= k0) r0 = t0;
-        if (c1 <= k0 + 1) r1 = t1;
-    }
-    const float c = clip_value(r0, r1, t != 0.0f && k0 + 1 < GS, t, amax);
-    const float s = act_scale(c);
-    if (lane == 0) sw[static_cast<int64_t>(g) * N + n] = s;
-    int8_t* w = out + n * K + static_cast<int64_t>(g) * GS;
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) w[lane + 32 * j] = clip_code(x[j], s);
+    for (int h = 0; h < GPW; ++h) {
+        const int g = g0 + h;
+        if (g >= G) break;  // warp-uniform
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) amax = fmaxf(amax, fabsf(x[h][i]));
+        amax = warp_max(amax);
+        auto each = [&](auto&& f) {
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) f(mag_bits(x[h][i]), i & 3);
+        };
+        uint32_t r0, r1;
+        warp_select2(GS, k0, each, r0, r1);
+        const float c = clip_value(r0, r1, t != 0.0f && k0 + 1 < GS, t, amax);
+        const float s = act_scale(c);
+        const float rs = __frcp_rn(s);
+        if (lane == 0) sw[static_cast<int64_t>(g) * N + n] = s;
+        int8_t* w = out + n * K + static_cast<int64_t>(g) * GS;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) w[lane + 32 * i] = clip_code_fast(x[h][i], s, rs);
+    }
 }
 
 cudaError_t launch_quantize_weight_clip(const float* W, int64_t N, int K, int gs, int k0, float t, int8_t* out,
                                         float* sw, cudaStream_t st) {
+    const bool vec = K % 4 == 0 && (reinterpret_cast<uintptr_t>(W) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(out) & 3) == 0;
+    if (gs == 0 && vec && K <= 32 * 128) {
+        const unsigned grid = static_cast<unsigned>((N + 7) / 8);  // a warp per row
+        if (K <= 32 * 64)
+            return launch_pdl(k_quantize_weight_pc_clip_warp<64>, grid, 256, 0, st, W, N, K, k0, t, out, sw);
+        if (K <= 32 * 80)
+            return launch_pdl(k_quantize_weight_pc_clip_warp<80>, grid, 256, 0, st, W, N, K, k0, t, out, sw);
+        return launch_pdl(k_quantize_weight_pc_clip_warp<128>, grid, 256, 0, st, W, N, K, k0, t, out, sw);
+    }
+    if (gs == 0 && K <= 256 * 16)
+        return launch_pdl(k_quantize_weight_pc_clip<16>, static_cast<unsigned>(N), 256, 0, st, W, K, k0, t, out, sw);
     if (gs == 0)
-        return launch_pdl(k_quantize_weight_pc_clip, static_cast<unsigned>(N), 256, 0, st, W, K, k0, t, out, sw);
-    const int64_t items = N * (K / gs);
+        return launch_pdl(k_quantize_weight_pc_clip<0>, static_cast<unsigned>(N), 256, 0, st, W, K, k0, t, out, sw);
+    const int64_t items = N * ((K / gs + kClipGroupsPerWarp - 1) / kClipGroupsPerWarp);  // warps
     const unsigned grid = static_cast<unsigned>((items + 7) / 8);
     if (gs == 64) return launch_pdl(k_quantize_weight_pg_clip<2>, grid, 256, 0, st, W, N, K, k0, t, out, sw);
     if (gs == 128) return launch_pdl(k_quantize_weight_pg_clip<4>, grid, 256, 0, st, W, N, K, k0, t, out, sw);
