@@ -25,12 +25,19 @@ def _device():
     cider.cider_device_status()
 
 
+@pytest.mark.parametrize("kernel", [0, 1])
 @pytest.mark.parametrize("M", [1, 2, 3, 4])
 @pytest.mark.parametrize("N,K", [(10240, 2560), (2560, 10240), (264, 1040), (8, 16)])
-def test_w8a16_mv(M, N, K):
+def test_w8a16_mv(kernel, M, N, K):
+    """The automatic choice (the one-shot kernel where its plan fits) and the
+    register ring, forced, on the same shapes."""
     x = act(M, K, seed=M + N + K)
     qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed=N + K))
-    y = cider.cider_w8a16_mv_pc(dev_bits(x, oracle.F16), dev(qw), dev(sw))
+    cider.cider_test_set_small_m_kernel(kernel)
+    try:
+        y = cider.cider_w8a16_mv_pc(dev_bits(x, oracle.F16), dev(qw), dev(sw))
+    finally:
+        cider.cider_test_set_small_m_kernel(0)
     check_y(y, oracle.w8a16_linear_pc(x, qw, sw), oracle.F16)
 
 
