@@ -118,7 +118,7 @@ def test_quantize_weight_pc_bitexact(N, K):
 
 
 @pytest.mark.parametrize("gs", [64, 128])
-@pytest.mark.parametrize("N,K", [(8, 256), (136, 2560)])
+@pytest.mark.parametrize("N,K", [(8, 256), (136, 2560), (5, 1920), (3, 128 * 7), (2560, 10240)])
 def test_quantize_weight_pg_bitexact(N, K, gs):
     W = synth.weights(N, K, seed=3 * N + K)
     w_ref, s_ref = oracle.quantize_weight_pg(W, gs)
@@ -128,7 +128,7 @@ def test_quantize_weight_pg_bitexact(N, K, gs):
 
 
 @pytest.mark.parametrize("gs", [64, 128])
-@pytest.mark.parametrize("N,K", [(8, 128), (136, 4096)])
+@pytest.mark.parametrize("N,K", [(8, 128), (136, 4096), (5, 640), (12288, 4096)])
 def test_pack_weight_int4_bitexact(N, K, gs):
     W = synth.weights(N, K, seed=5 * N + K)
     W[0, :gs] = 0.0  # an all-zero group

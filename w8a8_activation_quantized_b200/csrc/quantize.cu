@@ -331,38 +331,67 @@ __global__ void __launch_bounds__(256) k_pack_weight_int4_pc(const float* __rest
     }
 }
 
-// Per group (INT8 or INT4): one warp per (row n, group g); scales group-major [G][N].
-template <bool INT4>
+// Per group (INT8 or INT4): one warp per kWeightGroupsPerWarp consecutive
+// groups of a row.  Lane l holds elements 2l and 2l + 1 of every 64-wide part
+// of a group (2 * PPL values, gs = 64 * PPL), so its INT4 byte packs its own
+// pair; all the groups' loads go out before the first maximum, so a warp has
+// a few KB in flight.  Scales group-major [G][N].
+constexpr int kWeightGroupsPerWarp = 4;
+template <bool INT4, int PPL>
 __global__ void __launch_bounds__(256) k_quantize_weight_group(const float* __restrict__ W,
-                                                               int64_t N, int K, int gs,
+                                                               int64_t N, int K,
                                                                void* __restrict__ out,
                                                                float* __restrict__ sw) {
     pdl_wait();
     pdl_trigger();
+    constexpr int GS = 64 * PPL;
+    constexpr int GPW = kWeightGroupsPerWarp;
     const int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    const int G = K / gs;
-    if (item >= N * G) return;
-    const int64_t n = item / G;
-    const int g = static_cast<int>(item % G);
-    const float* wg = W + n * K + static_cast<int64_t>(g) * gs;
-    float amax = 0.0f;
-    for (int k = lane; k < gs; k += 32) amax = fmaxf(amax, fabsf(wg[k]));
-    amax = warp_max(amax);
-    const float s = INT4 ? __fdiv_rn(amax, 7.0f) : act_scale(amax);
-    if (lane == 0) sw[static_cast<int64_t>(g) * N + n] = s;
-    if (!INT4) {
-        int8_t* w = static_cast<int8_t*>(out) + n * K + static_cast<int64_t>(g) * gs;
-        for (int k = lane; k < gs; k += 32) w[k] = static_cast<int8_t>(quant_code(wg[k], s));
-    } else {
-        uint8_t* p = static_cast<uint8_t*>(out) + n * (K / 2) + static_cast<int64_t>(g) * (gs / 2);
-        for (int j = lane; j < gs / 2; j += 32) {
-            int c0 = 0, c1 = 0;
-            if (s != 0.0f) {
-                c0 = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(wg[2 * j], s)), -8.0f), 7.0f));
-                c1 = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(wg[2 * j + 1], s)), -8.0f), 7.0f));
+    const int G = K / GS;
+    const int wpr = (G + GPW - 1) / GPW;  // warps per row
+    if (item >= N * wpr) return;  // whole warps
+    const int64_t n = item / wpr;
+    const int g0 = static_cast<int>(item % wpr) * GPW;
+    float x[GPW][2 * PPL];
+#pragma unroll
+    for (int h = 0; h < GPW; ++h)
+        if (g0 + h < G) {
+            const float* wg = W + n * K + static_cast<int64_t>(g0 + h) * GS;
+#pragma unroll
+            for (int i = 0; i < PPL; ++i) {
+                x[h][2 * i] = wg[2 * lane + 64 * i];
+                x[h][2 * i + 1] = wg[2 * lane + 1 + 64 * i];
             }
-            p[j] = static_cast<uint8_t>((c0 + 8) | ((c1 + 8) << 4));
+        }
+#pragma unroll
+    for (int h = 0; h < GPW; ++h) {
+        const int g = g0 + h;
+        if (g >= G) break;  // warp-uniform
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 2 * PPL; ++i) amax = fmaxf(amax, fabsf(x[h][i]));
+        amax = warp_max(amax);
+        const float s = INT4 ? __fdiv_rn(amax, 7.0f) : act_scale(amax);
+        if (lane == 0) sw[static_cast<int64_t>(g) * N + n] = s;
+        if (!INT4) {
+            int8_t* w = static_cast<int8_t*>(out) + n * K + static_cast<int64_t>(g) * GS;
+#pragma unroll
+            for (int i = 0; i < PPL; ++i) {
+                w[2 * lane + 64 * i] = static_cast<int8_t>(quant_code(x[h][2 * i], s));
+                w[2 * lane + 1 + 64 * i] = static_cast<int8_t>(quant_code(x[h][2 * i + 1], s));
+            }
+        } else {
+            uint8_t* p = static_cast<uint8_t*>(out) + n * (K / 2) + static_cast<int64_t>(g) * (GS / 2);
+#pragma unroll
+            for (int i = 0; i < PPL; ++i) {
+                int c0 = 0, c1 = 0;
+                if (s != 0.0f) {
+                    c0 = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(x[h][2 * i], s)), -8.0f), 7.0f));
+                    c1 = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(x[h][2 * i + 1], s)), -8.0f), 7.0f));
+                }
+                p[lane + 32 * i] = static_cast<uint8_t>((c0 + 8) | ((c1 + 8) << 4));
+            }
         }
     }
 }
@@ -373,10 +402,14 @@ cudaError_t launch_quantize_weight(int mode, const float* W, int64_t N, int K, i
         return launch_pdl(k_quantize_weight_pc, static_cast<unsigned>(N), 256, 0, st, W, K, static_cast<int8_t*>(out), sw);
     if (mode == 3)
         return launch_pdl(k_pack_weight_int4_pc, static_cast<unsigned>(N), 256, 0, st, W, K, static_cast<uint8_t*>(out), sw);
-    const int64_t items = N * (K / gs);
-    const unsigned grid = static_cast<unsigned>((items + 7) / 8);
-    if (mode == 1) return launch_pdl(k_quantize_weight_group<false>, grid, 256, 0, st, W, N, K, gs, out, sw);
-    return launch_pdl(k_quantize_weight_group<true>, grid, 256, 0, st, W, N, K, gs, out, sw);
+    const int64_t warps = N * ((K / gs + kWeightGroupsPerWarp - 1) / kWeightGroupsPerWarp);
+    const unsigned grid = static_cast<unsigned>((warps + 7) / 8);
+    if (gs != 64 && gs != 128) return cudaErrorInvalidValue;  // rejected by the host checks first
+    if (mode == 1)
+        return gs == 64 ? launch_pdl(k_quantize_weight_group<false, 1>, grid, 256, 0, st, W, N, K, out, sw)
+                        : launch_pdl(k_quantize_weight_group<false, 2>, grid, 256, 0, st, W, N, K, out, sw);
+    return gs == 64 ? launch_pdl(k_quantize_weight_group<true, 1>, grid, 256, 0, st, W, N, K, out, sw)
+                    : launch_pdl(k_quantize_weight_group<true, 2>, grid, 256, 0, st, W, N, K, out, sw);
 }
 
 // ---- percentile-clipped weight scales (clip_percentile) ----------------------
