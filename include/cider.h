@@ -346,10 +346,11 @@ CIDER_API cider_status_t cider_test_set_sdpa_kernel(int kernel);
  * kernel), 1 = the register-ring kernel, 2 = the bulk-staged kernel with the
  * whole shared memory, 3 = the bulk-staged kernel within half of it, 4 = the
  * one-shot kernel where its plan fits.  Shapes a selected kernel's plan
- * cannot hold take the register-ring kernel.  The W8A16 products follow the
- * same rule, with the one-shot kernel in its W8A16 form (x unquantized in
- * shared memory).  Lets tests and measurements compare the kernels on the
- * same shapes. */
+ * cannot hold take the register-ring kernel.  The W8A16 products: 0 takes
+ * the one-shot form (x unquantized in shared memory) for the per-group
+ * product and the register ring for the per-channel one, 4 the one-shot form
+ * for both.  Lets tests and measurements compare the kernels on the same
+ * shapes. */
 CIDER_API cider_status_t cider_test_set_small_m_kernel(int kernel);
 /* Selects, for later calls (process-wide), how the per-channel linear
  * (cider_w8a8_linear_pc and the workspace-free form) quantizes its

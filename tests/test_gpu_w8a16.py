@@ -29,8 +29,9 @@ def _device():
 @pytest.mark.parametrize("M", [1, 2, 3, 4])
 @pytest.mark.parametrize("N,K", [(10240, 2560), (2560, 10240), (264, 1040), (8, 16)])
 def test_w8a16_mv(kernel, M, N, K):
-    """The automatic choice (the one-shot kernel where its plan fits) and the
-    register ring, forced, on the same shapes."""
+    """The automatic choice (the register ring per channel) and the ring
+    forced, on the same shapes; the one-shot form is forced in the tests
+    below."""
     x = act(M, K, seed=M + N + K)
     qw, sw = oracle.quantize_weight_pc(synth.weights(N, K, seed=N + K))
     cider.cider_test_set_small_m_kernel(kernel)

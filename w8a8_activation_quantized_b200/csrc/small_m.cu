@@ -1312,7 +1312,7 @@ static cudaError_t launch_small_m_v(const void* x, int xdt, int M, int K, const 
     const int sel = g_small_kernel.load();
     ShotGeom sg;
     int sgrid = 0, ssmem = 0;
-    if ((sel == 0 || sel == 4) && shot_plan(M, K, N, PG, W4, gs, num_sms, sg, sgrid, ssmem)) {
+    if (((sel == 0 && gs > 0) || sel == 4) && shot_plan(M, K, N, PG, W4, gs, num_sms, sg, sgrid, ssmem)) {
         if (xdt == 1)
             return launch_shot_m<__nv_bfloat16, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, sg, sgrid, ssmem, status, st);
         return launch_shot_m<__half, PG, W4>(x, M, K, w, sw, N, gs, y, ydt, sg, sgrid, ssmem, status, st);
@@ -1401,16 +1401,15 @@ static cudaError_t launch_mv_shot(const void* x, int M, int K, const int8_t* w, 
 
 cudaError_t launch_mv_w8a16(const void* x, int xdt, int M, int K, const int8_t* w, const float* sw, int N, int gs,
                             void* y, int ydt, int num_sms, unsigned* status, cudaStream_t st) {
-    // The one-shot kernel (A16 mode) where its plan fits, else the register
-    // ring.  Measured on B200 at M = 1: per group (N = 2560, K = 10240)
-    // 11.1 / 11.7 us at gs = 128 / 64 against 14.7 / 15.0 us for the ring;
-    // per channel (N = 10240, K = 2560) 9.6 against 9.7 us, since the
-    // one-shot kernel prefetches its first weight pieces before the
-    // grid-dependency wait (before that, 10.1 against 9.95 us: it widens the
-    // activations for every chunk where the ring stages them once).  The
-    // test switch's 1 forces the ring, 4 the one-shot kernel; the
-    // bulk-staged kernel (11.3 us per channel) runs when the switch selects
-    // it and its plan fits.
+    // Per group, the one-shot kernel (A16 mode) where its plan fits (M = 1,
+    // N = 2560, K = 10240 on B200: 11.1 / 11.7 us at gs = 128 / 64 against
+    // 14.7 / 15.0 us for the register ring); per channel the register ring,
+    // whose fp32 activation pairs are staged once (N = 10240, K = 2560: the
+    // one-shot kernel, which widens the activations for every chunk, was
+    // 1% faster timed alone but 10% slower within the full set of bench
+    // rows, 10.5 against 9.6 us).  The test switch's 1 forces the ring, 4
+    // the one-shot kernel for both; the bulk-staged kernel (11.3 us per
+    // channel) runs when the switch selects it and its plan fits.
     BulkGeom geo;
     int grid = 0;
     const int sel = g_small_kernel.load();
