@@ -117,6 +117,26 @@ def test_quantize_weight_pc_bitexact(N, K):
     np.testing.assert_array_equal(w.cpu().numpy(), w_ref)
 
 
+@pytest.mark.parametrize("offset", [0, 1])
+@pytest.mark.parametrize("N,K", [(37, 2048), (9, 2560), (7, 1020), (5, 2564), (3, 12), (10240, 2560)])
+def test_quantize_weight_pc_widths_and_offsets(N, K, offset):
+    """The per-channel INT8 quantizer and INT4 packer on several row widths,
+    on aligned storage and 4 bytes past a 16-byte boundary, bit for bit."""
+    W = synth.weights(N, K, seed=N * 7 + K)
+    W[0, : min(K, 64)] = 0.0  # a partly zero row
+    flat = torch.zeros(W.size + offset, dtype=torch.float32, device="cuda")
+    flat[offset:] = torch.from_numpy(W.ravel()).cuda()
+    Wd = flat[offset:].view(N, K)
+    w_ref, s_ref = oracle.quantize_weight_pc(W)
+    w, s = cider.cider_quantize_weight_pc(Wd)
+    np.testing.assert_array_equal(s.cpu().numpy(), s_ref)
+    np.testing.assert_array_equal(w.cpu().numpy(), w_ref)
+    p_ref, s4_ref = oracle.quantize_weight_int4_pc(W)
+    p, s4 = cider.cider_pack_weight_int4_pc(Wd)
+    np.testing.assert_array_equal(s4.cpu().numpy().view(np.uint32), s4_ref.view(np.uint32))
+    np.testing.assert_array_equal(p.cpu().numpy(), p_ref)
+
+
 @pytest.mark.parametrize("gs", [64, 128])
 @pytest.mark.parametrize("N,K", [(8, 256), (136, 2560), (5, 1920), (3, 128 * 7), (2560, 10240)])
 def test_quantize_weight_pg_bitexact(N, K, gs):
