@@ -249,6 +249,16 @@ __global__ void __launch_bounds__(kMergeThreads) k_sdpa_decode_merge(const float
     pdl_trigger();
     const int h = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
     const float* ph = part + static_cast<int64_t>(h) * chunks * kSdpaPartStride;
+    // The o vectors of each warp's first four chunks are requested now, beside
+    // the chunk maxima, so the weighted sum below does not wait for another
+    // L2 round trip once the maximum is known (the sums keep their order).
+    float4 o_first[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int cj = w + j * kMergeWarps;
+        o_first[j] = cj < chunks ? __ldg(reinterpret_cast<const float4*>(ph + cj * kSdpaPartStride) + lane)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float M = -INFINITY;
     for (int c = t; c < chunks; c += kMergeThreads) M = fmaxf(M, __ldg(ph + c * kSdpaPartStride + D));
     M = warp_reduce_max(M);
@@ -271,6 +281,29 @@ __global__ void __launch_bounds__(kMergeThreads) k_sdpa_decode_merge(const float
     for (int i = 0; i < kMergeWarps; ++i) L += s_red[1][i];
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     int c = w;
+    if (c + 3 * kMergeWarps < chunks) {  // the first four chunks, already in registers
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float sc = s_sc[c + j * kMergeWarps];
+            acc.x = fmaf(o_first[j].x, sc, acc.x);
+            acc.y = fmaf(o_first[j].y, sc, acc.y);
+            acc.z = fmaf(o_first[j].z, sc, acc.z);
+            acc.w = fmaf(o_first[j].w, sc, acc.w);
+        }
+        c += 4 * kMergeWarps;
+    } else {  // fewer than four chunks for this warp: the tail loop below, from registers
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (c + j * kMergeWarps < chunks) {
+                const float sc = s_sc[c + j * kMergeWarps];
+                acc.x = fmaf(o_first[j].x, sc, acc.x);
+                acc.y = fmaf(o_first[j].y, sc, acc.y);
+                acc.z = fmaf(o_first[j].z, sc, acc.z);
+                acc.w = fmaf(o_first[j].w, sc, acc.w);
+            }
+        }
+        c = chunks;  // all of this warp's chunks are added
+    }
     for (; c + 3 * kMergeWarps < chunks; c += 4 * kMergeWarps) {  // four chunks' loads in flight
         float4 o[4];
 #pragma unroll
